@@ -1,0 +1,346 @@
+/*
+ * FP64 CPU oracle for the fine stage of Video Sparse Attention (VSA).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may load or call
+ * this file: it is used by tests/, by the smoke check in __graft_entry__.py
+ * and by the CPU-baseline leg of bench.py.  It shares no code, header,
+ * table or helper with the CUDA library in video_block_sparse_b200/csrc.
+ *
+ * It is plain and slow on purpose: every result is the textbook definition
+ * written out in double precision, one element at a time, so that a reader
+ * can hold it against the pages by eye.
+ *
+ * Sources (titles of the pages this restates):
+ *  - "baseten-admin/wan2.2_production_values" (dataset card), sections
+ *    "Shapes" and "Operator contract": cube-major 4x4x4 tiling, 64-token
+ *    cubes, S_padded = 64 * Nq, out = softmax(q k_sel^T / sqrt(D)) v_sel,
+ *    topk_idx names the selected KV cubes per (batch, head, query cube),
+ *    vbs[c] keeps only the first vbs[c] of the 64 tokens of cube c.
+ *  - "align VisualGen VSA with block-sparse FMHA" (TensorRT-LLM PR #7),
+ *    review excerpts: cube means are sums over the valid tokens divided by
+ *    the valid count and cast back to the tiled dtype; untiling is an index
+ *    gather.
+ *  - "Video Sparse Attention Runner" (TensorRT-Edge-LLM API docs): block
+ *    means of K rounded to bf16 before they are used for routing, query
+ *    blocks routed by a centroid score.
+ *
+ * Readings where the pages leave a step open (each is listed in the design doc):
+ *  - inside a cube the real tokens come first, in local (t,h,w) row-major
+ *    order over the cube's real extent, then zero pads up to 64;
+ *  - routing scores are the dot products of bf16 cube means (sequential
+ *    FP64 sum, IEEE divide, RNE to bf16), accumulated sequentially in FP64
+ *    over d; top-k ordered by score descending, index ascending, NaN as -inf;
+ *  - a row whose selected tokens are all masked gives out = 0, lse = -inf;
+ *  - lse is the natural-log log-sum-exp of the scaled logits.
+ *
+ * Parity pins for every function live in tests/test_oracle_pins.py.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <float.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_ARG -1
+#define ORACLE_ERR_NOMEM -2
+
+/* ---- bf16 <-> double -------------------------------------------------- */
+
+/* A bf16 value is the upper half of an IEEE binary32 word. Widening is exact. */
+static double bf16_bits_to_f64(uint16_t h)
+{
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Round a double to the nearest bf16 value, ties to even, in one step
+ * (no intermediate rounding to binary32).  bf16 keeps 8 significant bits
+ * and the binary32 exponent range (normal from 2^-126, subnormal step
+ * 2^-133, largest finite (2 - 2^-7) * 2^127). */
+static uint16_t f64_to_bf16_bits(double x)
+{
+    if (isnan(x)) return (uint16_t)0x7FC0;
+    if (isinf(x)) return (uint16_t)(x > 0 ? 0x7F80 : 0xFF80);
+    if (x == 0.0) return (uint16_t)(signbit(x) ? 0x8000 : 0x0000);
+    double ax = fabs(x);
+    int e;
+    (void)frexp(ax, &e); /* ax = f * 2^e, f in [0.5, 1) -> leading bit weight 2^(e-1) */
+    int ulp_exp = (e - 1) - 7; /* 8 significant bits */
+    if (ulp_exp < -133) ulp_exp = -133; /* subnormal spacing */
+    double scaled = ldexp(ax, -ulp_exp); /* exact: power-of-two scaling */
+    double r = nearbyint(scaled); /* current rounding mode: to nearest, ties to even */
+    double y = ldexp(r, ulp_exp);
+    const double bf16_max = ldexp(255.0, 127 - 7); /* (2 - 2^-7) * 2^127 */
+    uint16_t sign = signbit(x) ? 0x8000 : 0x0000;
+    if (y > bf16_max) return (uint16_t)(sign | 0x7F80);
+    float f = (float)y; /* exact: y has at most 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(sign | ((u >> 16) & 0x7FFF));
+}
+
+int oracle_f64_to_bf16(const double *x, uint16_t *y, int64_t n)
+{
+    if (n < 0 || (n > 0 && (!x || !y))) return ORACLE_ERR_ARG;
+    for (int64_t i = 0; i < n; ++i) y[i] = f64_to_bf16_bits(x[i]);
+    return ORACLE_OK;
+}
+
+int oracle_bf16_to_f64(const uint16_t *x, double *y, int64_t n)
+{
+    if (n < 0 || (n > 0 && (!x || !y))) return ORACLE_ERR_ARG;
+    for (int64_t i = 0; i < n; ++i) y[i] = bf16_bits_to_f64(x[i]);
+    return ORACLE_OK;
+}
+
+/* ---- cube-major layout -------------------------------------------------
+ * Dataset card, "Shapes": Nq = ceil(T/4) * ceil(H/4) * ceil(W/4) cubes of
+ * 64 slots; cube c keeps vbs[c] real tokens. */
+
+static int ceil4(int n) { return (n + 3) / 4; }
+
+int oracle_cube_counts(int T, int Hh, int W, int32_t *vbs, int *nq_out)
+{
+    if (T <= 0 || Hh <= 0 || W <= 0) return ORACLE_ERR_ARG;
+    int nct = ceil4(T), nch = ceil4(Hh), ncw = ceil4(W);
+    if (nq_out) *nq_out = nct * nch * ncw;
+    if (!vbs) return ORACLE_OK;
+    for (int ct = 0; ct < nct; ++ct)
+        for (int ch = 0; ch < nch; ++ch)
+            for (int cw = 0; cw < ncw; ++cw) {
+                int et = (T - 4 * ct < 4) ? T - 4 * ct : 4;
+                int eh = (Hh - 4 * ch < 4) ? Hh - 4 * ch : 4;
+                int ew = (W - 4 * cw < 4) ? W - 4 * cw : 4;
+                vbs[(ct * nch + ch) * ncw + cw] = et * eh * ew;
+            }
+    return ORACLE_OK;
+}
+
+/* Slot (0..S-1) in the tiled sequence of raster token (t, h, w). */
+static int64_t tiled_slot(int t, int h, int w, int Hh, int W)
+{
+    int nch = ceil4(Hh), ncw = ceil4(W);
+    int ct = t / 4, ch = h / 4, cw = w / 4;
+    int eh = (Hh - 4 * ch < 4) ? Hh - 4 * ch : 4;
+    int ew = (W - 4 * cw < 4) ? W - 4 * cw : 4;
+    int lt = t - 4 * ct, lh = h - 4 * ch, lw = w - 4 * cw;
+    int64_t cube = ((int64_t)ct * nch + ch) * ncw + cw;
+    return cube * 64 + ((int64_t)lt * eh + lh) * ew + lw;
+}
+
+/* x_grid [B, T*Hh*W, H, D] raster order -> x_tiled [B, 64*Nq, H, D]; pads = 0. */
+int oracle_tile(const uint16_t *x_grid, uint16_t *x_tiled, int B, int T, int Hh, int W, int H, int D)
+{
+    int nq;
+    if (B <= 0 || H <= 0 || D <= 0 || oracle_cube_counts(T, Hh, W, NULL, &nq)) return ORACLE_ERR_ARG;
+    int64_t S = 64LL * nq, L = (int64_t)T * Hh * W, row = (int64_t)H * D;
+    memset(x_tiled, 0, (size_t)(B * S * row) * sizeof(uint16_t));
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t)
+            for (int h = 0; h < Hh; ++h)
+                for (int w = 0; w < W; ++w) {
+                    int64_t src = ((int64_t)t * Hh + h) * W + w;
+                    int64_t dst = tiled_slot(t, h, w, Hh, W);
+                    memcpy(x_tiled + ((int64_t)b * S + dst) * row,
+                           x_grid + ((int64_t)b * L + src) * row, (size_t)row * sizeof(uint16_t));
+                }
+    return ORACLE_OK;
+}
+
+/* Inverse of oracle_tile: keep the real slots, drop pads. */
+int oracle_untile(const uint16_t *x_tiled, uint16_t *x_grid, int B, int T, int Hh, int W, int H, int D)
+{
+    int nq;
+    if (B <= 0 || H <= 0 || D <= 0 || oracle_cube_counts(T, Hh, W, NULL, &nq)) return ORACLE_ERR_ARG;
+    int64_t S = 64LL * nq, L = (int64_t)T * Hh * W, row = (int64_t)H * D;
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t)
+            for (int h = 0; h < Hh; ++h)
+                for (int w = 0; w < W; ++w) {
+                    int64_t dst = ((int64_t)t * Hh + h) * W + w;
+                    int64_t src = tiled_slot(t, h, w, Hh, W);
+                    memcpy(x_grid + ((int64_t)b * L + dst) * row,
+                           x_tiled + ((int64_t)b * S + src) * row, (size_t)row * sizeof(uint16_t));
+                }
+    return ORACLE_OK;
+}
+
+/* ---- routing ----------------------------------------------------------- */
+
+/* Cube means over valid tokens (TensorRT-LLM PR #7 review excerpt: sum over
+ * valid tokens / valid count, cast back to the tiled dtype).
+ * x [B, S, H, D] bf16 -> xc [B, H, Nq, D] bf16.  A cube with vbs = 0 has mean 0. */
+int oracle_cube_means(const uint16_t *x, const int32_t *vbs, uint16_t *xc,
+                      int B, int S, int H, int D, int Nq)
+{
+    if (B <= 0 || H <= 0 || D <= 0 || Nq <= 0 || S != 64 * Nq) return ORACLE_ERR_ARG;
+    for (int c = 0; c < Nq; ++c)
+        if (vbs[c] < 0 || vbs[c] > 64) return ORACLE_ERR_ARG;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h)
+            for (int c = 0; c < Nq; ++c)
+                for (int d = 0; d < D; ++d) {
+                    double sum = 0.0;
+                    for (int u = 0; u < vbs[c]; ++u)
+                        sum += bf16_bits_to_f64(x[(((int64_t)b * S + 64LL * c + u) * H + h) * D + d]);
+                    double mean = vbs[c] > 0 ? sum / (double)vbs[c] : 0.0;
+                    xc[(((int64_t)b * H + h) * Nq + c) * D + d] = f64_to_bf16_bits(mean);
+                }
+    return ORACLE_OK;
+}
+
+typedef struct {
+    double score;
+    int32_t idx;
+} scored_t;
+
+/* Order: larger score first; NaN counts as -inf; equal scores -> lower index first. */
+static int cmp_scored(const void *pa, const void *pb)
+{
+    const scored_t *a = (const scored_t *)pa, *b = (const scored_t *)pb;
+    double sa = isnan(a->score) ? -INFINITY : a->score;
+    double sb = isnan(b->score) ? -INFINITY : b->score;
+    if (sa > sb) return -1;
+    if (sa < sb) return 1;
+    return (a->idx > b->idx) - (a->idx < b->idx);
+}
+
+/* Cube-mean q.k routing: for every (b, h, query cube i) pick the topk KV cubes
+ * with the largest score sc[i][j] = sum_d qc[i][d] * kc[j][d] (sequential FP64).
+ * scores (optional) receives sc as [B, H, Nq, Nq]. */
+int oracle_route(const uint16_t *q, const uint16_t *k, const int32_t *vbs, int32_t *topk_idx,
+                 int B, int S, int H, int D, int Nq, int topk, double *scores)
+{
+    if (topk < 1 || topk > Nq) return ORACLE_ERR_ARG;
+    int64_t nmean = (int64_t)B * H * Nq * D;
+    uint16_t *qc = (uint16_t *)malloc((size_t)nmean * sizeof(uint16_t));
+    uint16_t *kc = (uint16_t *)malloc((size_t)nmean * sizeof(uint16_t));
+    if (!qc || !kc) { free(qc); free(kc); return ORACLE_ERR_NOMEM; }
+    int rc = oracle_cube_means(q, vbs, qc, B, S, H, D, Nq);
+    if (!rc) rc = oracle_cube_means(k, vbs, kc, B, S, H, D, Nq);
+    if (rc) { free(qc); free(kc); return rc; }
+    int failed = 0;
+#pragma omp parallel
+    {
+        scored_t *row = (scored_t *)malloc((size_t)Nq * sizeof(scored_t));
+        if (!row) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for collapse(3) schedule(static)
+        for (int b = 0; b < B; ++b)
+            for (int h = 0; h < H; ++h)
+                for (int i = 0; i < Nq; ++i) {
+                    if (!row) continue;
+                    const uint16_t *qi = qc + (((int64_t)b * H + h) * Nq + i) * D;
+                    for (int j = 0; j < Nq; ++j) {
+                        const uint16_t *kj = kc + (((int64_t)b * H + h) * Nq + j) * D;
+                        double acc = 0.0;
+                        for (int d = 0; d < D; ++d)
+                            acc += bf16_bits_to_f64(qi[d]) * bf16_bits_to_f64(kj[d]);
+                        row[j].score = acc;
+                        row[j].idx = j;
+                        if (scores) scores[(((int64_t)b * H + h) * Nq + i) * Nq + j] = acc;
+                    }
+                    qsort(row, (size_t)Nq, sizeof(scored_t), cmp_scored);
+                    int32_t *dst = topk_idx + (((int64_t)b * H + h) * Nq + i) * topk;
+                    for (int t = 0; t < topk; ++t) dst[t] = row[t].idx;
+                }
+        free(row);
+    }
+    free(qc);
+    free(kc);
+    return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}
+
+/* ---- fine forward --------------------------------------------------------
+ * Dataset card, "Operator contract": for query row s of cube i, head h,
+ * batch b, the keys are the first vbs[j] tokens of every selected cube j
+ * (a cube listed twice counts twice); x_u = sigma * q_s . k_u;
+ * out_s = sum_u softmax(x)_u v_u; lse_s = log sum_u exp(x_u).
+ * Work is given as a list of (b, h, i) items; results are item-major:
+ * out [n_items, 64, D], lse [n_items, 64]. */
+int oracle_fwd_items(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                     const int32_t *topk_idx, const int32_t *vbs,
+                     int B, int S, int H, int D, int Nq, int topk, double sigma,
+                     const int32_t *items, int64_t n_items, double *out, double *lse)
+{
+    if (B <= 0 || H <= 0 || D <= 0 || Nq <= 0 || S != 64 * Nq || topk < 1) return ORACLE_ERR_ARG;
+    for (int c = 0; c < Nq; ++c)
+        if (vbs[c] < 0 || vbs[c] > 64) return ORACLE_ERR_ARG;
+    for (int64_t it = 0; it < n_items; ++it) {
+        int b = items[3 * it], h = items[3 * it + 1], i = items[3 * it + 2];
+        if (b < 0 || b >= B || h < 0 || h >= H || i < 0 || i >= Nq) return ORACLE_ERR_ARG;
+        const int32_t *sel = topk_idx + (((int64_t)b * H + h) * Nq + i) * topk;
+        for (int t = 0; t < topk; ++t)
+            if (sel[t] < 0 || sel[t] >= Nq) return ORACLE_ERR_ARG;
+    }
+    int failed = 0;
+#pragma omp parallel
+    {
+        int64_t *keys = (int64_t *)malloc((size_t)topk * 64 * sizeof(int64_t));
+        double *x = (double *)malloc((size_t)topk * 64 * sizeof(double));
+        if (!keys || !x) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t it = 0; it < n_items; ++it) {
+            if (!keys || !x) continue;
+            int b = items[3 * it], h = items[3 * it + 1], i = items[3 * it + 2];
+            const int32_t *sel = topk_idx + (((int64_t)b * H + h) * Nq + i) * topk;
+            /* the selected token set, multiplicity kept */
+            int64_t nkeys = 0;
+            for (int t = 0; t < topk; ++t)
+                for (int u = 0; u < vbs[sel[t]]; ++u) keys[nkeys++] = 64LL * sel[t] + u;
+            for (int r = 0; r < 64; ++r) {
+                int64_t s = 64LL * i + r;
+                const uint16_t *qs = q + (((int64_t)b * S + s) * H + h) * D;
+                double *o = out + (it * 64 + r) * D;
+                if (nkeys == 0) {
+                    for (int d = 0; d < D; ++d) o[d] = 0.0;
+                    lse[it * 64 + r] = -INFINITY;
+                    continue;
+                }
+                double m = -INFINITY;
+                for (int64_t n = 0; n < nkeys; ++n) {
+                    const uint16_t *ku = k + (((int64_t)b * S + keys[n]) * H + h) * D;
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) dot += bf16_bits_to_f64(qs[d]) * bf16_bits_to_f64(ku[d]);
+                    x[n] = sigma * dot;
+                    if (x[n] > m) m = x[n];
+                }
+                double l = 0.0;
+                for (int d = 0; d < D; ++d) o[d] = 0.0;
+                for (int64_t n = 0; n < nkeys; ++n) {
+                    double p = exp(x[n] - m);
+                    const uint16_t *vu = v + (((int64_t)b * S + keys[n]) * H + h) * D;
+                    l += p;
+                    for (int d = 0; d < D; ++d) o[d] += p * bf16_bits_to_f64(vu[d]);
+                }
+                for (int d = 0; d < D; ++d) o[d] /= l;
+                lse[it * 64 + r] = m + log(l);
+            }
+        }
+        free(keys);
+        free(x);
+    }
+    return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,377 @@
+"""Pins for the FP64 oracle, against things other than the oracle itself:
+the pages' printed shapes, exact rational arithmetic, textbook library
+routines (torch float64 softmax / SDPA / logsumexp), closed forms and
+invariants.  CPU only."""
+from __future__ import annotations
+
+import json
+import math
+import os
+import struct
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from tests import exact
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def f32_bits(x: float) -> int:
+    return struct.unpack("<I", struct.pack("<f", x))[0] >> 16
+
+
+# ---------------------------------------------------------------- bf16 rounding
+
+def test_bf16_rounding_special_values(oracle_lib):
+    o = oracle_lib
+    cases = [
+        (1.0, 0x3F80),
+        (-2.0, 0xC000),
+        (1.0 + 2.0 ** -8, 0x3F80),  # tie -> even (1.0)
+        (1.0 + 3 * 2.0 ** -8, 0x3F82),  # tie -> even (1 + 2^-6)
+        (1.0 + 2.0 ** -8 + 2.0 ** -40, 0x3F81),  # above the tie; a float32 detour would give 0x3F80
+        (2.0 ** -133, 0x0001),  # smallest bf16 subnormal
+        (0.5 * 2.0 ** -133, 0x0000),  # tie between 0 and 2^-133 -> even
+        (1.5 * 2.0 ** -133, 0x0002),  # tie -> even
+        (3.3895313892515355e38, 0x7F7F),  # largest finite bf16
+        (3.40e38, 0x7F80),  # rounds past the largest finite -> inf
+        (0.0, 0x0000),
+        (-0.0, 0x8000),
+        (math.inf, 0x7F80),
+        (-math.inf, 0xFF80),
+    ]
+    xs = np.array([c[0] for c in cases], dtype=np.float64)
+    got = o.f64_to_bf16(xs)
+    for (x, want), g in zip(cases, got):
+        assert int(g) == want, (x, hex(int(g)), hex(want))
+    assert int(o.f64_to_bf16(np.array([math.nan]))[0]) & 0x7FFF > 0x7F80
+
+
+def test_bf16_rounding_matches_library_cast_on_float32(oracle_lib):
+    """On float32 inputs a single rounding step is what torch's cast does."""
+    g = np.random.default_rng(1)
+    x = (g.standard_normal(200000) * np.exp(g.uniform(-60, 60, 200000))).astype(np.float32)
+    want = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = oracle_lib.f64_to_bf16(x.astype(np.float64))
+    np.testing.assert_array_equal(got, want)
+
+
+def test_bf16_rounding_matches_exact_rational(oracle_lib):
+    g = np.random.default_rng(2)
+    xs = g.standard_normal(3000) * np.exp(g.uniform(-30, 30, 3000))
+    got = oracle_lib.f64_to_bf16(xs)
+    for x, b in zip(xs, got):
+        assert int(b) == exact.fraction_to_bf16_bits(Fraction(float(x)))
+
+
+# ---------------------------------------------------------------- layout
+
+def test_wan480_shapes_match_pages(oracle_lib):
+    gold = json.load(open(os.path.join(GOLDEN, "wan480_shapes.json")))
+    T, Hh, W = gold["latent_grid"]
+    vbs = oracle_lib.cube_counts(T, Hh, W)
+    assert len(vbs) == gold["num_cubes"] == int(np.prod(gold["cubes_per_axis"]))
+    assert int(vbs.sum()) == gold["real_tokens"] == T * Hh * W
+    assert 64 * len(vbs) == gold["S_padded"]
+    assert 1.0 - gold["topk"] / len(vbs) == pytest.approx(gold["sparsity"])
+    # per-axis extents 21 = 5*4+1, 30 = 7*4+2, 52 = 13*4 give these cube sizes
+    vals, counts = np.unique(vbs, return_counts=True)
+    assert dict(zip(vals.tolist(), counts.tolist())) == {64: 455, 32: 65, 16: 91, 8: 13}
+
+
+def test_tiny_cube_counts(oracle_lib):
+    vbs = oracle_lib.cube_counts(5, 6, 7)
+    assert vbs.tolist() == [64, 48, 32, 24, 16, 12, 8, 6]
+    assert int(vbs.sum()) == 210
+    assert oracle_lib.cube_counts(24, 32, 52).tolist() == [64] * 624
+    vbs720 = oracle_lib.cube_counts(21, 45, 80)
+    assert len(vbs720) == 1440 and int(vbs720.sum()) == 21 * 45 * 80
+
+
+@pytest.mark.parametrize("grid", [(5, 6, 7), (1, 1, 1), (4, 4, 4), (9, 3, 5), (8, 8, 1)])
+def test_tile_by_brute_force(oracle_lib, grid):
+    """Each cube holds the raster tokens that fall inside it, in raster order,
+    followed by zero pads: derived here by filtering all tokens per cube."""
+    T, Hh, W = grid
+    H, D = 2, 8  # narrow rows suffice for the layout
+    L = T * Hh * W
+    g = np.random.default_rng(3)
+    x = g.integers(1, 60000, size=(2, L, H, D)).astype(np.uint16)
+    tiled = oracle_lib.tile(x, T, Hh, W)
+    nct, nch, ncw = -(-T // 4), -(-Hh // 4), -(-W // 4)
+    coords = [(t, h, w) for t in range(T) for h in range(Hh) for w in range(W)]  # raster order
+    expect = np.zeros((2, 64 * nct * nch * ncw, H, D), dtype=np.uint16)
+    for c, (ct, ch, cw) in enumerate((a, b, d) for a in range(nct) for b in range(nch) for d in range(ncw)):
+        members = [r for r, (t, h, w) in enumerate(coords) if t // 4 == ct and h // 4 == ch and w // 4 == cw]
+        expect[:, 64 * c: 64 * c + len(members)] = x[:, members]
+    np.testing.assert_array_equal(tiled, expect)
+    back = oracle_lib.untile(tiled, T, Hh, W)
+    np.testing.assert_array_equal(back, x)
+
+
+# ---------------------------------------------------------------- routing
+
+def test_cube_means_exact_rational(oracle_lib):
+    cfg = synth.CONFIGS["tiny"]
+    T, Hh, W = cfg.grid
+    q, _, _ = synth.grid_qkv(cfg)
+    qt = oracle_lib.tile(q, T, Hh, W)
+    vbs = oracle_lib.cube_counts(T, Hh, W)
+    means = oracle_lib.cube_means(qt, vbs)
+    for h in range(cfg.H):
+        for c in range(len(vbs)):
+            for d in range(0, 128, 7):
+                want = exact.exact_cube_mean_bits(qt[0, 64 * c: 64 * c + 64, h, d], int(vbs[c]))
+                assert int(means[0, h, c, d]) == want, (h, c, d)
+
+
+def test_cube_means_ignore_pads_and_empty_cube(oracle_lib):
+    g = np.random.default_rng(4)
+    x = synth.f32_to_bf16_bits(g.standard_normal((1, 3 * 64, 1, 128)).astype(np.float32))
+    vbs = np.array([64, 5, 0], dtype=np.int32)
+    m1 = oracle_lib.cube_means(x, vbs)
+    x2 = x.copy()
+    x2[0, 64 + 5: 128] = synth.f32_to_bf16_bits(np.full((59, 1, 128), 1e30, np.float32))
+    x2[0, 128:] = 0x7FC0  # NaN everywhere in the empty cube
+    m2 = oracle_lib.cube_means(x2, vbs)
+    np.testing.assert_array_equal(m1, m2)
+    assert np.all(m1[0, 0, 2] == 0)
+
+
+def test_route_planted_order(oracle_lib):
+    """Constant cubes along one channel: score = a_i * b_j in closed form, so the
+    selection is the topk largest (a_i > 0) or smallest (a_i < 0) b_j,
+    equal b_j ordered by lower index first."""
+    nq, topk = 12, 5
+    b_vals = np.array([3, -1, 7, 7, 0.5, 2, -8, 7, 1, 0.25, 4, 2], dtype=np.float32)
+    a_vals = np.array([1, -1, 2, -0.5, 1, 1, -3, 0.75, 1, -1, 1, 2], dtype=np.float32)
+    q = np.zeros((1, 64 * nq, 1, 128), np.float32)
+    k = np.zeros_like(q)
+    for c in range(nq):
+        q[0, 64 * c: 64 * c + 64, 0, 9] = a_vals[c]
+        k[0, 64 * c: 64 * c + 64, 0, 9] = b_vals[c]
+    vbs = np.full(nq, 64, np.int32)
+    vbs[3] = 17
+    idx, sc = oracle_lib.route(synth.f32_to_bf16_bits(q), synth.f32_to_bf16_bits(k), vbs, topk, want_scores=True)
+    np.testing.assert_array_equal(sc[0, 0], np.outer(a_vals, b_vals).astype(np.float64))
+    for i in range(nq):
+        order = sorted(range(nq), key=lambda j: (-(a_vals[i] * b_vals[j]), j))
+        assert idx[0, 0, i].tolist() == order[:topk], i
+
+
+def test_route_exact_scores_small(oracle_lib):
+    """Scores equal the exact rational dot products of the bf16 means, and the
+    selection is the exact top-k (ties by lower index)."""
+    cfg = synth.CONFIGS["tiny"]
+    T, Hh, W = cfg.grid
+    q, k, _ = synth.grid_qkv(cfg)
+    qt, kt = oracle_lib.tile(q, T, Hh, W), oracle_lib.tile(k, T, Hh, W)
+    vbs = oracle_lib.cube_counts(T, Hh, W)
+    nq = len(vbs)
+    idx, sc = oracle_lib.route(qt, kt, vbs, 3, want_scores=True)
+    qc = np.array([[[exact.exact_cube_mean_bits(qt[0, 64 * c: 64 * c + 64, h, d], int(vbs[c]))
+                     for d in range(128)] for c in range(nq)] for h in range(cfg.H)])
+    kc = np.array([[[exact.exact_cube_mean_bits(kt[0, 64 * c: 64 * c + 64, h, d], int(vbs[c]))
+                     for d in range(128)] for c in range(nq)] for h in range(cfg.H)])
+    for h in range(cfg.H):
+        for i in range(nq):
+            ex = []
+            for j in range(nq):
+                s = sum((exact.bf16_bits_to_fraction(a) * exact.bf16_bits_to_fraction(b)
+                         for a, b in zip(qc[h, i], kc[h, j])), Fraction(0))
+                ex.append(s)
+                assert abs(Fraction(sc[0, h, i, j]) - s) <= abs(s) * Fraction(1, 2 ** 45) + Fraction(1, 2 ** 100)
+            order = sorted(range(nq), key=lambda j: (-ex[j], j))
+            assert idx[0, h, i].tolist() == order[:3]
+
+
+def test_route_wan480_lists_distinct_and_valid(oracle_lib):
+    """On the Wan shape every list is a set of distinct valid cubes and the lists
+    differ across heads and query cubes (the dataset card's 'not banded')."""
+    cfg = synth.CONFIGS["wan480"]
+    T, Hh, W = cfg.grid
+    # three heads are enough for the property and keep the test short
+    q, k, _ = synth.grid_qkv(dataclasses_replace(cfg, H=3))
+    qt, kt = oracle_lib.tile(q, T, Hh, W), oracle_lib.tile(k, T, Hh, W)
+    vbs = oracle_lib.cube_counts(T, Hh, W)
+    idx = oracle_lib.route(qt, kt, vbs, cfg.topk)
+    assert idx.shape == (1, 3, 624, 78)
+    assert idx.min() >= 0 and idx.max() < 624
+    srt = np.sort(idx, axis=-1)
+    assert np.all(srt[..., 1:] != srt[..., :-1])
+    rows = {tuple(r) for r in srt.reshape(-1, 78).tolist()}
+    assert len(rows) > 0.99 * 3 * 624
+
+
+def dataclasses_replace(cfg, **kw):
+    import dataclasses
+    return dataclasses.replace(cfg, **kw)
+
+
+# ---------------------------------------------------------------- fine forward
+
+def _dense_reference(q, k, v, idx, vbs, sm_scale):
+    """Textbook masked attention in torch float64: logits + log(multiplicity)
+    for selected valid keys, -inf elsewhere, softmax, times V; plus logsumexp."""
+    B, S, H, D = q.shape
+    nq = S // 64
+    qd = torch.from_numpy(exact_bits_to_f64(q))
+    kd = torch.from_numpy(exact_bits_to_f64(k))
+    vd = torch.from_numpy(exact_bits_to_f64(v))
+    sigma = float(np.float32(sm_scale))
+    out = torch.zeros(B, S, H, D, dtype=torch.float64)
+    lse = torch.zeros(B, H, S, dtype=torch.float64)
+    valid = torch.zeros(S, dtype=torch.bool)
+    for c in range(nq):
+        valid[64 * c: 64 * c + int(vbs[c])] = True
+    for b in range(B):
+        for h in range(H):
+            logits = sigma * (qd[b, :, h] @ kd[b, :, h].T)  # [S, S]
+            bias = torch.full((S, S), -math.inf, dtype=torch.float64)
+            for i in range(nq):
+                cnt = np.bincount(idx[b, h, i], minlength=nq)
+                for j in np.nonzero(cnt)[0]:
+                    cols = torch.arange(64 * j, 64 * j + 64)
+                    cols = cols[valid[cols]]
+                    bias[64 * i: 64 * i + 64, cols] = math.log(cnt[j])
+            z = logits + bias
+            lse[b, h] = torch.logsumexp(z, dim=1)
+            p = torch.softmax(z, dim=1)
+            p = torch.nan_to_num(p, nan=0.0)  # rows with no key at all
+            out[b, :, h] = p @ vd[b, :, h]
+    return out.numpy(), lse.numpy()
+
+
+def exact_bits_to_f64(x):
+    return (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _random_case(seed, B, H, nq, topk, vbs=None, dup=False, scale=2.0):
+    g = np.random.default_rng(seed)
+    S = 64 * nq
+    q, k, v = (synth.f32_to_bf16_bits((g.standard_normal((B, S, H, 128)) * scale).astype(np.float32))
+               for _ in range(3))
+    if vbs is None:
+        vbs = g.integers(0, 65, size=nq).astype(np.int32)
+        vbs[0] = 64
+    idx = synth.random_topk(seed, B, H, nq, topk, distinct=not dup)
+    return q, k, v, idx, np.asarray(vbs, np.int32)
+
+
+@pytest.mark.parametrize("seed,B,H,nq,topk,dup", [(0, 1, 2, 4, 2, False), (1, 2, 1, 5, 3, True),
+                                                   (2, 1, 1, 3, 3, False), (3, 1, 2, 6, 1, False)])
+def test_fwd_matches_masked_dense_attention(oracle_lib, seed, B, H, nq, topk, dup):
+    q, k, v, idx, vbs = _random_case(seed, B, H, nq, topk, dup=dup)
+    out, lse = oracle_lib.fwd(q, k, v, idx, vbs, 1 / math.sqrt(128))
+    ref, ref_lse = _dense_reference(q, k, v, idx, vbs, 1 / math.sqrt(128))
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+    finite = np.isfinite(ref_lse)
+    assert np.array_equal(finite, np.isfinite(lse))
+    np.testing.assert_allclose(lse[finite], ref_lse[finite], rtol=1e-13, atol=0)
+
+
+def test_fwd_tiny_config_matches_masked_dense(oracle_lib):
+    cfg = synth.CONFIGS["tiny"]
+    T, Hh, W = cfg.grid
+    q, k, v = synth.grid_qkv(cfg)
+    qt, kt, vt = (oracle_lib.tile(x, T, Hh, W) for x in (q, k, v))
+    vbs = oracle_lib.cube_counts(T, Hh, W)
+    idx = oracle_lib.route(qt, kt, vbs, cfg.topk)
+    out, lse = oracle_lib.fwd(qt, kt, vt, idx, vbs, cfg.sm_scale)
+    ref, ref_lse = _dense_reference(qt, kt, vt, idx, vbs, cfg.sm_scale)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse, rtol=1e-13)
+
+
+def test_fwd_full_selection_is_dense_attention(oracle_lib):
+    """topk = Nq with every cube full: plain dense attention (torch SDPA)."""
+    nq = 4
+    q, k, v, _, _ = _random_case(5, 1, 2, nq, nq, vbs=[64] * nq)
+    idx = np.broadcast_to(np.arange(nq, dtype=np.int32), (1, 2, nq, nq)).copy()
+    out, _ = oracle_lib.fwd(q, k, v, idx, np.full(nq, 64, np.int32), 1 / math.sqrt(128))
+    qd, kd, vd = (torch.from_numpy(exact_bits_to_f64(x)).permute(0, 2, 1, 3) for x in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        qd, kd, vd, scale=float(np.float32(1 / math.sqrt(128)))).permute(0, 2, 1, 3).numpy()
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+def test_fwd_constant_v(oracle_lib):
+    q, k, v, idx, vbs = _random_case(6, 1, 2, 5, 3)
+    vbs[:] = np.maximum(vbs, 1)
+    v[:] = f32_bits(1.0)
+    out, _ = oracle_lib.fwd(q, k, v, idx, vbs, 1 / math.sqrt(128))
+    assert np.all(out == 1.0)  # sum(p * 1) / sum(p) in the same order: exactly 1
+    v[:] = f32_bits(-1.625)
+    out, _ = oracle_lib.fwd(q, k, v, idx, vbs, 1 / math.sqrt(128))
+    np.testing.assert_allclose(out, -1.625, rtol=1e-14, atol=0)
+
+
+def test_fwd_permuted_selection(oracle_lib):
+    q, k, v, idx, vbs = _random_case(7, 1, 2, 6, 4)
+    out, lse = oracle_lib.fwd(q, k, v, idx, vbs, 0.1)
+    perm = idx[..., ::-1].copy()
+    out2, lse2 = oracle_lib.fwd(q, k, v, perm, vbs, 0.1)
+    # only the summation order changes: a few FP64 ulps of the largest |v|
+    np.testing.assert_allclose(out2, out, rtol=0, atol=1e-14 * np.abs(out).max())
+    np.testing.assert_allclose(lse2, lse, rtol=1e-15)
+
+
+def test_fwd_single_token_selection(oracle_lib):
+    """One selected cube with one valid token: every row is that v row exactly."""
+    q, k, v, _, _ = _random_case(8, 1, 2, 4, 1)
+    vbs = np.array([64, 1, 30, 64], np.int32)
+    idx = np.full((1, 2, 4, 1), 1, np.int32)
+    out, lse = oracle_lib.fwd(q, k, v, idx, vbs, 1 / math.sqrt(128))
+    vrow = exact_bits_to_f64(v[0, 64, :, :])  # [H, D]
+    for h in range(2):
+        np.testing.assert_array_equal(out[0, :, h, :], np.broadcast_to(vrow[h], (256, 128)))
+    qd, kd = exact_bits_to_f64(q), exact_bits_to_f64(k)
+    sigma = float(np.float32(1 / math.sqrt(128)))
+    np.testing.assert_allclose(lse[0, 0], sigma * (qd[0, :, 0] @ kd[0, 64, 0]), rtol=1e-13)
+
+
+def test_fwd_all_masked_rows(oracle_lib):
+    q, k, v, _, _ = _random_case(9, 1, 1, 3, 2)
+    vbs = np.array([0, 0, 64], np.int32)
+    idx = np.array([[[[0, 1], [2, 0], [1, 1]]]], np.int32)
+    out, lse = oracle_lib.fwd(q, k, v, idx, vbs, 0.2)
+    assert np.all(out[0, 0:64] == 0) and np.all(lse[0, 0, 0:64] == -np.inf)
+    assert np.all(out[0, 128:] == 0) and np.all(lse[0, 0, 128:] == -np.inf)
+    assert np.all(np.isfinite(lse[0, 0, 64:128]))
+
+
+def test_fwd_nan_in_pads_is_ignored(oracle_lib):
+    q, k, v, idx, vbs = _random_case(10, 1, 2, 5, 3)
+    vbs[:] = [64, 10, 33, 1, 0]
+    out, lse = oracle_lib.fwd(q, k, v, idx, vbs, 1 / math.sqrt(128))
+    k2, v2 = k.copy(), v.copy()
+    for c in range(5):
+        k2[0, 64 * c + vbs[c]: 64 * c + 64] = 0x7FC0
+        v2[0, 64 * c + vbs[c]: 64 * c + 64] = 0xFF80
+    out2, lse2 = oracle_lib.fwd(q, k2, v2, idx, vbs, 1 / math.sqrt(128))
+    np.testing.assert_array_equal(out2, out)
+    np.testing.assert_array_equal(lse2, lse)
+
+
+def test_fwd_items_subset_equals_full(oracle_lib):
+    q, k, v, idx, vbs = _random_case(11, 2, 2, 4, 2)
+    out, lse = oracle_lib.fwd(q, k, v, idx, vbs, 0.3)
+    items = np.array([[1, 0, 3], [0, 1, 0], [1, 1, 2]], np.int32)
+    o, l = oracle_lib.fwd_items(q, k, v, idx, vbs, 0.3, items)
+    for n, (b, h, i) in enumerate(items):
+        np.testing.assert_array_equal(o[n], out[b, 64 * i: 64 * i + 64, h])
+        np.testing.assert_array_equal(l[n], lse[b, h, 64 * i: 64 * i + 64])
+
+
+def test_oracle_rejects_bad_arguments(oracle_lib):
+    q, k, v, idx, vbs = _random_case(12, 1, 1, 3, 2)
+    bad = idx.copy()
+    bad[0, 0, 0, 0] = 3
+    with pytest.raises(ValueError):
+        oracle_lib.fwd(q, k, v, bad, vbs, 0.1)
+    with pytest.raises(ValueError):
+        oracle_lib.fwd(q, k, v, idx, np.array([65, 1, 1], np.int32), 0.1)
