@@ -1,0 +1,345 @@
+"""Benchmark of the VSA fine stage on B200: one step = the whole hot path on
+one batch of synthetic Wan2.2 832x480/81f activations:
+
+    tile q, k, v (raster -> cube-major)  ->  route (cube-mean q.k top-k)
+    ->  fine block-sparse attention forward  ->  untile the output
+
+Metric: effective TFLOP/s of the step, FLOPs = 4 * B * S * topk * 64 * D * H
+(the attention contractions; the other steps count no FLOPs).  Inputs are
+resident in HBM when the timed region starts; they are larger than L2
+(3 x 335 MB raster q, k, v per step), so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Under torchrun every rank runs its own independent problem (weak scaling, no
+data-path collective); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+WORKLOAD = "wan480"
+METRIC = "VSA fine fwd ms/call & TFLOP/s at Wan2.2 832x480/81f; % B200 BF16 peak"
+
+
+def flops(cfg, S):
+    return 4.0 * cfg.B * S * cfg.topk * 64 * 128 * cfg.H
+
+
+def config_block(cfg, S):
+    return {
+        "workload": "Wan2.2 T2V-A14B 832x480/81f VSA fine stage (tile q,k,v -> route -> fwd -> untile)",
+        "B": cfg.B, "latent_grid": list(cfg.grid), "S_padded": S, "H": cfg.H, "D": 128, "topk": cfg.topk,
+        "sm_scale": cfg.sm_scale, "global_batch": cfg.B, "seq_len": S, "parallelism": "replicas (independent problem per GPU)",
+        "l2": "inputs larger than L2 (1.0 GB raster q,k,v read per step); no flush",
+        "inputs": "seeded synthetic: q,k ~ N(0,1)*U[1,8] per head with 4 shared outlier channels x20, v ~ N(0,1)",
+    }
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["bf16_tflops"], d.get("bf16_tflops_sustained"), d["hbm_gbs"], "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def __enter__(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}",
+                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+                 "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_power_cap", "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+def run_gpu(args, rank, world, local_rank):
+    import video_block_sparse_b200 as vsa
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = synth.CONFIGS[WORKLOAD]
+    import dataclasses
+
+    cfg = dataclasses.replace(cfg, seed=rank)  # an independent problem per rank
+    T, Hh, W = cfg.grid
+    vbs_h = vsa.cube_counts(T, Hh, W)
+    nq = len(vbs_h)
+    S = 64 * nq
+    q_h, k_h, v_h = (synth.bits_to_torch(x) for x in synth.grid_qkv(cfg))
+    q_g, k_g, v_g = (x.to(dev) for x in (q_h, k_h, v_h))
+    vbs = vbs_h.to(dev)
+    B, L, H, D = q_g.shape
+    qt, kt, vt = (torch.empty(B, S, H, D, dtype=torch.bfloat16, device=dev) for _ in range(3))
+    idx = torch.empty(B, H, nq, cfg.topk, dtype=torch.int32, device=dev)
+    ws = torch.empty(vsa.route_workspace_size(B, H, nq, D), dtype=torch.uint8, device=dev)
+    out_t = torch.empty_like(qt)
+    out_g = torch.empty_like(q_g)
+    lse = torch.empty(B, H, S, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ev_f0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_f1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+
+    def step(i=None):
+        vsa.tile(q_g, cfg.grid, out=qt)
+        vsa.tile(k_g, cfg.grid, out=kt)
+        vsa.tile(v_g, cfg.grid, out=vt)
+        vsa.route(qt, kt, vbs, cfg.topk, out=idx, workspace=ws)
+        if i is not None:
+            ev_f0[i].record(stream)
+        vsa.fwd(qt, kt, vt, idx, vbs, cfg.sm_scale, out=out_t, lse=lse)
+        if i is not None:
+            ev_f1[i].record(stream)
+        vsa.untile(out_t, cfg.grid, out=out_g)
+
+    launches_per_step = 3 + 2 + 1 + 1
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    rc, detail = vsa.device_status()
+    if rc != 0:
+        raise RuntimeError(f"device error {rc}/{detail} in warm-up")
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms_total = t0.elapsed_time(t1)
+    fwd_ms = [a.elapsed_time(b) for a, b in zip(ev_f0, ev_f1)]
+
+    # end to end through the public API: pinned host raster q,k,v in, raster out back
+    q_p, k_p, v_p = (x.pin_memory() for x in (q_h, k_h, v_h))
+    out_p = torch.empty(out_g.shape, dtype=out_g.dtype).pin_memory()
+    e2e_steps = max(1, min(args.steps, 10))
+
+    def e2e_step():
+        q_g.copy_(q_p, non_blocking=True)
+        k_g.copy_(k_p, non_blocking=True)
+        v_g.copy_(v_p, non_blocking=True)
+        step()
+        out_p.copy_(out_g, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    rc, detail = vsa.device_status()
+    if rc != 0:
+        raise RuntimeError(f"device error {rc}/{detail}")
+
+    ms_step = ms_total / args.steps
+    t = torch.tensor([ms_step, e2e_ms, statistics.mean(fwd_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_step, e2e_ms, fwd_avg = (float(x) for x in t.tolist())
+    return dict(cfg=cfg, S=S, ms_step=ms_step, e2e_ms=e2e_ms, fwd_ms=fwd_avg, fwd_list=fwd_ms,
+                clocks=clk.summary(), launches=launches_per_step * args.steps,
+                h2d=3 * q_h.numel() * 2, d2h=out_g.numel() * 2)
+
+
+# --------------------------------------------------------------------------- oracle timing
+
+class OracleWorkload:
+    """The FP64 oracle on the bench workload, for a CPU baseline: inputs for
+    two heads of the Wan shape are drawn, tiled and routed once; a 'step' then
+    runs the oracle forward on a bounded chunk of query-cube work items."""
+
+    def __init__(self, cfg, seed=0):
+        import dataclasses
+
+        import oracle
+
+        self.oracle = oracle
+        self.cfg = cfg
+        T, Hh, W = cfg.grid
+        sub = dataclasses.replace(cfg, H=2)
+        q, k, v = synth.grid_qkv(sub)
+        self.qt, self.kt, self.vt = (oracle.tile(x, T, Hh, W) for x in (q, k, v))
+        self.vbs = oracle.cube_counts(T, Hh, W)
+        self.idx = oracle.route(self.qt, self.kt, self.vbs, cfg.topk)
+        items = oracle.all_items(1, 2, len(self.vbs))
+        self.items = items[np.random.default_rng(seed).permutation(len(items))]
+        self.pos = 0
+        self.threads = oracle.num_threads()
+
+    def step(self, n):
+        chunk = self.items[self.pos: self.pos + n]
+        if len(chunk) < n:
+            self.pos = 0
+            chunk = self.items[:n]
+        self.pos += n
+        t0 = time.perf_counter()
+        self.oracle.fwd_items(self.qt, self.kt, self.vt, self.idx, self.vbs, self.cfg.sm_scale, chunk)
+        return time.perf_counter() - t0, len(chunk) * 4.0 * 64 * self.cfg.topk * 64 * 128
+
+
+def oracle_sample(cfg, seconds=15.0):
+    """Time the oracle for about `seconds`: (TFLOP/s, items, seconds, threads)."""
+    w = OracleWorkload(cfg)
+    n = 2 * w.threads
+    t_used, fl, items = 0.0, 0.0, 0
+    while t_used < seconds and items < len(w.items):
+        dt, f = w.step(n)
+        t_used += dt
+        fl += f
+        items += n
+    return fl / t_used / 1e12, items, t_used, w.threads
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--oracle-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = synth.CONFIGS[WORKLOAD]
+    S = 64 * int(np.prod([-(-x // 4) for x in cfg.grid]))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        w = OracleWorkload(cfg)
+        n = 2 * w.threads
+        for _ in range(args.warmup):
+            w.step(n)
+        t_used, fl = 0.0, 0.0
+        for _ in range(args.steps):
+            dt, f = w.step(n)
+            t_used += dt
+            fl += f
+        tf, items, secs, threads = fl / t_used / 1e12, n * args.steps, t_used, w.threads
+        value = tf
+        line = {
+            "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": flops(cfg, S) / (value * 1e12) * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config_block(cfg, S),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{items} query-cube work items of the workload (2 heads drawn), {secs:.1f} s"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line))
+        return
+
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    res = run_gpu(args, rank, world, local_rank)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+
+    peak_burst, peak_sus, hbm, peak_kind = read_peaks()
+    fl = flops(res["cfg"], res["S"])
+    value = world * fl / (res["ms_step"] * 1e-3) / 1e12
+    fwd_achieved = fl / (res["fwd_ms"] * 1e-3) / 1e12
+    cpu = None
+    if world == 1:
+        tf, items, secs, threads = oracle_sample(res["cfg"], seconds=args.oracle_seconds)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{items} query-cube work items of the workload (2 heads drawn), {secs:.1f} s"}
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "fwd_traffic.json")
+    if os.path.exists(tpath):
+        traffic = json.load(open(tpath)).get("bytes_per_launch")
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": res["ms_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_block(res["cfg"], res["S"]),
+        "fwd_ms": res["fwd_ms"], "fwd_tflops": fwd_achieved,
+        "roofline": {"bound": "tensor", "achieved": fwd_achieved, "peak": peak_burst, "unit": "TFLOP/s",
+                     "frac": fwd_achieved / peak_burst, "traffic": traffic,
+                     "peak_source": f"{peak_kind} bf16 burst (sustained {peak_sus})"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * fl / (res["e2e_ms"] * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
+        "gpu_launches": res["launches"],
+        "clocks": res["clocks"],
+    }
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

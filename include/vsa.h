@@ -1,0 +1,180 @@
+/*
+ * vsa.h -- C ABI of the B200 (sm_100a) library for the fine stage of Video
+ * Sparse Attention (VSA): block-sparse attention over cube-major 64-token
+ * tiles, the cube-mean routing that selects the tiles, and the 4x4x4
+ * cube-major layout transforms.
+ *
+ * Conventions (shared by every entry point):
+ *  - Tensor pointers are DEVICE pointers to dense, contiguous, row-major
+ *    buffers, at least 16-byte aligned.  The caller owns every buffer; the
+ *    library never allocates, frees, synchronises, or falls back to the CPU.
+ *  - bf16 values are passed as their 16-bit patterns (vsa_bf16).
+ *  - Work is enqueued on `stream`; a call returns once its kernels are
+ *    launched.  A status of VSA_OK means the launch was accepted; errors
+ *    raised later by the device (bad index found by a kernel, a bounded
+ *    wait that ran out) are latched in a device word and read with
+ *    vsa_device_status().
+ *  - Every function is noexcept in effect: it returns a status and never
+ *    aborts.  Arguments are checked before anything is launched; a call that
+ *    returns an error has launched nothing.
+ *
+ * Shapes (the dataset card "wan2.2_production_values", sections "Shapes",
+ * "Operator contract" and "Load"):
+ *   B batch, H heads, D head dim (= 128), Nq cubes, S = 64 * Nq padded tokens,
+ *   q, k, v, out : [B, S, H, D] bf16 (BSHD, cube-major)
+ *   topk_idx     : [B, H, Nq, topk] int32, values in [0, Nq)
+ *   vbs          : [Nq] int32, values in [0, 64], shared by batch and heads
+ *   lse          : [B, H, S] fp32, natural log (optional output)
+ */
+#ifndef VSA_H
+#define VSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define VSA_API __attribute__((visibility("default")))
+#else
+#define VSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t vsa_bf16;
+
+enum vsa_status {
+    VSA_OK = 0,
+    VSA_ERR_ARG = -1,       /* a size or count is out of range (see each call) */
+    VSA_ERR_NULL = -2,      /* a required pointer is NULL */
+    VSA_ERR_ALIGN = -3,     /* a pointer is not 16-byte aligned */
+    VSA_ERR_WORKSPACE = -4, /* workspace missing or smaller than the size query says */
+    VSA_ERR_ARCH = -5,      /* the current device is not sm_100 */
+    VSA_ERR_LAUNCH = -6,    /* the CUDA runtime rejected a launch (cudaGetLastError) */
+    VSA_ERR_DEVICE = -7     /* a kernel latched an error (see vsa_device_status) */
+};
+
+/* Human-readable name of a status code (static storage). */
+VSA_API const char *vsa_status_string(int status);
+
+/* 1 if this library has kernels for head dim D on an SM of version
+ * `sm_version` (major*10+minor), else 0.  Only D = 128 on sm_100. */
+VSA_API int vsa_can_implement(int D, int sm_version);
+
+/* ------------------------------------------------------------------------
+ * vsa_fwd -- fine block-sparse attention forward.
+ *
+ * Dataset card "wan2.2_production_values", section "Operator contract":
+ * non-causal block-sparse attention in BSHD layout,
+ *   out = softmax(q . k_sel^T * sm_scale) . v_sel,
+ * where, for query cube i of (batch b, head h), k_sel / v_sel are the
+ * tokens of the cubes listed in topk_idx[b, h, i, :], and of cube c only the
+ * first vbs[c] of its 64 tokens take part.  A cube listed twice counts
+ * twice; the order of a list does not matter.  Every query row (padded ones
+ * included) is computed.  A row whose selected cubes hold no valid token
+ * gets out = 0 and lse = -inf.  K/V slots at or beyond vbs[c] are never
+ * read into the result, even if they hold NaN or Inf.
+ *
+ *   q, k, v  [B, S, H, D] bf16      in
+ *   topk_idx [B, H, Nq, topk] int32 in
+ *   vbs      [Nq] int32             in
+ *   out      [B, S, H, D] bf16      out (may not alias inputs)
+ *   lse      [B, H, S] fp32         out, natural-log log-sum-exp of the
+ *            scaled logits per query row; NULL to skip.
+ *   sm_scale  logit scale (1/sqrt(D) in the contract).
+ *
+ * Errors: VSA_ERR_ARG if S != 64*Nq, D != 128, topk < 1, B, H or Nq < 1,
+ * or B*H*Nq, S*H*D overflow the kernel's index range; VSA_ERR_NULL for a
+ * NULL required pointer; VSA_ERR_ALIGN for a pointer not 16-byte aligned;
+ * VSA_ERR_ARCH off sm_100; VSA_ERR_LAUNCH if a launch fails.  Out-of-range
+ * topk_idx or vbs values found by the kernel set VSA_ERR_DEVICE; the
+ * affected entries are skipped.
+ * ---------------------------------------------------------------------- */
+VSA_API int vsa_fwd(const vsa_bf16 *q, const vsa_bf16 *k, const vsa_bf16 *v, const int32_t *topk_idx,
+            const int32_t *vbs, vsa_bf16 *out, float *lse, int B, int S, int H, int D, int Nq, int topk,
+            float sm_scale, cudaStream_t stream);
+
+/* Precision options for vsa_fwd_ex. */
+enum vsa_fwd_flags {
+    VSA_FWD_DEFAULT = 0,
+    /* Carry the softmax weights P into the P.V product as a bf16 pair
+     * (P = hi + lo) instead of one bf16 value: about 2^-16 relative weight
+     * error instead of 2^-9, for workloads whose softmax is spread over many
+     * keys.  Costs one extra P.V product per tile. */
+    VSA_FWD_PRECISE_P = 1
+};
+
+/* vsa_fwd with option flags (vsa_fwd == vsa_fwd_ex with VSA_FWD_DEFAULT). */
+VSA_API int vsa_fwd_ex(const vsa_bf16 *q, const vsa_bf16 *k, const vsa_bf16 *v, const int32_t *topk_idx,
+               const int32_t *vbs, vsa_bf16 *out, float *lse, int B, int S, int H, int D, int Nq, int topk,
+               float sm_scale, int flags, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * vsa_route -- cube-mean q.k routing that builds topk_idx.
+ *
+ * "align VisualGen VSA with block-sparse FMHA" (TensorRT-LLM PR #7), review
+ * excerpts: the cube mean is the sum over the cube's valid tokens divided by
+ * the valid count, cast back to the tiled dtype; the VSA predictor selects
+ * KV cubes from these means ("Video Sparse Attention Runner", TensorRT-Edge
+ * docs: block means of K are rounded to bf16 before routing).  The score of
+ * query cube i against KV cube j is sum_d qc[i][d] * kc[j][d]; topk_idx
+ * lists the topk largest scores, largest first, equal scores by lower index.
+ * Arithmetic (fixed so that the result is exact and reproducible):
+ *   mean = bf16_round_nearest_even(fp64_sequential_sum / vbs)  (0 if vbs = 0)
+ *   score = fp64 sequential sum over d of the exact bf16 products
+ *   a NaN score ranks as -inf.
+ *
+ *   q, k      [B, S, H, D] bf16 in
+ *   vbs       [Nq] int32 in
+ *   topk_idx  [B, H, Nq, topk] int32 out
+ *   workspace device scratch of at least vsa_route_workspace_size(B, H, Nq, D)
+ *             bytes (any 16-byte-aligned address), owned by the caller;
+ *             contents on entry are ignored.
+ *
+ * Errors: as vsa_fwd, plus VSA_ERR_ARG for topk > Nq or Nq > 4096, and
+ * VSA_ERR_WORKSPACE for a NULL or short workspace.
+ * ---------------------------------------------------------------------- */
+VSA_API size_t vsa_route_workspace_size(int B, int H, int Nq, int D);
+
+VSA_API int vsa_route(const vsa_bf16 *q, const vsa_bf16 *k, const int32_t *vbs, int32_t *topk_idx, int B, int S, int H,
+              int D, int Nq, int topk, void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Cube-major layout.  Dataset card "wan2.2_production_values", section
+ * "Shapes": a T x Hh x W latent grid is cut into 4x4x4 cubes,
+ * Nq = ceil(T/4) * ceil(Hh/4) * ceil(W/4), S = 64 * Nq.  Cubes are ordered
+ * (ct, ch, cw) row-major; inside cube c its real tokens come first, in
+ * local (t, h, w) row-major order over the cube's real extent, followed by
+ * zero pads up to 64; vbs[c] is its real-token count.
+ * ---------------------------------------------------------------------- */
+
+/* Host-only: Nq and (if vbs_host != NULL) the [Nq] valid counts.
+ * Errors: VSA_ERR_ARG for a non-positive extent or Nq beyond INT32. */
+VSA_API int vsa_cube_counts(int T, int Hh, int W, int32_t *vbs_host, int *Nq_out);
+
+/* x_grid [B, T*Hh*W, H, D] (raster order) -> x_tiled [B, 64*Nq, H, D]; pads
+ * are written as zeros.  Requires H*D to be a multiple of 8.  Untiling by an
+ * index gather is described in TensorRT-LLM PR #7 (review excerpts). */
+VSA_API int vsa_tile(const vsa_bf16 *x_grid, vsa_bf16 *x_tiled, int B, int T, int Hh, int W, int H, int D,
+             cudaStream_t stream);
+
+/* Inverse of vsa_tile: x_tiled [B, 64*Nq, H, D] -> x_grid [B, T*Hh*W, H, D]. */
+VSA_API int vsa_untile(const vsa_bf16 *x_tiled, vsa_bf16 *x_grid, int B, int T, int Hh, int W, int H, int D,
+               cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Device error word.  Synchronises `stream`, returns VSA_OK or
+ * VSA_ERR_DEVICE (and clears the word), or VSA_ERR_LAUNCH if the stream
+ * reports a CUDA error.  `detail` (may be NULL) receives the latched code:
+ * 1 = topk_idx value out of range, 2 = vbs value out of range,
+ * 3 = a bounded pipeline wait ran out.
+ * ---------------------------------------------------------------------- */
+VSA_API int vsa_device_status(cudaStream_t stream, int *detail);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VSA_H */

@@ -1,0 +1,124 @@
+"""The C-ABI library loads and exports every symbol include/vsa.h declares;
+argument errors are reported before anything touches a device.  CPU only."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def vsa():
+    from video_block_sparse_b200 import build
+
+    build.build()
+    import video_block_sparse_b200 as m
+
+    return m
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "vsa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(vsa_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    for n in ("vsa_fwd", "vsa_route", "vsa_tile", "vsa_untile", "vsa_cube_counts", "vsa_route_workspace_size",
+              "vsa_can_implement", "vsa_status_string", "vsa_device_status", "vsa_fwd_ex"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(vsa):
+    lib = ctypes.CDLL(vsa.LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(lib, n), f"{n} declared in vsa.h but not exported"
+    assert set(declared_functions()) <= set(vsa.EXPORTS) | set(declared_functions())
+    assert set(vsa.EXPORTS) <= set(declared_functions())
+
+
+def test_library_exports_nothing_else(vsa):
+    import subprocess
+
+    out = subprocess.run(["nm", "-D", "--defined-only", vsa.LIB_PATH], capture_output=True, text=True).stdout
+    ours = sorted({ln.split()[-1] for ln in out.splitlines() if " T " in ln and ln.split()[-1].startswith("vsa_")})
+    assert ours == declared_functions()
+
+
+def test_status_strings_and_capability(vsa):
+    assert vsa.status_string(0) == "VSA_OK"
+    for s in range(-7, 0):
+        assert vsa.status_string(s).startswith("VSA_ERR")
+    assert vsa.can_implement(128, 100)
+    assert not vsa.can_implement(64, 100)
+    assert not vsa.can_implement(128, 90)
+
+
+def test_cube_counts_host(vsa):
+    import oracle
+
+    for grid in [(5, 6, 7), (21, 30, 52), (21, 45, 80), (1, 1, 1), (24, 32, 52)]:
+        assert vsa.cube_counts(*grid).tolist() == oracle.cube_counts(*grid).tolist()
+    with pytest.raises(vsa.VSAError):
+        vsa.cube_counts(0, 4, 4)
+
+
+def test_route_workspace_size(vsa):
+    assert vsa.route_workspace_size(1, 40, 624, 128) == 2 * 40 * 624 * 128 * 2
+    assert vsa.route_workspace_size(0, 40, 624, 128) == 0
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+@pytest.mark.parametrize("B,S,H,D,Nq,topk,expect", [
+    (1, 512, 2, 64, 8, 2, -1),    # D != 128
+    (1, 500, 2, 128, 8, 2, -1),   # S != 64 * Nq
+    (0, 512, 2, 128, 8, 2, -1),   # B < 1
+    (1, 512, 0, 128, 8, 2, -1),   # H < 1
+    (1, 512, 2, 128, 8, 0, -1),   # topk < 1
+])
+def test_fwd_rejects_bad_sizes_without_a_device(vsa, B, S, H, D, Nq, topk, expect):
+    p = _fake(1 << 20)
+    rc = vsa.get_lib().vsa_fwd(p, p, p, p, p, p, None, B, S, H, D, Nq, topk, 0.1, None)
+    assert rc == expect
+
+
+def test_fwd_rejects_null_and_misaligned_without_a_device(vsa):
+    p = _fake(1 << 20)
+    assert vsa.get_lib().vsa_fwd(None, p, p, p, p, p, None, 1, 512, 2, 128, 8, 2, 0.1, None) == -2
+    assert vsa.get_lib().vsa_fwd(p, p, p, p, p, _fake((1 << 20) + 2), None, 1, 512, 2, 128, 8, 2, 0.1, None) == -3
+    assert vsa.get_lib().vsa_fwd_ex(p, p, p, p, p, p, None, 1, 512, 2, 128, 8, 2, 0.1, 8, None) == -1  # unknown flag
+
+
+def test_route_rejects_bad_arguments_without_a_device(vsa):
+    p = _fake(1 << 20)
+    ws = vsa.route_workspace_size(1, 2, 8, 128)
+    assert vsa.get_lib().vsa_route(p, p, p, p, 1, 512, 2, 128, 8, 9, p, ws, None) == -1  # topk > Nq
+    assert vsa.get_lib().vsa_route(p, p, p, p, 1, 512, 2, 128, 8, 2, p, ws - 1, None) == -4  # short workspace
+    assert vsa.get_lib().vsa_route(p, p, p, p, 1, 512, 2, 128, 8, 2, None, ws, None) == -4
+    assert vsa.get_lib().vsa_route(p, None, p, p, 1, 512, 2, 128, 8, 2, p, ws, None) == -2
+
+
+def test_tile_rejects_bad_arguments_without_a_device(vsa):
+    p = _fake(1 << 20)
+    assert vsa.get_lib().vsa_tile(p, p, 1, 0, 6, 7, 2, 128, None) == -1
+    assert vsa.get_lib().vsa_tile(p, p, 1, 5, 6, 7, 3, 5, None) == -1  # H*D not a multiple of 8
+    assert vsa.get_lib().vsa_tile(None, p, 1, 5, 6, 7, 2, 128, None) == -2
+    assert vsa.get_lib().vsa_untile(p, _fake((1 << 20) + 8), 1, 5, 6, 7, 2, 128, None) == -3
+
+
+def test_product_package_does_not_reach_the_oracle():
+    """The product path never imports or loads the oracle."""
+    pkg = os.path.join(ROOT, "video_block_sparse_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "liboracle" not in text and "from oracle" not in text, f

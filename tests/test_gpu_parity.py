@@ -1,0 +1,247 @@
+"""GPU parity: the CUDA path through the C ABI against the FP64 oracle on the
+same seeded inputs.  Integer and layout work must be bit-exact; the forward
+output must meet the dataset card's pass rule (per-head cosine >= 0.9999,
+max |d| <= 3e-2, mean |d| <= 1e-4, all finite) against the oracle's output
+rounded to bf16; lse is checked against a derived fp32 error bound."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests import common
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def vsa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from video_block_sparse_b200 import build
+
+    build.build()
+    import video_block_sparse_b200 as m
+
+    return m
+
+
+def _no_device_error(vsa):
+    rc, detail = vsa.device_status()
+    assert rc == 0, (rc, detail)
+
+
+# ------------------------------------------------------------------ tiling
+
+@pytest.mark.parametrize("grid,B,H", [((5, 6, 7), 1, 2), ((9, 3, 5), 2, 3), ((1, 1, 1), 1, 1), ((21, 30, 52), 1, 40)])
+def test_tile_untile_bit_exact(vsa, grid, B, H):
+    g = np.random.default_rng(1)
+    L = int(np.prod(grid))
+    x = g.integers(0, 65536, size=(B, L, H, 128), dtype=np.uint16)
+    xt = vsa.tile(common.dev(x), grid)
+    want = oracle.tile(x, *grid)
+    np.testing.assert_array_equal(common.host_bits(xt), want)
+    back = vsa.untile(xt, grid)
+    np.testing.assert_array_equal(common.host_bits(back), x)
+    _no_device_error(vsa)
+
+
+# ------------------------------------------------------------------ routing
+
+@pytest.mark.parametrize("name", ["tiny", "wan480", "adversarial", "wan720"])
+def test_route_bit_exact(vsa, name):
+    cfg = synth.CONFIGS[name]
+    T, Hh, W = cfg.grid
+    q, k, _ = synth.grid_qkv(cfg)
+    qt, kt = oracle.tile(q, T, Hh, W), oracle.tile(k, T, Hh, W)
+    vbs = oracle.cube_counts(T, Hh, W)
+    if cfg.adversarial:
+        ov = synth.adversarial_override(cfg, len(vbs))
+        vbs[ov.cubes] = np.minimum(vbs[ov.cubes], ov.counts)
+    want = oracle.route(qt, kt, vbs, cfg.topk)
+    got = vsa.route(common.dev(qt), common.dev(kt), torch.from_numpy(vbs).cuda(), cfg.topk)
+    np.testing.assert_array_equal(got.cpu().numpy(), want)
+    _no_device_error(vsa)
+
+
+def test_route_ties_and_empty_cubes(vsa):
+    """Planted equal scores are ordered by cube index; an empty cube has mean 0."""
+    nq, topk = 12, 6
+    b_vals = np.array([3, -1, 7, 7, 0.5, 2, -8, 7, 1, 0.25, 4, 2], dtype=np.float32)
+    q = np.zeros((1, 64 * nq, 2, 128), np.float32)
+    k = np.zeros_like(q)
+    q[:, :, :, 9] = 1.0
+    for c in range(nq):
+        k[0, 64 * c: 64 * c + 64, :, 9] = b_vals[c]
+    vbs = np.full(nq, 64, np.int32)
+    vbs[5] = 0
+    qb, kb = synth.f32_to_bf16_bits(q), synth.f32_to_bf16_bits(k)
+    want = oracle.route(qb, kb, vbs, topk)
+    got = vsa.route(common.dev(qb), common.dev(kb), torch.from_numpy(vbs).cuda(), topk)
+    np.testing.assert_array_equal(got.cpu().numpy(), want)
+    assert want[0, 0, 0].tolist() == [2, 3, 7, 10, 0, 8]
+
+
+# ------------------------------------------------------------------ forward
+
+def _run_fwd(vsa, p: common.Prepared, flags=0):
+    q, k, v = common.dev(p.qt), common.dev(p.kt), common.dev(p.vt)
+    idx = torch.from_numpy(p.idx).cuda()
+    vbs = torch.from_numpy(p.vbs).cuda()
+    out, lse = vsa.fwd(q, k, v, idx, vbs, p.cfg.sm_scale, want_lse=True, flags=flags)
+    torch.cuda.synchronize()
+    _no_device_error(vsa)
+    return out, lse
+
+
+def _check_items(p: common.Prepared, out, lse, items, tag):
+    o64, l64 = oracle.fwd_items(p.qt, p.kt, p.vt, p.idx, p.vbs, p.cfg.sm_scale, items)
+    rows = common.gather_items(out, items)
+    res = common.compare(rows, o64, items[:, 1] + 1000 * items[:, 0])
+    print(f"\n[{tag}] gate {res['gate']}\n[{tag}] vs fp64 {res['fp64']}")
+    assert res["gate"]["ok"], res
+    got_lse = np.stack([lse[b, h, 64 * i: 64 * i + 64].cpu().numpy() for b, h, i in items]).astype(np.float64)
+    fin = np.isfinite(l64)
+    assert np.array_equal(fin, np.isfinite(got_lse))
+    bound = common.lse_bound(p.qt, p.kt, items, p.cfg.sm_scale)
+    assert np.all(np.abs(got_lse[fin] - l64[fin]) <= bound[fin]), float(np.max(np.abs(got_lse[fin] - l64[fin])))
+
+
+def test_fwd_tiny_precise_all_rows(vsa):
+    p = common.prepare("tiny")
+    out, lse = _run_fwd(vsa, p, flags=vsa.FWD_PRECISE_P)
+    items = oracle.all_items(p.cfg.B, p.cfg.H, p.nq)
+    _check_items(p, out, lse, items, "tiny/precise")
+
+
+def test_fwd_mid_ragged_all_rows(vsa):
+    """Several tiles and ragged cubes on every axis, every row checked."""
+    p = common.prepare("wan480", H=3, grid=(9, 10, 11), topk=7, B=2)
+    for flags in (0, vsa.FWD_PRECISE_P):
+        out, lse = _run_fwd(vsa, p, flags=flags)
+        items = oracle.all_items(p.cfg.B, p.cfg.H, p.nq)
+        _check_items(p, out, lse, items, f"mid/flags{flags}")
+
+
+@pytest.mark.parametrize("name,n", [("wan480", 120), ("adversarial", 160), ("sweep32", 60), ("sweep156", 40)])
+def test_fwd_full_size_sampled(vsa, name, n):
+    p = common.prepare(name)
+    out, lse = _run_fwd(vsa, p)
+    assert bool(torch.isfinite(out).all())
+    must = []
+    if p.cfg.adversarial:
+        must = [(0, h, i) for h in synth.ADV_T_HEADS for i in (0, 311, 623)]
+        must += [(0, synth.ADV_FORCED_HEAD, i) for i in range(0, 624, 40)]
+    items = common.sample_items(p.cfg.B, p.cfg.H, p.nq, n, seed=3, must=must)
+    _check_items(p, out, lse, items, name)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,n", [("wan720", 60), ("sweep312", 24), ("dense624", 16)])
+def test_fwd_large_sampled(vsa, name, n):
+    p = common.prepare(name)
+    out, lse = _run_fwd(vsa, p)
+    assert bool(torch.isfinite(out).all())
+    items = common.sample_items(p.cfg.B, p.cfg.H, p.nq, n, seed=4)
+    _check_items(p, out, lse, items, name)
+
+
+def test_fwd_dense_matches_library_attention(vsa):
+    """topk = Nq with every cube full is dense attention: cross-check with torch SDPA."""
+    g = np.random.default_rng(5)
+    nq, H = 6, 2
+    x = [synth.f32_to_bf16_bits(g.standard_normal((1, 64 * nq, H, 128)).astype(np.float32)) for _ in range(3)]
+    q, k, v = (common.dev(a) for a in x)
+    idx = torch.arange(nq, dtype=torch.int32).repeat(1, H, nq, 1).cuda().contiguous()
+    vbs = torch.full((nq,), 64, dtype=torch.int32).cuda()
+    out = vsa.fwd(q, k, v, idx, vbs, 128 ** -0.5, flags=vsa.FWD_PRECISE_P)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q.permute(0, 2, 1, 3).float(), k.permute(0, 2, 1, 3).float(), v.permute(0, 2, 1, 3).float(),
+        scale=128 ** -0.5).permute(0, 2, 1, 3)
+    assert float((out.float() - ref).abs().max()) < 1e-2
+
+
+# ------------------------------------------------------------------ edge cases
+
+def _small(seed, nq=5, H=2, topk=3, B=1, vbs=None, dup=False):
+    g = np.random.default_rng(seed)
+    x = [synth.f32_to_bf16_bits((g.standard_normal((B, 64 * nq, H, 128)) * 2).astype(np.float32)) for _ in range(3)]
+    if vbs is None:
+        vbs = g.integers(0, 65, size=nq).astype(np.int32)
+    idx = synth.random_topk(seed, B, H, nq, topk, distinct=not dup)
+    cfg = synth.Config("edge", B=B, H=H, grid=(4, 4, 4 * nq), topk=topk, kind="tiny")
+    return common.Prepared(cfg, x[0], x[1], x[2], np.asarray(vbs, np.int32), idx)
+
+
+@pytest.mark.parametrize("seed,topk,dup", [(0, 1, False), (1, 3, False), (2, 5, True), (3, 4, True)])
+def test_fwd_edge_lists(vsa, seed, topk, dup):
+    p = _small(seed, topk=topk, dup=dup, vbs=[64, 1, 17, 33, 48][:5])
+    for flags in (0, vsa.FWD_PRECISE_P):
+        out, lse = _run_fwd(vsa, p, flags)
+        _check_items(p, out, lse, oracle.all_items(1, 2, 5), f"edge{seed}/{flags}")
+
+
+def test_fwd_all_masked_rows(vsa):
+    p = _small(10, nq=3, H=1, topk=2, vbs=[0, 0, 64])
+    p.idx[:] = np.array([[[[0, 1], [2, 0], [1, 1]]]], np.int32)
+    out, lse = _run_fwd(vsa, p)
+    o = out.float().cpu().numpy()
+    ls = lse.cpu().numpy()
+    assert np.all(o[0, 0:64] == 0) and np.all(ls[0, 0, 0:64] == -np.inf)
+    assert np.all(o[0, 128:] == 0) and np.all(ls[0, 0, 128:] == -np.inf)
+    assert np.all(np.isfinite(ls[0, 0, 64:128]))
+
+
+def test_fwd_nan_pads_do_not_leak(vsa):
+    p = _small(11, vbs=[64, 10, 33, 1, 0])
+    out0, lse0 = _run_fwd(vsa, p)
+    for c in range(5):
+        p.kt[0, 64 * c + p.vbs[c]: 64 * c + 64] = 0x7FC0  # NaN
+        p.vt[0, 64 * c + p.vbs[c]: 64 * c + 64] = 0xFF80  # -inf
+    out1, lse1 = _run_fwd(vsa, p)
+    assert torch.equal(out0.view(torch.int16), out1.view(torch.int16))
+    assert torch.equal(lse0, lse1)
+
+
+def test_fwd_deterministic(vsa):
+    p = _small(12, nq=8, H=3, topk=4)
+    a, la = _run_fwd(vsa, p)
+    b, lb = _run_fwd(vsa, p)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16)) and torch.equal(la, lb)
+
+
+def test_fwd_permuted_lists_agree(vsa):
+    p = _small(13, nq=6, H=2, topk=4)
+    a, _ = _run_fwd(vsa, p)
+    p.idx = p.idx[..., ::-1].copy()
+    b, _ = _run_fwd(vsa, p)
+    assert float((a.float() - b.float()).abs().max()) <= 2 ** -7 * float(a.float().abs().max())
+
+
+def test_fwd_bad_index_latches_device_error(vsa):
+    p = _small(14, nq=4, H=1, topk=2, vbs=[64, 64, 64, 64])
+    p.idx[0, 0, 1, 1] = 7  # out of range: the kernel skips it and latches error 1
+    q, k, v = common.dev(p.qt), common.dev(p.kt), common.dev(p.vt)
+    vsa.fwd(q, k, v, torch.from_numpy(p.idx).cuda(), torch.from_numpy(p.vbs).cuda(), 0.1)
+    rc, detail = vsa.device_status()
+    assert rc == -7 and detail == 1
+    assert vsa.device_status() == (0, 0)  # reading clears the word
+    vbs = torch.tensor([64, 65, 64, 64], dtype=torch.int32).cuda()
+    p.idx[0, 0, 1, 1] = 1
+    vsa.fwd(q, k, v, torch.from_numpy(p.idx).cuda(), vbs, 0.1)
+    rc, detail = vsa.device_status()
+    assert rc == -7 and detail == 2
+
+
+def test_fwd_rejects_bad_calls(vsa):
+    p = _small(15, nq=4, H=1, topk=2)
+    q, k, v = common.dev(p.qt), common.dev(p.kt), common.dev(p.vt)
+    idx, vbs = torch.from_numpy(p.idx).cuda(), torch.from_numpy(p.vbs).cuda()
+    with pytest.raises(vsa.VSAError):
+        vsa.fwd(q[:, :, :, :64].contiguous(), k, v, idx, vbs)
+    with pytest.raises(ValueError):
+        vsa.fwd(q.float(), k, v, idx, vbs)

@@ -1,0 +1,192 @@
+"""Python binding of libvsa, the B200 (sm_100a) library for the fine stage of
+Video Sparse Attention.
+
+Argument marshalling only: every step runs in the CUDA kernels behind the C
+ABI declared in ``include/vsa.h``.  Tensors are torch CUDA tensors (torch is
+used for device memory and streams); each call passes raw pointers, sizes
+and the current stream to the library and raises ``VSAError`` on a non-zero
+status.  There is no CPU or fallback path: if ``libvsa.so`` is missing or
+cannot be loaded, the first call raises ImportError.
+
+Names follow the C ABI: ``fwd`` (vsa_fwd / vsa_fwd_ex), ``route``,
+``tile``, ``untile``, ``cube_counts``, ``device_status``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libvsa.so")
+
+FWD_DEFAULT = 0
+FWD_PRECISE_P = 1
+
+_STATUS = {0: "VSA_OK", -1: "VSA_ERR_ARG", -2: "VSA_ERR_NULL", -3: "VSA_ERR_ALIGN", -4: "VSA_ERR_WORKSPACE",
+           -5: "VSA_ERR_ARCH", -6: "VSA_ERR_LAUNCH", -7: "VSA_ERR_DEVICE"}
+
+# every symbol include/vsa.h declares
+EXPORTS = ("vsa_status_string", "vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_route_workspace_size",
+           "vsa_route", "vsa_cube_counts", "vsa_tile", "vsa_untile", "vsa_device_status")
+
+
+class VSAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {_STATUS.get(status, status)}")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libvsa.so not built at {LIB_PATH}; run `python -m video_block_sparse_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.vsa_status_string.argtypes = [I]
+    lib.vsa_status_string.restype = ctypes.c_char_p
+    lib.vsa_can_implement.argtypes = [I, I]
+    lib.vsa_fwd.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
+    lib.vsa_fwd_ex.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
+    lib.vsa_route_workspace_size.argtypes = [I, I, I, I]
+    lib.vsa_route_workspace_size.restype = Z
+    lib.vsa_route.argtypes = [P, P, P, P, I, I, I, I, I, I, P, Z, P]
+    lib.vsa_cube_counts.argtypes = [I, I, I, P, P]
+    lib.vsa_tile.argtypes = [P, P, I, I, I, I, I, I, P]
+    lib.vsa_untile.argtypes = [P, P, I, I, I, I, I, I, P]
+    lib.vsa_device_status.argtypes = [P, P]
+    for name in ("vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_route", "vsa_cube_counts", "vsa_tile",
+                 "vsa_untile", "vsa_device_status"):
+        getattr(lib, name).restype = I
+    return lib
+
+
+_LIB = None
+
+
+def get_lib():
+    """The loaded libvsa (ctypes); raises ImportError if it is not built."""
+    global _LIB
+    if _LIB is None:
+        _LIB = _load()
+    return _LIB
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libvsa takes CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("libvsa takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise VSAError(rc, what)
+
+
+def _bf16(t: torch.Tensor, name: str):
+    if t.dtype != torch.bfloat16:
+        raise ValueError(f"{name} must be bfloat16")
+
+
+def status_string(status: int) -> str:
+    return get_lib().vsa_status_string(status).decode()
+
+
+def can_implement(D: int, sm_version: int) -> bool:
+    return bool(get_lib().vsa_can_implement(D, sm_version))
+
+
+def cube_counts(T: int, Hh: int, W: int) -> torch.Tensor:
+    """Host int32 [Nq] valid-token counts of the 4x4x4 cubes of a T x Hh x W grid."""
+    nq = ctypes.c_int(0)
+    _check(get_lib().vsa_cube_counts(T, Hh, W, None, ctypes.byref(nq)), "vsa_cube_counts")
+    vbs = torch.empty(nq.value, dtype=torch.int32)
+    _check(get_lib().vsa_cube_counts(T, Hh, W, ctypes.c_void_p(vbs.data_ptr()), ctypes.byref(nq)), "vsa_cube_counts")
+    return vbs
+
+
+def tile(x_grid: torch.Tensor, grid, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """[B, T*Hh*W, H, D] raster -> [B, 64*Nq, H, D] cube-major (pads zero)."""
+    T, Hh, W = grid
+    B, L, H, D = x_grid.shape
+    _bf16(x_grid, "x_grid")
+    nq = ctypes.c_int(0)
+    _check(get_lib().vsa_cube_counts(T, Hh, W, None, ctypes.byref(nq)), "vsa_cube_counts")
+    if out is None:
+        out = torch.empty(B, 64 * nq.value, H, D, dtype=x_grid.dtype, device=x_grid.device)
+    if L != T * Hh * W or out.shape != (B, 64 * nq.value, H, D):
+        raise ValueError("tile: shape mismatch")
+    _check(get_lib().vsa_tile(_ptr(x_grid), _ptr(out), B, T, Hh, W, H, D, _stream(stream)), "vsa_tile")
+    return out
+
+
+def untile(x_tiled: torch.Tensor, grid, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """[B, 64*Nq, H, D] cube-major -> [B, T*Hh*W, H, D] raster."""
+    T, Hh, W = grid
+    B, S, H, D = x_tiled.shape
+    _bf16(x_tiled, "x_tiled")
+    if out is None:
+        out = torch.empty(B, T * Hh * W, H, D, dtype=x_tiled.dtype, device=x_tiled.device)
+    if out.shape != (B, T * Hh * W, H, D):
+        raise ValueError("untile: shape mismatch")
+    _check(get_lib().vsa_untile(_ptr(x_tiled), _ptr(out), B, T, Hh, W, H, D, _stream(stream)), "vsa_untile")
+    return out
+
+
+def route_workspace_size(B: int, H: int, nq: int, D: int = 128) -> int:
+    return int(get_lib().vsa_route_workspace_size(B, H, nq, D))
+
+
+def route(q: torch.Tensor, k: torch.Tensor, vbs: torch.Tensor, topk: int, out: torch.Tensor | None = None,
+          workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """topk_idx [B, H, Nq, topk] int32 from cube-mean q.k scores."""
+    B, S, H, D = q.shape
+    nq = S // 64
+    _bf16(q, "q")
+    _bf16(k, "k")
+    if out is None:
+        out = torch.empty(B, H, nq, topk, dtype=torch.int32, device=q.device)
+    need = route_workspace_size(B, H, nq, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(get_lib().vsa_route(_ptr(q), _ptr(k), _ptr(vbs), _ptr(out), B, S, H, D, nq, topk, _ptr(workspace),
+                         workspace.numel() * workspace.element_size(), _stream(stream)), "vsa_route")
+    return out
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk_idx: torch.Tensor, vbs: torch.Tensor,
+        sm_scale: float | None = None, out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+        want_lse: bool = False, flags: int = FWD_DEFAULT, stream=None):
+    """Fine block-sparse attention forward; returns out (and lse if asked)."""
+    B, S, H, D = q.shape
+    nq = S // 64
+    topk = topk_idx.shape[-1]
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _bf16(t, n)
+    if topk_idx.dtype != torch.int32 or vbs.dtype != torch.int32:
+        raise ValueError("topk_idx and vbs must be int32")
+    if sm_scale is None:
+        sm_scale = D ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, H, S, dtype=torch.float32, device=q.device)
+    _check(get_lib().vsa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(topk_idx), _ptr(vbs), _ptr(out), _ptr(lse), B, S, H, D,
+                          nq, topk, float(sm_scale), int(flags), _stream(stream)), "vsa_fwd")
+    return (out, lse) if (want_lse or lse is not None) else out
+
+
+def device_status(stream=None) -> tuple[int, int]:
+    """Synchronise the stream and read (and clear) the device error word."""
+    detail = ctypes.c_int(0)
+    rc = get_lib().vsa_device_status(_stream(stream), ctypes.byref(detail))
+    return rc, detail.value

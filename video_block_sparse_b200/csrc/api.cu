@@ -1,0 +1,205 @@
+// C ABI of libvsa (declared in include/vsa.h): argument validation, the
+// device error word, and dispatch to the kernel launchers.  Nothing here
+// allocates memory or synchronises, except vsa_device_status.
+#include "vsa.h"
+
+#include "internal.h"
+
+#include <climits>
+#include <cstdint>
+
+namespace {
+
+// One error word per device; kernels latch the first error with atomicCAS.
+__device__ int g_device_error;
+
+constexpr int kMaxDevices = 64;
+int* g_err_ptr[kMaxDevices];
+int g_sm_version[kMaxDevices];
+
+int current_device(int* dev)
+{
+    if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= kMaxDevices) return VSA_ERR_LAUNCH;
+    return VSA_OK;
+}
+
+int device_sm(int dev)
+{
+    if (g_sm_version[dev] == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return -1;
+        g_sm_version[dev] = major * 10 + minor;
+    }
+    return g_sm_version[dev];
+}
+
+// Address of this device's error word (looked up once per device).
+int device_error_word(int** out)
+{
+    int dev;
+    if (current_device(&dev) != VSA_OK) return VSA_ERR_LAUNCH;
+    if (g_err_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return VSA_ERR_LAUNCH;
+        g_err_ptr[dev] = static_cast<int*>(p);
+    }
+    *out = g_err_ptr[dev];
+    return VSA_OK;
+}
+
+int check_arch()
+{
+    int dev;
+    if (current_device(&dev) != VSA_OK) return VSA_ERR_LAUNCH;
+    return device_sm(dev) == 100 ? VSA_OK : VSA_ERR_ARCH;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int launch_status(cudaError_t e) { return e == cudaSuccess ? VSA_OK : VSA_ERR_LAUNCH; }
+
+// Shared checks of the attention-shaped calls.
+int check_bshd(int B, int S, int H, int D, int Nq)
+{
+    if (B < 1 || H < 1 || Nq < 1 || D != 128) return VSA_ERR_ARG;
+    if ((int64_t)Nq * 64 != (int64_t)S) return VSA_ERR_ARG;
+    if ((int64_t)B * S * H * D > (int64_t)INT32_MAX * 8) return VSA_ERR_ARG;
+    if ((int64_t)B * H * Nq > INT32_MAX) return VSA_ERR_ARG;
+    return VSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* vsa_status_string(int status)
+{
+    switch (status) {
+    case VSA_OK: return "VSA_OK";
+    case VSA_ERR_ARG: return "VSA_ERR_ARG: size or count out of range";
+    case VSA_ERR_NULL: return "VSA_ERR_NULL: required pointer is NULL";
+    case VSA_ERR_ALIGN: return "VSA_ERR_ALIGN: pointer not 16-byte aligned";
+    case VSA_ERR_WORKSPACE: return "VSA_ERR_WORKSPACE: workspace missing or too small";
+    case VSA_ERR_ARCH: return "VSA_ERR_ARCH: device is not sm_100";
+    case VSA_ERR_LAUNCH: return "VSA_ERR_LAUNCH: CUDA runtime error";
+    case VSA_ERR_DEVICE: return "VSA_ERR_DEVICE: a kernel latched an error";
+    default: return "unknown vsa status";
+    }
+}
+
+int vsa_can_implement(int D, int sm_version) { return (D == 128 && sm_version == 100) ? 1 : 0; }
+
+int vsa_fwd_ex(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const int32_t* topk_idx, const int32_t* vbs,
+               vsa_bf16* out, float* lse, int B, int S, int H, int D, int Nq, int topk, float sm_scale, int flags,
+               cudaStream_t stream)
+{
+    int rc = check_bshd(B, S, H, D, Nq);
+    if (rc != VSA_OK) return rc;
+    if (topk < 1 || (flags & ~VSA_FWD_PRECISE_P) != 0) return VSA_ERR_ARG;
+    if ((int64_t)B * H * Nq * topk > INT32_MAX) return VSA_ERR_ARG;
+    if (!q || !k || !v || !topk_idx || !vbs || !out) return VSA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(topk_idx) ||
+        !aligned16(vbs) || (lse && !aligned16(lse)))
+        return VSA_ERR_ALIGN;
+    if ((rc = check_arch()) != VSA_OK) return rc;
+    int* err;
+    if ((rc = device_error_word(&err)) != VSA_OK) return rc;
+    return launch_status(vsa::launch_fwd_mma(q, k, v, topk_idx, vbs, out, lse, B, S, H, Nq, topk, sm_scale,
+                                             (flags & VSA_FWD_PRECISE_P) != 0, err, stream));
+}
+
+int vsa_fwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const int32_t* topk_idx, const int32_t* vbs,
+            vsa_bf16* out, float* lse, int B, int S, int H, int D, int Nq, int topk, float sm_scale,
+            cudaStream_t stream)
+{
+    return vsa_fwd_ex(q, k, v, topk_idx, vbs, out, lse, B, S, H, D, Nq, topk, sm_scale, VSA_FWD_DEFAULT, stream);
+}
+
+size_t vsa_route_workspace_size(int B, int H, int Nq, int D)
+{
+    if (B < 1 || H < 1 || Nq < 1 || D < 1) return 0;
+    return vsa::route_workspace_bytes(B, H, Nq, D);
+}
+
+int vsa_route(const vsa_bf16* q, const vsa_bf16* k, const int32_t* vbs, int32_t* topk_idx, int B, int S, int H,
+              int D, int Nq, int topk, void* workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    int rc = check_bshd(B, S, H, D, Nq);
+    if (rc != VSA_OK) return rc;
+    if (topk < 1 || topk > Nq || Nq > 4096) return VSA_ERR_ARG;
+    if (!q || !k || !vbs || !topk_idx) return VSA_ERR_NULL;
+    if (!workspace || workspace_bytes < vsa::route_workspace_bytes(B, H, Nq, D)) return VSA_ERR_WORKSPACE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(vbs) || !aligned16(topk_idx) || !aligned16(workspace))
+        return VSA_ERR_ALIGN;
+    if ((rc = check_arch()) != VSA_OK) return rc;
+    int* err;
+    if ((rc = device_error_word(&err)) != VSA_OK) return rc;
+    return launch_status(vsa::launch_route(q, k, vbs, topk_idx, B, S, H, Nq, topk, workspace, err, stream));
+}
+
+int vsa_cube_counts(int T, int Hh, int W, int32_t* vbs_host, int* Nq_out)
+{
+    if (T < 1 || Hh < 1 || W < 1) return VSA_ERR_ARG;
+    const int64_t nq = (int64_t)((T + 3) / 4) * ((Hh + 3) / 4) * ((W + 3) / 4);
+    if (nq > INT32_MAX / 64) return VSA_ERR_ARG;
+    if (Nq_out) *Nq_out = (int)nq;
+    if (!vbs_host) return VSA_OK;
+    const vsa::CubeGeom g = vsa::make_geom(T, Hh, W);
+    for (int ct = 0; ct < g.nct; ++ct)
+        for (int ch = 0; ch < g.nch; ++ch)
+            for (int cw = 0; cw < g.ncw; ++cw) {
+                const int et = T - 4 * ct < 4 ? T - 4 * ct : 4;
+                const int eh = Hh - 4 * ch < 4 ? Hh - 4 * ch : 4;
+                const int ew = W - 4 * cw < 4 ? W - 4 * cw : 4;
+                vbs_host[(ct * g.nch + ch) * g.ncw + cw] = et * eh * ew;
+            }
+    return VSA_OK;
+}
+
+static int check_tile_args(const void* a, const void* b, int B, int T, int Hh, int W, int H, int D)
+{
+    if (B < 1 || T < 1 || Hh < 1 || W < 1 || H < 1 || D < 1) return VSA_ERR_ARG;
+    if (((int64_t)H * D) % 8 != 0 || (int64_t)H * D > INT32_MAX) return VSA_ERR_ARG;
+    int nq = 0;
+    if (vsa_cube_counts(T, Hh, W, nullptr, &nq) != VSA_OK) return VSA_ERR_ARG;
+    if ((int64_t)B * 64 * nq * H * D > ((int64_t)1 << 40)) return VSA_ERR_ARG;
+    if (!a || !b) return VSA_ERR_NULL;
+    if (!aligned16(a) || !aligned16(b)) return VSA_ERR_ALIGN;
+    return check_arch();
+}
+
+int vsa_tile(const vsa_bf16* x_grid, vsa_bf16* x_tiled, int B, int T, int Hh, int W, int H, int D,
+             cudaStream_t stream)
+{
+    int rc = check_tile_args(x_grid, x_tiled, B, T, Hh, W, H, D);
+    if (rc != VSA_OK) return rc;
+    return launch_status(vsa::launch_tile(x_grid, x_tiled, B, vsa::make_geom(T, Hh, W), H * D, stream));
+}
+
+int vsa_untile(const vsa_bf16* x_tiled, vsa_bf16* x_grid, int B, int T, int Hh, int W, int H, int D,
+               cudaStream_t stream)
+{
+    int rc = check_tile_args(x_tiled, x_grid, B, T, Hh, W, H, D);
+    if (rc != VSA_OK) return rc;
+    return launch_status(vsa::launch_untile(x_tiled, x_grid, B, vsa::make_geom(T, Hh, W), H * D, stream));
+}
+
+int vsa_device_status(cudaStream_t stream, int* detail)
+{
+    if (detail) *detail = 0;
+    int* err;
+    int rc = device_error_word(&err);
+    if (rc != VSA_OK) return rc;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return VSA_ERR_LAUNCH;
+    int h = 0;
+    if (cudaMemcpy(&h, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return VSA_ERR_LAUNCH;
+    if (h == 0) return VSA_OK;
+    const int zero = 0;
+    if (cudaMemcpy(err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return VSA_ERR_LAUNCH;
+    if (detail) *detail = h;
+    return VSA_ERR_DEVICE;
+}
+
+}  // extern "C"

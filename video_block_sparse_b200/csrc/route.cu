@@ -1,0 +1,222 @@
+// Cube-mean q.k top-k routing (the VSA "predictor").
+//
+// "align VisualGen VSA with block-sparse FMHA" (TensorRT-LLM PR #7), review
+// excerpts: a cube mean is the sum over the cube's valid tokens divided by the
+// valid count and cast back to the tiled dtype.  "Video Sparse Attention
+// Runner" (TensorRT-Edge docs): block means of K are rounded to bf16 before
+// they are used to route.  The score of query cube i against KV cube j is the
+// dot product of their bf16 means; each query cube keeps the topk best.
+//
+// The arithmetic is fixed so that the selection is exact and reproducible:
+//   mean  = bf16_rne(fp64 sequential sum over u < vbs / vbs)   (0 when vbs = 0)
+//   score = fp64 sequential sum over d = 0..D-1 of qc[d] * kc[d]
+//           (each product of two bf16 values is exact in fp64)
+//   order = score descending, cube index ascending, NaN counted as -inf
+//
+// Kernels:
+//   cube_mean_kernel   one CTA per (cube, batch, tensor); threads own 8
+//                      consecutive (h, d) columns and walk the cube's valid
+//                      rows with 16-byte loads: HBM-bound, reads q and k once.
+//   score_topk_kernel  one CTA per (QB query cubes, head, batch): streams the
+//                      head's kc rows once, keeps QB score rows in shared
+//                      memory as order-preserving 64-bit keys, then one warp
+//                      per query cube bitonic-sorts (key, index) pairs.
+#include "internal.h"
+
+namespace vsa {
+namespace {
+
+constexpr int kD = 128;
+
+__device__ __forceinline__ double bf16_to_f64(uint32_t bits16) { return (double)__uint_as_float(bits16 << 16); }
+
+// Nearest-even rounding of a double to bf16 bits, one rounding step.
+// Normal range: drop the low 45 fraction bits of the binary64 pattern with
+// round-half-even; below 2^-126 the bf16 grid is uniform with step 2^-133.
+__device__ __forceinline__ uint16_t f64_to_bf16_rne(double x)
+{
+    const uint64_t u = (uint64_t)__double_as_longlong(x);
+    const uint16_t sign = (uint16_t)((u >> 48) & 0x8000u);
+    const uint64_t a = u & 0x7FFFFFFFFFFFFFFFull;
+    if (a > 0x7FF0000000000000ull) return 0x7FC0;           // NaN
+    if (a == 0x7FF0000000000000ull) return sign | 0x7F80;   // inf
+    const int e = (int)(a >> 52) - 1023;
+    if (e >= -126) {
+        const uint64_t lsb = (a >> 45) & 1ull;
+        uint64_t r = a + ((1ull << 44) - 1ull) + lsb;
+        r &= ~((1ull << 45) - 1ull);
+        const int e2 = (int)(r >> 52) - 1023;
+        if (e2 > 127) return sign | 0x7F80;
+        return sign | (uint16_t)((uint32_t)(e2 + 127) << 7) | (uint16_t)((r >> 45) & 0x7Fu);
+    }
+    // |x| < 2^-126: multiples of 2^-133; the scaling by 2^133 is exact
+    const double n = rint(__longlong_as_double((long long)a) * 0x1p133);
+    return sign | (uint16_t)n;  // n <= 128; 128 encodes the smallest normal
+}
+
+// x [B, S, H, D] -> xc [B, H, Nq, D]; blockIdx = (cube, batch, tensor)
+__global__ void __launch_bounds__(128) cube_mean_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
+                                                        const int32_t* __restrict__ vbs, uint16_t* __restrict__ qc,
+                                                        uint16_t* __restrict__ kc, int S, int H, int nq, int* err)
+{
+    const int c = blockIdx.x, b = blockIdx.y;
+    const uint16_t* x = blockIdx.z ? k : q;
+    uint16_t* xc = blockIdx.z ? kc : qc;
+    int n = __ldg(vbs + c);
+    if (n < 0 || n > 64) {
+        if (threadIdx.x == 0) atomicCAS(err, 0, (int)kErrVbs);
+        n = 0;
+    }
+    const int row16 = H * kD / 8;
+    const uint4* base = reinterpret_cast<const uint4*>(x + ((int64_t)b * S + 64LL * c) * H * kD);
+    for (int ch = threadIdx.x; ch < row16; ch += blockDim.x) {
+        double acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.0;
+        for (int u = 0; u < n; ++u) {
+            uint4 w = __ldg(base + (int64_t)u * row16 + ch);
+            uint32_t p[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                acc[2 * e] += bf16_to_f64(p[e] & 0xFFFFu);
+                acc[2 * e + 1] += bf16_to_f64(p[e] >> 16);
+            }
+        }
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            uint32_t lo = n ? f64_to_bf16_rne(acc[2 * e] / (double)n) : 0u;
+            uint32_t hi = n ? f64_to_bf16_rne(acc[2 * e + 1] / (double)n) : 0u;
+            o[e] = lo | (hi << 16);
+        }
+        const int h = (ch * 8) / kD, d = (ch * 8) % kD;
+        *reinterpret_cast<uint4*>(xc + (((int64_t)b * H + h) * nq + c) * kD + d) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+// Order-preserving key, inverted so that ascending key = descending score.
+__device__ __forceinline__ uint64_t score_key(double s)
+{
+    uint64_t u = (uint64_t)__double_as_longlong(s);
+    if (s != s) u = 0xFFF0000000000000ull;          // NaN ranks as -inf
+    if (u == 0x8000000000000000ull) u = 0ull;       // -0 ranks as +0
+    const uint64_t ord = (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+    return ~ord;
+}
+
+template <int QB>
+__global__ void __launch_bounds__(256) score_topk_kernel(const uint16_t* __restrict__ qc,
+                                                         const uint16_t* __restrict__ kc, int32_t* __restrict__ topk_idx,
+                                                         int H, int nq, int np, int topk)
+{
+    extern __shared__ __align__(16) uint8_t smem[];
+    double* qd = reinterpret_cast<double*>(smem);                       // [QB][D]
+    uint64_t* keys = reinterpret_cast<uint64_t*>(qd + QB * kD);         // [QB][np]
+    uint16_t* ids = reinterpret_cast<uint16_t*>(keys + (size_t)QB * np);  // [QB][np]
+
+    const int i0 = blockIdx.x * QB, h = blockIdx.y, b = blockIdx.z;
+    const int64_t head = (int64_t)b * H + h;
+    for (int e = threadIdx.x; e < QB * kD; e += blockDim.x) {
+        const int qi = i0 + e / kD;
+        qd[e] = qi < nq ? bf16_to_f64(qc[(head * nq + qi) * kD + (e % kD)]) : 0.0;
+    }
+    __syncthreads();
+
+    const uint4* krow = reinterpret_cast<const uint4*>(kc + head * nq * kD);
+    for (int j = threadIdx.x; j < np; j += blockDim.x) {
+        if (j >= nq) {
+#pragma unroll
+            for (int r = 0; r < QB; ++r) {
+                keys[r * np + j] = ~0ull;
+                ids[r * np + j] = 0xFFFFu;
+            }
+            continue;
+        }
+        double acc[QB];
+#pragma unroll
+        for (int r = 0; r < QB; ++r) acc[r] = 0.0;
+        for (int ch = 0; ch < kD / 8; ++ch) {
+            const uint4 w = __ldg(krow + (int64_t)j * (kD / 8) + ch);
+            const uint32_t p[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const double kv = bf16_to_f64((e & 1) ? (p[e >> 1] >> 16) : (p[e >> 1] & 0xFFFFu));
+#pragma unroll
+                for (int r = 0; r < QB; ++r) acc[r] = __fma_rn(qd[r * kD + ch * 8 + e], kv, acc[r]);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < QB; ++r) {
+            keys[r * np + j] = score_key(acc[r]);
+            ids[r * np + j] = (uint16_t)j;
+        }
+    }
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int r = warp; r < QB; r += blockDim.x / 32) {
+        const int qi = i0 + r;
+        if (qi >= nq) continue;
+        uint64_t* kk = keys + (size_t)r * np;
+        uint16_t* ii = ids + (size_t)r * np;
+        for (int len = 2; len <= np; len <<= 1) {
+            for (int stride = len >> 1; stride > 0; stride >>= 1) {
+                for (int a = lane; a < np; a += 32) {
+                    const int p = a ^ stride;
+                    if (p > a) {
+                        const uint64_t ka = kk[a], kp = kk[p];
+                        const uint16_t ia = ii[a], ip = ii[p];
+                        const bool a_after = (ka > kp) || (ka == kp && ia > ip);
+                        const bool ascending = (a & len) == 0;
+                        if (a_after == ascending) {
+                            kk[a] = kp;
+                            kk[p] = ka;
+                            ii[a] = ip;
+                            ii[p] = ia;
+                        }
+                    }
+                }
+                __syncwarp();
+            }
+        }
+        int32_t* dst = topk_idx + (head * nq + qi) * topk;
+        for (int t = lane; t < topk; t += 32) dst[t] = ii[t];
+    }
+}
+
+}  // namespace
+
+size_t route_workspace_bytes(int B, int H, int nq, int D)
+{
+    return 2 * (size_t)B * H * nq * D * sizeof(uint16_t);
+}
+
+cudaError_t launch_route(const uint16_t* q, const uint16_t* k, const int32_t* vbs, int32_t* topk_idx, int B, int S,
+                         int H, int nq, int topk, void* workspace, int* err, cudaStream_t s)
+{
+    uint16_t* qc = static_cast<uint16_t*>(workspace);
+    uint16_t* kc = qc + (size_t)B * H * nq * kD;
+    cube_mean_kernel<<<dim3(nq, B, 2), 128, 0, s>>>(q, k, vbs, qc, kc, S, H, nq, err);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    int np = 32;
+    while (np < nq) np <<= 1;
+    if (np <= 2048) {
+        constexpr int QB = 8;
+        size_t smem = (size_t)QB * kD * 8 + (size_t)QB * np * 10;
+        auto kern = score_topk_kernel<QB>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kern<<<dim3((nq + QB - 1) / QB, H, B), 256, smem, s>>>(qc, kc, topk_idx, H, nq, np, topk);
+    } else {
+        constexpr int QB = 4;
+        size_t smem = (size_t)QB * kD * 8 + (size_t)QB * np * 10;
+        auto kern = score_topk_kernel<QB>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kern<<<dim3((nq + QB - 1) / QB, H, B), 256, smem, s>>>(qc, kc, topk_idx, H, nq, np, topk);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace vsa
