@@ -142,6 +142,36 @@ VSA_API int vsa_route(const vsa_bf16 *q, const vsa_bf16 *k, const int32_t *vbs, 
               int D, int Nq, int topk, void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * vsa_route_noalloc -- vsa_route for callers that cannot allocate device
+ * memory.  The pages have no counterpart of this call; it exists for this
+ * library's users.
+ *
+ * Some callers cannot call cudaMalloc (or any allocator) at the point where
+ * they route: code running inside a CUDA graph capture whose capture mode
+ * forbids allocation, plugins and runtimes that are handed only their
+ * input/output buffers by a host framework, and deployments that fix every
+ * device allocation at start-up.  This entry point takes the same arguments
+ * as vsa_route minus the workspace: its scratch (the bf16 cube means of q
+ * and k, 2*B*H*Nq*D*2 bytes) lives in a 16 MiB array that is part of the
+ * library's device code.  Every GPU that loads the library holds that array
+ * until the process exits.
+ *
+ *  - Limit: 2*B*H*Nq*D*2 <= 16 MiB (B*H*Nq <= 32768 at D = 128); larger
+ *    problems return VSA_ERR_WORKSPACE and launch nothing.
+ *  - The first call on a device looks up the array's device address with
+ *    cudaGetSymbolAddress while that device is current; make that first call
+ *    before any stream capture on that device.
+ *  - All calls share the one array and it keeps the last call's contents.
+ *    Calls whose kernels may overlap on the GPU (different streams without
+ *    ordering between them) race on it; serialise them on one stream.  The
+ *    routing overwrites every scratch byte it reads, so nothing needs
+ *    clearing between calls.
+ *  - Otherwise as vsa_route: same arguments, checks, results and errors.
+ * ---------------------------------------------------------------------- */
+VSA_API int vsa_route_noalloc(const vsa_bf16 *q, const vsa_bf16 *k, const int32_t *vbs, int32_t *topk_idx, int B,
+                              int S, int H, int D, int Nq, int topk, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * Cube-major layout.  Dataset card "wan2.2_production_values", section
  * "Shapes": a T x Hh x W latent grid is cut into 4x4x4 cubes,
  * Nq = ceil(T/4) * ceil(Hh/4) * ceil(W/4), S = 64 * Nq.  Cubes are ordered

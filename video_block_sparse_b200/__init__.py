@@ -29,7 +29,7 @@ _STATUS = {0: "VSA_OK", -1: "VSA_ERR_ARG", -2: "VSA_ERR_NULL", -3: "VSA_ERR_ALIG
 
 # every symbol include/vsa.h declares
 EXPORTS = ("vsa_status_string", "vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_route_workspace_size",
-           "vsa_route", "vsa_cube_counts", "vsa_tile", "vsa_untile", "vsa_device_status")
+           "vsa_route", "vsa_route_noalloc", "vsa_cube_counts", "vsa_tile", "vsa_untile", "vsa_device_status")
 
 
 class VSAError(RuntimeError):
@@ -51,11 +51,13 @@ def _load():
     lib.vsa_route_workspace_size.argtypes = [I, I, I, I]
     lib.vsa_route_workspace_size.restype = Z
     lib.vsa_route.argtypes = [P, P, P, P, I, I, I, I, I, I, P, Z, P]
+    lib.vsa_route_noalloc.argtypes = [P, P, P, P, I, I, I, I, I, I, P]
     lib.vsa_cube_counts.argtypes = [I, I, I, P, P]
     lib.vsa_tile.argtypes = [P, P, I, I, I, I, I, I, P]
     lib.vsa_untile.argtypes = [P, P, I, I, I, I, I, I, P]
     lib.vsa_device_status.argtypes = [P, P]
-    for name in ("vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_route", "vsa_cube_counts", "vsa_tile",
+    for name in ("vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_route", "vsa_route_noalloc", "vsa_cube_counts",
+                 "vsa_tile",
                  "vsa_untile", "vsa_device_status"):
         getattr(lib, name).restype = I
     return lib
@@ -160,6 +162,18 @@ def route(q: torch.Tensor, k: torch.Tensor, vbs: torch.Tensor, topk: int, out: t
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     _check(get_lib().vsa_route(_ptr(q), _ptr(k), _ptr(vbs), _ptr(out), B, S, H, D, nq, topk, _ptr(workspace),
                          workspace.numel() * workspace.element_size(), _stream(stream)), "vsa_route")
+    return out
+
+
+def route_noalloc(q: torch.Tensor, k: torch.Tensor, vbs: torch.Tensor, topk: int, out: torch.Tensor,
+                  stream=None) -> torch.Tensor:
+    """vsa_route_noalloc: routing with the library's built-in scratch (no
+    allocation by the library; `out` must be provided by the caller)."""
+    B, S, H, D = q.shape
+    _bf16(q, "q")
+    _bf16(k, "k")
+    _check(get_lib().vsa_route_noalloc(_ptr(q), _ptr(k), _ptr(vbs), _ptr(out), B, S, H, D, S // 64, topk,
+                                       _stream(stream)), "vsa_route_noalloc")
     return out
 
 
