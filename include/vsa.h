@@ -103,7 +103,11 @@ enum vsa_fwd_flags {
      * (P = hi + lo) instead of one bf16 value: about 2^-16 relative weight
      * error instead of 2^-9, for workloads whose softmax is spread over many
      * keys.  Costs one extra P.V product per tile. */
-    VSA_FWD_PRECISE_P = 1
+    VSA_FWD_PRECISE_P = 1,
+    /* Run the warp-level mma.sync kernel instead of the tcgen05/TMEM/TMA
+     * kernel: the legacy tensor-core path, kept as the measured baseline the
+     * tcgen05 kernel is compared against.  Same results contract. */
+    VSA_FWD_LEGACY_MMA = 2
 };
 
 /* vsa_fwd with option flags (vsa_fwd == vsa_fwd_ex with VSA_FWD_DEFAULT). */

@@ -375,3 +375,20 @@ def test_oracle_rejects_bad_arguments(oracle_lib):
         oracle_lib.fwd(q, k, v, bad, vbs, 0.1)
     with pytest.raises(ValueError):
         oracle_lib.fwd(q, k, v, idx, np.array([65, 1, 1], np.int32), 0.1)
+
+
+# ---------------------------------------------------------------- comparator
+
+def test_near_tie_reference_accepts_only_midpoint_flips():
+    """The parity comparator accepts the other bf16 neighbour only when the exact
+    value sits within 1/32 ulp of the midpoint; any other difference stays."""
+    from tests import common
+
+    ulp = 2.0 ** -5  # bf16 spacing in [4, 8)
+    exact = np.array([4.0 + 0.5 * ulp + 1e-4 * ulp,   # just above the midpoint: ideal = 4 + ulp
+                      4.0 + 0.5 * ulp + 0.2 * ulp,    # well above: ideal = 4 + ulp
+                      4.0 + 0.5 * ulp + 1e-4 * ulp])  # just above, but the GPU is 2 ulps off
+    gpu = np.array([4.0, 4.0, 4.0 - ulp], dtype=np.float32)
+    ref, n = common.near_tie_reference(gpu, exact)
+    assert n == 1
+    assert ref[0] == 4.0 and ref[1] == np.float32(4.0 + ulp) and ref[2] == np.float32(4.0 + ulp)

@@ -23,6 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libvsa.so")
 
 FWD_DEFAULT = 0
 FWD_PRECISE_P = 1
+FWD_LEGACY_MMA = 2
 
 _STATUS = {0: "VSA_OK", -1: "VSA_ERR_ARG", -2: "VSA_ERR_NULL", -3: "VSA_ERR_ALIGN", -4: "VSA_ERR_WORKSPACE",
            -5: "VSA_ERR_ARCH", -6: "VSA_ERR_LAUNCH", -7: "VSA_ERR_DEVICE"}

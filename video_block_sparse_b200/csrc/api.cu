@@ -97,7 +97,7 @@ int vsa_fwd_ex(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const in
 {
     int rc = check_bshd(B, S, H, D, Nq);
     if (rc != VSA_OK) return rc;
-    if (topk < 1 || (flags & ~VSA_FWD_PRECISE_P) != 0) return VSA_ERR_ARG;
+    if (topk < 1 || (flags & ~(VSA_FWD_PRECISE_P | VSA_FWD_LEGACY_MMA)) != 0) return VSA_ERR_ARG;
     if ((int64_t)B * H * Nq * topk > INT32_MAX) return VSA_ERR_ARG;
     if (!q || !k || !v || !topk_idx || !vbs || !out) return VSA_ERR_NULL;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(topk_idx) ||
@@ -106,8 +106,12 @@ int vsa_fwd_ex(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const in
     if ((rc = check_arch()) != VSA_OK) return rc;
     int* err;
     if ((rc = device_error_word(&err)) != VSA_OK) return rc;
-    return launch_status(vsa::launch_fwd_mma(q, k, v, topk_idx, vbs, out, lse, B, S, H, Nq, topk, sm_scale,
-                                             (flags & VSA_FWD_PRECISE_P) != 0, err, stream));
+    const bool precise = (flags & VSA_FWD_PRECISE_P) != 0;
+    if (flags & VSA_FWD_LEGACY_MMA)
+        return launch_status(
+            vsa::launch_fwd_mma(q, k, v, topk_idx, vbs, out, lse, B, S, H, Nq, topk, sm_scale, precise, err, stream));
+    return launch_status(
+        vsa::launch_fwd_tc(q, k, v, topk_idx, vbs, out, lse, B, S, H, Nq, topk, sm_scale, precise, err, stream));
 }
 
 int vsa_fwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const int32_t* topk_idx, const int32_t* vbs,

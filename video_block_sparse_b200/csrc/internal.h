@@ -41,4 +41,9 @@ cudaError_t launch_fwd_mma(const uint16_t* q, const uint16_t* k, const uint16_t*
                            const int32_t* vbs, uint16_t* out, float* lse, int B, int S, int H, int nq, int topk,
                            float sm_scale, bool precise_p, int* err, cudaStream_t s);
 
+// ---- fwd_tc.cu (tcgen05 / TMEM / TMA kernel)
+cudaError_t launch_fwd_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* topk_idx,
+                          const int32_t* vbs, uint16_t* out, float* lse, int B, int S, int H, int nq, int topk,
+                          float sm_scale, bool precise_p, int* err, cudaStream_t s);
+
 }  // namespace vsa
