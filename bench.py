@@ -121,6 +121,8 @@ def run_gpu(args, rank, world, local_rank):
     import dataclasses
 
     cfg = dataclasses.replace(cfg, seed=rank)  # an independent problem per rank
+    if args.heads:
+        cfg = dataclasses.replace(cfg, H=args.heads)  # a reduced case for profiler captures only
     T, Hh, W = cfg.grid
     vbs_h = vsa.cube_counts(T, Hh, W)
     nq = len(vbs_h)
@@ -266,7 +268,10 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--oracle-seconds", type=float, default=15.0)
+    ap.add_argument("--oracle-seconds", type=float, default=15.0,
+                    help="CPU time for the oracle baseline sample (0 skips it)")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the head count (a smaller case for ncu captures; not a bench line)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -316,14 +321,20 @@ def main():
     value = world * fl / (res["ms_step"] * 1e-3) / 1e12
     fwd_achieved = fl / (res["fwd_ms"] * 1e-3) / 1e12
     cpu = None
-    if world == 1:
+    if world == 1 and args.oracle_seconds > 0:
         tf, items, secs, threads = oracle_sample(res["cfg"], seconds=args.oracle_seconds)
         cpu = {"value": tf, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": f"{items} query-cube work items of the workload (2 heads drawn), {secs:.1f} s"}
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "fwd_traffic.json")
     if os.path.exists(tpath):
-        traffic = json.load(open(tpath)).get("bytes_per_launch")
+        # the counters are only valid for the kernel source they were taken on
+        import hashlib
+
+        t = json.load(open(tpath))
+        src = os.path.join(ROOT, t.get("kernel_source", ""))
+        if os.path.exists(src) and hashlib.sha256(open(src, "rb").read()).hexdigest() == t.get("kernel_source_sha256"):
+            traffic = t.get("bytes_per_launch")
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": res["ms_step"], "higher_is_better": True, "scaling": "weak",

@@ -55,9 +55,10 @@ def _load():
         lib.oracle_cube_means.argtypes = [P, P, P, I, I, I, I, I]
         lib.oracle_route.argtypes = [P, P, P, P, I, I, I, I, I, I, P]
         lib.oracle_fwd_items.argtypes = [P, P, P, P, P, I, I, I, I, I, I, ctypes.c_double, P, I64, P, P]
+        lib.oracle_fwd_items_ex.argtypes = [P, P, P, P, P, I, I, I, I, I, I, ctypes.c_double, P, I64, P, P, P]
         lib.oracle_num_threads.argtypes = []
         for name in ("oracle_f64_to_bf16", "oracle_bf16_to_f64", "oracle_cube_counts", "oracle_tile",
-                     "oracle_untile", "oracle_cube_means", "oracle_route", "oracle_fwd_items",
+                     "oracle_untile", "oracle_cube_means", "oracle_route", "oracle_fwd_items", "oracle_fwd_items_ex",
                      "oracle_num_threads"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
@@ -146,10 +147,11 @@ def route(q: np.ndarray, k: np.ndarray, vbs: np.ndarray, topk: int, want_scores:
     return (idx, scores) if want_scores else idx
 
 
-def fwd_items(q, k, v, topk_idx, vbs, sm_scale: float, items: np.ndarray):
+def fwd_items(q, k, v, topk_idx, vbs, sm_scale: float, items: np.ndarray, want_wabs: bool = False):
     """Fine forward for the listed (b, h, query cube) items.
 
-    Returns out [n, 64, D] float64 and lse [n, 64] float64 (natural log).
+    Returns out [n, 64, D] float64 and lse [n, 64] float64 (natural log), and
+    with want_wabs also wabs [n, 64, D] = sum_u softmax(x)_u |v_u[d]|.
     sm_scale is used as the binary32 value a GPU kernel receives."""
     B, S, H, D = q.shape
     nq = S // 64
@@ -165,10 +167,12 @@ def fwd_items(q, k, v, topk_idx, vbs, sm_scale: float, items: np.ndarray):
     out = np.empty((n, 64, D), dtype=np.float64)
     lse = np.empty((n, 64), dtype=np.float64)
     sigma = float(np.float32(sm_scale))
-    _check(_load().oracle_fwd_items(_ptr(q), _ptr(k), _ptr(v), _ptr(topk_idx), _ptr(vbs),
-                                    B, S, H, D, nq, topk, sigma, _ptr(items), n, _ptr(out), _ptr(lse)),
+    wabs = np.empty((n, 64, D), dtype=np.float64) if want_wabs else None
+    _check(_load().oracle_fwd_items_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(topk_idx), _ptr(vbs),
+                                       B, S, H, D, nq, topk, sigma, _ptr(items), n, _ptr(out), _ptr(lse),
+                                       _ptr(wabs) if want_wabs else None),
            "fwd_items")
-    return out, lse
+    return (out, lse, wabs) if want_wabs else (out, lse)
 
 
 def all_items(B: int, H: int, nq: int) -> np.ndarray:

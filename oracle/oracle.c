@@ -267,11 +267,13 @@ int oracle_route(const uint16_t *q, const uint16_t *k, const int32_t *vbs, int32
  * (a cube listed twice counts twice); x_u = sigma * q_s . k_u;
  * out_s = sum_u softmax(x)_u v_u; lse_s = log sum_u exp(x_u).
  * Work is given as a list of (b, h, i) items; results are item-major:
- * out [n_items, 64, D], lse [n_items, 64]. */
-int oracle_fwd_items(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                     const int32_t *topk_idx, const int32_t *vbs,
-                     int B, int S, int H, int D, int Nq, int topk, double sigma,
-                     const int32_t *items, int64_t n_items, double *out, double *lse)
+ * out [n_items, 64, D], lse [n_items, 64].  If wabs is not NULL it receives,
+ * per output element, sum_u softmax(x)_u |v_u[d]| (same layout as out): the
+ * scale of the error that rounding each weight to a short format can cause. */
+int oracle_fwd_items_ex(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                        const int32_t *topk_idx, const int32_t *vbs,
+                        int B, int S, int H, int D, int Nq, int topk, double sigma,
+                        const int32_t *items, int64_t n_items, double *out, double *lse, double *wabs)
 {
     if (B <= 0 || H <= 0 || D <= 0 || Nq <= 0 || S != 64 * Nq || topk < 1) return ORACLE_ERR_ARG;
     for (int c = 0; c < Nq; ++c)
@@ -307,6 +309,8 @@ int oracle_fwd_items(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                 double *o = out + (it * 64 + r) * D;
                 if (nkeys == 0) {
                     for (int d = 0; d < D; ++d) o[d] = 0.0;
+                    if (wabs != NULL)
+                        for (int d = 0; d < D; ++d) wabs[(it * 64 + r) * D + d] = 0.0;
                     lse[it * 64 + r] = -INFINITY;
                     continue;
                 }
@@ -328,12 +332,31 @@ int oracle_fwd_items(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                 }
                 for (int d = 0; d < D; ++d) o[d] /= l;
                 lse[it * 64 + r] = m + log(l);
+                if (wabs != NULL) {
+                    /* the softmax-weighted mean of |v|: sum_u (p_u / l) |v_u[d]| */
+                    double *a = wabs + (it * 64 + r) * D;
+                    for (int d = 0; d < D; ++d) a[d] = 0.0;
+                    for (int64_t n = 0; n < nkeys; ++n) {
+                        double w = exp(x[n] - m) / l;
+                        const uint16_t *vu = v + (((int64_t)b * S + keys[n]) * H + h) * D;
+                        for (int d = 0; d < D; ++d) a[d] += w * fabs(bf16_bits_to_f64(vu[d]));
+                    }
+                }
             }
         }
         free(keys);
         free(x);
     }
     return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}
+
+int oracle_fwd_items(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                     const int32_t *topk_idx, const int32_t *vbs,
+                     int B, int S, int H, int D, int Nq, int topk, double sigma,
+                     const int32_t *items, int64_t n_items, double *out, double *lse)
+{
+    return oracle_fwd_items_ex(q, k, v, topk_idx, vbs, B, S, H, D, Nq, topk, sigma, items, n_items, out, lse,
+                               NULL);
 }
 
 int oracle_num_threads(void)

