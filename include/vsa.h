@@ -107,13 +107,42 @@ enum vsa_fwd_flags {
     /* Run the warp-level mma.sync kernel instead of the tcgen05/TMEM/TMA
      * kernel: the legacy tensor-core path, kept as the measured baseline the
      * tcgen05 kernel is compared against.  Same results contract. */
-    VSA_FWD_LEGACY_MMA = 2
+    VSA_FWD_LEGACY_MMA = 2,
+    /* Run the tcgen05 kernel that puts keys on the TMEM lanes (one query
+     * cube per CTA step, S^T = K Q^T) instead of the default paired-tile
+     * kernel; kept as the measured alternative.  Same results contract. */
+    VSA_FWD_KEYS_ON_LANES = 4
 };
 
 /* vsa_fwd with option flags (vsa_fwd == vsa_fwd_ex with VSA_FWD_DEFAULT). */
 VSA_API int vsa_fwd_ex(const vsa_bf16 *q, const vsa_bf16 *k, const vsa_bf16 *v, const int32_t *topk_idx,
                const int32_t *vbs, vsa_bf16 *out, float *lse, int B, int S, int H, int D, int Nq, int topk,
                float sm_scale, int flags, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * vsa_fwd_planned -- vsa_fwd_ex with an explicit tile plan.
+ *
+ * The default kernel computes two query cubes of one (b, h) per 128-row
+ * tile and walks the union of their selections, loading a KV cube that
+ * both select once for both.  vsa_fwd / vsa_fwd_ex pair cubes (2p, 2p+1);
+ * a plan (from vsa_plan, or the caller's own) names the pairs instead:
+ *
+ *   plan [B*H][ceil(Nq/2)][2] int32, in: tile p of (b, h) computes query
+ *        cubes plan[bh][p][0] and plan[bh][p][1]; the second may be -1 (a
+ *        tile with one cube).  Every query cube of (b, h) must appear in
+ *        exactly one tile of (b, h); a cube that appears in none is not
+ *        written.  Entries out of range latch device error 4 and are
+ *        skipped.  The plan changes only which cubes share a tile: results
+ *        are those of vsa_fwd_ex up to the order of floating-point sums.
+ *
+ * Errors: as vsa_fwd_ex, plus VSA_ERR_NULL for a NULL plan and VSA_ERR_ARG
+ * if flags select another kernel or Nq > 8192 or topk > 1024 (the limits
+ * of the paired kernel; without a plan, larger problems run the
+ * keys-on-lanes kernel).
+ * ---------------------------------------------------------------------- */
+VSA_API int vsa_fwd_planned(const vsa_bf16 *q, const vsa_bf16 *k, const vsa_bf16 *v, const int32_t *topk_idx,
+                            const int32_t *vbs, const int32_t *plan, vsa_bf16 *out, float *lse, int B, int S,
+                            int H, int D, int Nq, int topk, float sm_scale, int flags, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
  * vsa_route -- cube-mean q.k routing that builds topk_idx.
@@ -203,7 +232,7 @@ VSA_API int vsa_untile(const vsa_bf16 *x_tiled, vsa_bf16 *x_grid, int B, int T, 
  * VSA_ERR_DEVICE (and clears the word), or VSA_ERR_LAUNCH if the stream
  * reports a CUDA error.  `detail` (may be NULL) receives the latched code:
  * 1 = topk_idx value out of range, 2 = vbs value out of range,
- * 3 = a bounded pipeline wait ran out.
+ * 3 = a bounded pipeline wait ran out, 4 = a tile plan entry out of range.
  * ---------------------------------------------------------------------- */
 VSA_API int vsa_device_status(cudaStream_t stream, int *detail);
 

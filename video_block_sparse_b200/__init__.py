@@ -24,12 +24,14 @@ LIB_PATH = os.path.join(_HERE, "libvsa.so")
 FWD_DEFAULT = 0
 FWD_PRECISE_P = 1
 FWD_LEGACY_MMA = 2
+FWD_KEYS_ON_LANES = 4
 
 _STATUS = {0: "VSA_OK", -1: "VSA_ERR_ARG", -2: "VSA_ERR_NULL", -3: "VSA_ERR_ALIGN", -4: "VSA_ERR_WORKSPACE",
            -5: "VSA_ERR_ARCH", -6: "VSA_ERR_LAUNCH", -7: "VSA_ERR_DEVICE"}
 
 # every symbol include/vsa.h declares
-EXPORTS = ("vsa_status_string", "vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_route_workspace_size",
+EXPORTS = ("vsa_status_string", "vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_fwd_planned",
+           "vsa_route_workspace_size",
            "vsa_route", "vsa_route_noalloc", "vsa_cube_counts", "vsa_tile", "vsa_untile", "vsa_device_status")
 
 
@@ -49,6 +51,7 @@ def _load():
     lib.vsa_can_implement.argtypes = [I, I]
     lib.vsa_fwd.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
     lib.vsa_fwd_ex.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
+    lib.vsa_fwd_planned.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.vsa_route_workspace_size.argtypes = [I, I, I, I]
     lib.vsa_route_workspace_size.restype = Z
     lib.vsa_route.argtypes = [P, P, P, P, I, I, I, I, I, I, P, Z, P]
@@ -57,7 +60,7 @@ def _load():
     lib.vsa_tile.argtypes = [P, P, I, I, I, I, I, I, P]
     lib.vsa_untile.argtypes = [P, P, I, I, I, I, I, I, P]
     lib.vsa_device_status.argtypes = [P, P]
-    for name in ("vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_route", "vsa_route_noalloc", "vsa_cube_counts",
+    for name in ("vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_fwd_planned", "vsa_route", "vsa_route_noalloc", "vsa_cube_counts",
                  "vsa_tile",
                  "vsa_untile", "vsa_device_status"):
         getattr(lib, name).restype = I
@@ -180,8 +183,9 @@ def route_noalloc(q: torch.Tensor, k: torch.Tensor, vbs: torch.Tensor, topk: int
 
 def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk_idx: torch.Tensor, vbs: torch.Tensor,
         sm_scale: float | None = None, out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
-        want_lse: bool = False, flags: int = FWD_DEFAULT, stream=None):
-    """Fine block-sparse attention forward; returns out (and lse if asked)."""
+        want_lse: bool = False, flags: int = FWD_DEFAULT, plan: torch.Tensor | None = None, stream=None):
+    """Fine block-sparse attention forward; returns out (and lse if asked).
+    plan: optional int32 [B*H, ceil(Nq/2), 2] tile plan (vsa_fwd_planned)."""
     B, S, H, D = q.shape
     nq = S // 64
     topk = topk_idx.shape[-1]
@@ -195,8 +199,15 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk_idx: torch.Tenso
         out = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty(B, H, S, dtype=torch.float32, device=q.device)
-    _check(get_lib().vsa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(topk_idx), _ptr(vbs), _ptr(out), _ptr(lse), B, S, H, D,
-                          nq, topk, float(sm_scale), int(flags), _stream(stream)), "vsa_fwd")
+    if plan is None:
+        _check(get_lib().vsa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(topk_idx), _ptr(vbs), _ptr(out), _ptr(lse), B, S,
+                                    H, D, nq, topk, float(sm_scale), int(flags), _stream(stream)), "vsa_fwd")
+    else:
+        if plan.dtype != torch.int32 or plan.numel() != B * H * ((nq + 1) // 2) * 2:
+            raise ValueError("plan must be int32 [B*H, ceil(Nq/2), 2]")
+        _check(get_lib().vsa_fwd_planned(_ptr(q), _ptr(k), _ptr(v), _ptr(topk_idx), _ptr(vbs), _ptr(plan), _ptr(out),
+                                         _ptr(lse), B, S, H, D, nq, topk, float(sm_scale), int(flags),
+                                         _stream(stream)), "vsa_fwd_planned")
     return (out, lse) if (want_lse or lse is not None) else out
 
 

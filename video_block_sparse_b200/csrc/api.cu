@@ -70,6 +70,10 @@ int check_bshd(int B, int S, int H, int D, int Nq)
     return VSA_OK;
 }
 
+int fwd_dispatch(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const int32_t* topk_idx,
+                 const int32_t* vbs, const int32_t* plan, vsa_bf16* out, float* lse, int B, int S, int H, int D,
+                 int Nq, int topk, float sm_scale, int flags, cudaStream_t stream);
+
 }  // namespace
 
 extern "C" {
@@ -91,17 +95,26 @@ const char* vsa_status_string(int status)
 
 int vsa_can_implement(int D, int sm_version) { return (D == 128 && sm_version == 100) ? 1 : 0; }
 
-int vsa_fwd_ex(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const int32_t* topk_idx, const int32_t* vbs,
-               vsa_bf16* out, float* lse, int B, int S, int H, int D, int Nq, int topk, float sm_scale, int flags,
-               cudaStream_t stream)
+}  // extern "C"
+
+namespace {
+
+// Shared by vsa_fwd_ex and vsa_fwd_planned: checks, then the kernel the flags name.
+int fwd_dispatch(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const int32_t* topk_idx,
+                 const int32_t* vbs, const int32_t* plan, vsa_bf16* out, float* lse, int B, int S, int H, int D,
+                 int Nq, int topk, float sm_scale, int flags, cudaStream_t stream)
 {
     int rc = check_bshd(B, S, H, D, Nq);
     if (rc != VSA_OK) return rc;
-    if (topk < 1 || (flags & ~(VSA_FWD_PRECISE_P | VSA_FWD_LEGACY_MMA)) != 0) return VSA_ERR_ARG;
+    if (topk < 1 || (flags & ~(VSA_FWD_PRECISE_P | VSA_FWD_LEGACY_MMA | VSA_FWD_KEYS_ON_LANES)) != 0)
+        return VSA_ERR_ARG;
+    if ((flags & VSA_FWD_LEGACY_MMA) && (flags & VSA_FWD_KEYS_ON_LANES)) return VSA_ERR_ARG;
     if ((int64_t)B * H * Nq * topk > INT32_MAX) return VSA_ERR_ARG;
+    const bool pair_kernel = (flags & (VSA_FWD_LEGACY_MMA | VSA_FWD_KEYS_ON_LANES)) == 0;
+    if (plan != nullptr && (!pair_kernel || !vsa::fwd_pair_supported(Nq, topk))) return VSA_ERR_ARG;
     if (!q || !k || !v || !topk_idx || !vbs || !out) return VSA_ERR_NULL;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(topk_idx) ||
-        !aligned16(vbs) || (lse && !aligned16(lse)))
+        !aligned16(vbs) || (lse && !aligned16(lse)) || (plan && !aligned16(plan)))
         return VSA_ERR_ALIGN;
     if ((rc = check_arch()) != VSA_OK) return rc;
     int* err;
@@ -110,8 +123,30 @@ int vsa_fwd_ex(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const in
     if (flags & VSA_FWD_LEGACY_MMA)
         return launch_status(
             vsa::launch_fwd_mma(q, k, v, topk_idx, vbs, out, lse, B, S, H, Nq, topk, sm_scale, precise, err, stream));
+    if (pair_kernel && vsa::fwd_pair_supported(Nq, topk))
+        return launch_status(vsa::launch_fwd_pair(q, k, v, topk_idx, vbs, plan, out, lse, B, S, H, Nq, topk, sm_scale,
+                                                  precise, err, stream));
     return launch_status(
         vsa::launch_fwd_tc(q, k, v, topk_idx, vbs, out, lse, B, S, H, Nq, topk, sm_scale, precise, err, stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+int vsa_fwd_ex(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const int32_t* topk_idx, const int32_t* vbs,
+               vsa_bf16* out, float* lse, int B, int S, int H, int D, int Nq, int topk, float sm_scale, int flags,
+               cudaStream_t stream)
+{
+    return fwd_dispatch(q, k, v, topk_idx, vbs, nullptr, out, lse, B, S, H, D, Nq, topk, sm_scale, flags, stream);
+}
+
+int vsa_fwd_planned(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const int32_t* topk_idx,
+                    const int32_t* vbs, const int32_t* plan, vsa_bf16* out, float* lse, int B, int S, int H, int D,
+                    int Nq, int topk, float sm_scale, int flags, cudaStream_t stream)
+{
+    if (!plan) return VSA_ERR_NULL;
+    return fwd_dispatch(q, k, v, topk_idx, vbs, plan, out, lse, B, S, H, D, Nq, topk, sm_scale, flags, stream);
 }
 
 int vsa_fwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const int32_t* topk_idx, const int32_t* vbs,

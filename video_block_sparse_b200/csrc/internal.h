@@ -15,6 +15,7 @@ enum DeviceError : int {
     kErrTopkIdx = 1,
     kErrVbs = 2,
     kErrWaitTimeout = 3,
+    kErrPlan = 4,
 };
 
 struct CubeGeom {
@@ -45,5 +46,11 @@ cudaError_t launch_fwd_mma(const uint16_t* q, const uint16_t* k, const uint16_t*
 cudaError_t launch_fwd_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* topk_idx,
                           const int32_t* vbs, uint16_t* out, float* lse, int B, int S, int H, int nq, int topk,
                           float sm_scale, bool precise_p, int* err, cudaStream_t s);
+
+// ---- fwd_pair.cu (tcgen05 kernel, two query cubes per 128-row tile)
+bool fwd_pair_supported(int nq, int topk);
+cudaError_t launch_fwd_pair(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* topk_idx,
+                            const int32_t* vbs, const int32_t* plan, uint16_t* out, float* lse, int B, int S, int H,
+                            int nq, int topk, float sm_scale, bool precise_p, int* err, cudaStream_t s);
 
 }  // namespace vsa
