@@ -2,6 +2,7 @@
 one batch of synthetic Wan2.2 832x480/81f activations:
 
     tile q, k, v (raster -> cube-major)  ->  route (cube-mean q.k top-k)
+    ->  plan (pair query cubes by selection overlap)
     ->  fine block-sparse attention forward  ->  untile the output
 
 Metric: effective TFLOP/s of the step, FLOPs = 4 * B * S * topk * 64 * D * H
@@ -42,7 +43,7 @@ def flops(cfg, S):
 
 def config_block(cfg, S):
     return {
-        "workload": "Wan2.2 T2V-A14B 832x480/81f VSA fine stage (tile q,k,v -> route -> fwd -> untile)",
+        "workload": "Wan2.2 T2V-A14B 832x480/81f VSA fine stage (tile q,k,v -> route -> plan -> fwd -> untile)",
         "B": cfg.B, "latent_grid": list(cfg.grid), "S_padded": S, "H": cfg.H, "D": 128, "topk": cfg.topk,
         "sm_scale": cfg.sm_scale, "global_batch": cfg.B, "seq_len": S, "parallelism": "replicas (independent problem per GPU)",
         "l2": "inputs larger than L2 (1.0 GB raster q,k,v read per step); no flush",
@@ -134,6 +135,8 @@ def run_gpu(args, rank, world, local_rank):
     qt, kt, vt = (torch.empty(B, S, H, D, dtype=torch.bfloat16, device=dev) for _ in range(3))
     idx = torch.empty(B, H, nq, cfg.topk, dtype=torch.int32, device=dev)
     ws = torch.empty(vsa.route_workspace_size(B, H, nq, D), dtype=torch.uint8, device=dev)
+    plan = torch.empty(B * H, (nq + 1) // 2, 2, dtype=torch.int32, device=dev)
+    plan_ws = torch.empty(vsa.plan_workspace_size(B, H, nq, cfg.topk), dtype=torch.uint8, device=dev)
     out_t = torch.empty_like(qt)
     out_g = torch.empty_like(q_g)
     lse = torch.empty(B, H, S, dtype=torch.float32, device=dev)
@@ -146,14 +149,15 @@ def run_gpu(args, rank, world, local_rank):
         vsa.tile(k_g, cfg.grid, out=kt)
         vsa.tile(v_g, cfg.grid, out=vt)
         vsa.route(qt, kt, vbs, cfg.topk, out=idx, workspace=ws)
+        vsa.plan(idx, out=plan, workspace=plan_ws)
         if i is not None:
             ev_f0[i].record(stream)
-        vsa.fwd(qt, kt, vt, idx, vbs, cfg.sm_scale, out=out_t, lse=lse)
+        vsa.fwd(qt, kt, vt, idx, vbs, cfg.sm_scale, out=out_t, lse=lse, plan=plan)
         if i is not None:
             ev_f1[i].record(stream)
         vsa.untile(out_t, cfg.grid, out=out_g)
 
-    launches_per_step = 3 + 2 + 1 + 1
+    launches_per_step = 3 + 2 + 3 + 1 + 1  # tile x3, route, plan, fwd, untile
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()

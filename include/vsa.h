@@ -205,6 +205,40 @@ VSA_API int vsa_route_noalloc(const vsa_bf16 *q, const vsa_bf16 *k, const int32_
                               int S, int H, int D, int Nq, int topk, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * vsa_plan -- pair the query cubes of every (b, h) for vsa_fwd_planned.
+ *
+ * The paired forward kernel computes two query cubes per tile and loads a
+ * KV cube that both select once for both, so its work falls with the
+ * overlap of the two selection lists.  This call pairs cubes whose lists
+ * overlap most.  The pages define no such schedule; it changes only which
+ * cubes share a tile, never the attention result.  Steps (integer work,
+ * fixed tie rules, deterministic):
+ *   1. overlap(i, j) = number of distinct cubes both lists name;
+ *   2. each cube keeps its 8 best partners j != i (larger overlap first,
+ *      then smaller j);
+ *   3. rounds: every unpaired cube proposes to its first still-unpaired
+ *      candidate; cubes that propose to each other are paired; repeated
+ *      until a round pairs none;
+ *   4. cubes left over are paired in index order (an odd one last, alone);
+ *   5. tiles are listed by their smaller cube index: (smaller, larger) or
+ *      (i, -1).
+ *
+ *   topk_idx  [B, H, Nq, topk] int32 in (values in [0, Nq); others are
+ *             ignored and latch device error 1)
+ *   plan      [B*H][ceil(Nq/2)][2] int32 out
+ *   workspace device scratch of vsa_plan_workspace_size(B, H, Nq, topk)
+ *             bytes, 16-byte aligned, owned by the caller.
+ *
+ * Errors: VSA_ERR_ARG unless 1 <= topk <= Nq <= 8192 and B, H >= 1;
+ * VSA_ERR_NULL, VSA_ERR_ALIGN, VSA_ERR_WORKSPACE, VSA_ERR_ARCH,
+ * VSA_ERR_LAUNCH as for the other calls.
+ * ---------------------------------------------------------------------- */
+VSA_API size_t vsa_plan_workspace_size(int B, int H, int Nq, int topk);
+
+VSA_API int vsa_plan(const int32_t *topk_idx, int32_t *plan, int B, int H, int Nq, int topk, void *workspace,
+                     size_t workspace_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * Cube-major layout.  Dataset card "wan2.2_production_values", section
  * "Shapes": a T x Hh x W latent grid is cut into 4x4x4 cubes,
  * Nq = ceil(T/4) * ceil(Hh/4) * ceil(W/4), S = 64 * Nq.  Cubes are ordered

@@ -57,9 +57,10 @@ def _load():
         lib.oracle_fwd_items.argtypes = [P, P, P, P, P, I, I, I, I, I, I, ctypes.c_double, P, I64, P, P]
         lib.oracle_fwd_items_ex.argtypes = [P, P, P, P, P, I, I, I, I, I, I, ctypes.c_double, P, I64, P, P, P]
         lib.oracle_num_threads.argtypes = []
+        lib.oracle_plan.argtypes = [P, I, I, I, I, P]
         for name in ("oracle_f64_to_bf16", "oracle_bf16_to_f64", "oracle_cube_counts", "oracle_tile",
                      "oracle_untile", "oracle_cube_means", "oracle_route", "oracle_fwd_items", "oracle_fwd_items_ex",
-                     "oracle_num_threads"):
+                     "oracle_num_threads", "oracle_plan"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -189,3 +190,13 @@ def fwd(q, k, v, topk_idx, vbs, sm_scale: float):
     out = o.reshape(B, H, nq, 64, D).transpose(0, 2, 3, 1, 4).reshape(B, S, H, D)
     lse = l.reshape(B, H, nq * 64)
     return np.ascontiguousarray(out), np.ascontiguousarray(lse)
+
+
+def plan(topk_idx: np.ndarray) -> np.ndarray:
+    """Pairing of the query cubes of every (b, h) by selection overlap:
+    int32 [B*H, ceil(Nq/2), 2] (see oracle.c, "tile plan")."""
+    B, H, nq, topk = topk_idx.shape
+    topk_idx = np.ascontiguousarray(topk_idx, dtype=np.int32)
+    out = np.empty((B * H, (nq + 1) // 2, 2), dtype=np.int32)
+    _check(_load().oracle_plan(_ptr(topk_idx), B, H, nq, topk, _ptr(out)), "plan")
+    return out

@@ -359,6 +359,100 @@ int oracle_fwd_items(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                                NULL);
 }
 
+/* ---- tile plan -----------------------------------------------------------
+ * Not from the pages: the pairing schedule of the paired forward kernel,
+ * restated as plainly as possible so the GPU planner can be checked bit for
+ * bit.  For each (b, h): overlap(i, j) = number of distinct cubes that both
+ * lists name; each cube's candidates are the 8 cubes j != i with the largest
+ * overlap (ties: smaller j); rounds: each unpaired cube proposes to its first
+ * unpaired candidate, mutual proposals pair, until a round pairs none;
+ * leftovers pair in index order; tiles are listed by smaller index as
+ * (smaller, larger) or (i, -1).  plan is [B*H][ceil(Nq/2)][2]. */
+int oracle_plan(const int32_t *topk_idx, int B, int H, int Nq, int topk, int32_t *plan)
+{
+    if (B <= 0 || H <= 0 || Nq <= 0 || topk < 1) return ORACLE_ERR_ARG;
+    const int NC = 8;
+    unsigned char *member = (unsigned char *)malloc((size_t)Nq * Nq);
+    int *cand = (int *)malloc((size_t)Nq * NC * sizeof(int));
+    int *partner = (int *)malloc((size_t)Nq * sizeof(int));
+    int *prop = (int *)malloc((size_t)Nq * sizeof(int));
+    int *dist = (int *)malloc((size_t)Nq * (topk < Nq ? topk : Nq) * sizeof(int));
+    int *ndist = (int *)malloc((size_t)Nq * sizeof(int));
+    if (!member || !cand || !partner || !prop || !dist || !ndist) {
+        free(member); free(cand); free(partner); free(prop); free(dist); free(ndist);
+        return ORACLE_ERR_NOMEM;
+    }
+    const int tiles = (Nq + 1) / 2;
+    for (int bh = 0; bh < B * H; ++bh) {
+        memset(member, 0, (size_t)Nq * Nq);
+        for (int i = 0; i < Nq; ++i)
+            for (int t = 0; t < topk; ++t) {
+                int j = topk_idx[((int64_t)bh * Nq + i) * topk + t];
+                if (j >= 0 && j < Nq) member[(size_t)i * Nq + j] = 1;
+            }
+        /* the distinct cubes of each list, ascending */
+        int ndist_max = topk < Nq ? topk : Nq;
+        for (int j = 0; j < Nq; ++j) {
+            int n = 0;
+            for (int c = 0; c < Nq; ++c)
+                if (member[(size_t)j * Nq + c]) dist[(size_t)j * ndist_max + n++] = c;
+            ndist[j] = n;
+        }
+        for (int i = 0; i < Nq; ++i) {
+            int best_ov[8], best_j[8];
+            for (int c = 0; c < NC; ++c) { best_ov[c] = -1; best_j[c] = -1; }
+            for (int j = 0; j < Nq; ++j) {
+                if (j == i) continue;
+                int ov = 0;
+                for (int e = 0; e < ndist[j]; ++e) ov += member[(size_t)i * Nq + dist[(size_t)j * ndist_max + e]];
+                /* j ascends, so a later j with an equal overlap never displaces an earlier one */
+                int pos = NC;
+                while (pos > 0 && ov > best_ov[pos - 1]) --pos;
+                if (pos < NC) {
+                    for (int c = NC - 1; c > pos; --c) { best_ov[c] = best_ov[c - 1]; best_j[c] = best_j[c - 1]; }
+                    best_ov[pos] = ov;
+                    best_j[pos] = j;
+                }
+            }
+            for (int c = 0; c < NC; ++c) cand[i * NC + c] = best_j[c];
+        }
+        for (int i = 0; i < Nq; ++i) partner[i] = -1;
+        for (int round = 0; round < 64; ++round) {
+            for (int i = 0; i < Nq; ++i) {
+                prop[i] = -1;
+                if (partner[i] >= 0) continue;
+                for (int c = 0; c < NC; ++c) {
+                    int j = cand[i * NC + c];
+                    if (j >= 0 && partner[j] < 0) { prop[i] = j; break; }
+                }
+            }
+            int changed = 0;
+            for (int i = 0; i < Nq; ++i) {
+                int j = prop[i];
+                if (j >= 0 && prop[j] == i) { partner[i] = j; changed = 1; }
+            }
+            if (!changed) break;
+        }
+        int pending = -1, odd = -1;
+        for (int i = 0; i < Nq; ++i) {
+            if (partner[i] >= 0) continue;
+            if (pending < 0) pending = i;
+            else { partner[pending] = i; partner[i] = pending; pending = -1; }
+        }
+        odd = pending;
+        int p = 0;
+        for (int i = 0; i < Nq; ++i) {
+            if (partner[i] > i || i == odd) {
+                plan[((int64_t)bh * tiles + p) * 2] = i;
+                plan[((int64_t)bh * tiles + p) * 2 + 1] = i == odd ? -1 : partner[i];
+                ++p;
+            }
+        }
+    }
+    free(member); free(cand); free(partner); free(prop); free(dist); free(ndist);
+    return ORACLE_OK;
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

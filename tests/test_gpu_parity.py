@@ -267,3 +267,73 @@ def test_fwd_negative_scale(vsa):
         assert res["gate"]["ok"], res
         got_lse = np.stack([lse[b, h, 64 * i: 64 * i + 64].cpu().numpy() for b, h, i in items])
         assert np.allclose(got_lse, l64, rtol=1e-5, atol=1e-3)
+
+
+# ------------------------------------------------------------------ tile plan
+
+@pytest.mark.parametrize("case", ["tiny", "random33", "wan480"])
+def test_plan_bit_exact(vsa, case):
+    if case == "random33":
+        idx = synth.random_topk(21, 2, 2, 33, 5)
+    else:
+        p = common.prepare(case)
+        idx = p.idx
+    want = oracle.plan(idx)
+    got = vsa.plan(torch.from_numpy(idx).cuda())
+    torch.cuda.synchronize()
+    _no_device_error(vsa)
+    np.testing.assert_array_equal(got.cpu().numpy(), want)
+
+
+def test_fwd_with_plan_mid(vsa):
+    """The paired kernel on the planner's pairing: every row checked (both modes)."""
+    p = common.prepare("wan480", H=3, grid=(9, 10, 11), topk=7, B=2)
+    plan = oracle.plan(p.idx)
+    q, k, v = common.dev(p.qt), common.dev(p.kt), common.dev(p.vt)
+    idx, vbs = torch.from_numpy(p.idx).cuda(), torch.from_numpy(p.vbs).cuda()
+    for flags in (0, vsa.FWD_PRECISE_P):
+        out, lse = vsa.fwd(q, k, v, idx, vbs, p.cfg.sm_scale, want_lse=True, flags=flags,
+                           plan=torch.from_numpy(plan).cuda())
+        torch.cuda.synchronize()
+        _no_device_error(vsa)
+        _check_items(p, out, lse, oracle.all_items(p.cfg.B, p.cfg.H, p.nq), f"plan-mid/{flags}", precise=flags != 0)
+
+
+def test_fwd_with_arbitrary_pairing(vsa):
+    """Any valid pairing gives the same results: a random one, singles included."""
+    p = _small(17, nq=9, H=2, topk=4, vbs=[64, 7, 64, 33, 64, 1, 16, 0, 48])
+    g = np.random.default_rng(17)
+    plan = np.empty((2, 5, 2), np.int32)
+    for bh in range(2):
+        perm = g.permutation(9).tolist()
+        tiles = [sorted(perm[2 * t: 2 * t + 2]) for t in range(4)] + [[perm[8], -1]]
+        plan[bh] = np.array(sorted(tiles), np.int32)
+    q, k, v = common.dev(p.qt), common.dev(p.kt), common.dev(p.vt)
+    idx, vbs = torch.from_numpy(p.idx).cuda(), torch.from_numpy(p.vbs).cuda()
+    out, lse = vsa.fwd(q, k, v, idx, vbs, p.cfg.sm_scale, want_lse=True, plan=torch.from_numpy(plan).cuda())
+    torch.cuda.synchronize()
+    _no_device_error(vsa)
+    _check_items(p, out, lse, oracle.all_items(1, 2, 9), "arbitrary-pairing")
+
+
+def test_fwd_plan_bad_entry_latches_error(vsa):
+    p = _small(18, nq=4, H=1, topk=2, vbs=[64, 64, 64, 64])
+    plan = np.array([[[0, 1], [2, 9]]], np.int32)  # 9 is not a cube: the kernel drops it, error 4
+    q, k, v = common.dev(p.qt), common.dev(p.kt), common.dev(p.vt)
+    vsa.fwd(q, k, v, torch.from_numpy(p.idx).cuda(), torch.from_numpy(p.vbs).cuda(), 0.1,
+            plan=torch.from_numpy(plan).cuda())
+    rc, detail = vsa.device_status()
+    assert rc == -7 and detail == 4
+
+
+def test_fwd_planned_full_size_sampled(vsa):
+    """Wan 832x480 shape, planner's pairing from the GPU planner, sampled rows."""
+    p = common.prepare("wan480")
+    q, k, v = common.dev(p.qt), common.dev(p.kt), common.dev(p.vt)
+    idx, vbs = torch.from_numpy(p.idx).cuda(), torch.from_numpy(p.vbs).cuda()
+    plan = vsa.plan(idx)
+    out, lse = vsa.fwd(q, k, v, idx, vbs, p.cfg.sm_scale, want_lse=True, plan=plan)
+    torch.cuda.synchronize()
+    _no_device_error(vsa)
+    items = common.sample_items(p.cfg.B, p.cfg.H, p.nq, 120, seed=5)
+    _check_items(p, out, lse, items, "wan480/planned")

@@ -408,3 +408,66 @@ def test_near_tie_reference_accepts_only_midpoint_flips():
     ref, n = common.near_tie_reference(gpu, exact, bound=np.array([0.25 * ulp, 0.25 * ulp, 10 * ulp]))
     assert n == 2
     assert ref[0] == 4.0 and ref[1] == 4.0 and ref[2] == np.float32(4.0 + ulp)
+
+
+# ---------------------------------------------------------------- tile plan
+
+def _check_pairing(plan, nq):
+    """Every cube of every (b, h) in exactly one tile; tiles ordered by their
+    smaller cube; a single cube only as the last leftover of an odd count."""
+    for row in plan:
+        seen = []
+        for a, b in row:
+            assert b == -1 or a < b
+            seen += [a] + ([b] if b >= 0 else [])
+        assert sorted(seen) == list(range(nq))
+        firsts = [a for a, _ in row]
+        assert firsts == sorted(firsts)
+        assert sum(1 for _, b in row if b < 0) == nq % 2
+
+
+def test_plan_hand_example(oracle_lib):
+    """Five cubes: 0 and 2 share both cubes, 1 and 3 share both, 4 shares one
+    with 0 and 2.  Round 1 pairs (0,2) and (1,3) by mutual choice; 4 has no
+    unpaired candidate left and is the odd one out."""
+    idx = np.array([[[[0, 1], [2, 3], [0, 1], [2, 3], [4, 0]]]], np.int32)
+    assert oracle_lib.plan(idx).tolist() == [[[0, 2], [1, 3], [4, -1]]]
+
+
+def test_plan_pairs_planted_twins(oracle_lib):
+    """Cubes planted in pairs with identical lists (and lists that share
+    nothing across pairs) are paired with their twin, whatever their order."""
+    g = np.random.default_rng(8)
+    nq, topk = 12, 2
+    perm = g.permutation(nq)
+    idx = np.empty((1, 1, nq, topk), np.int32)
+    for p in range(nq // 2):
+        a, b = perm[2 * p], perm[2 * p + 1]
+        idx[0, 0, a] = idx[0, 0, b] = [2 * p, 2 * p + 1]
+    plan = oracle_lib.plan(idx)
+    _check_pairing(plan, nq)
+    want = sorted(tuple(sorted((perm[2 * p], perm[2 * p + 1]))) for p in range(nq // 2))
+    assert sorted(tuple(t) for t in plan[0].tolist()) == want
+
+
+@pytest.mark.parametrize("nq,topk,seed", [(7, 3, 0), (10, 4, 1), (33, 5, 2), (64, 8, 3)])
+def test_plan_is_a_pairing_and_beats_index_order(oracle_lib, nq, topk, seed):
+    """Random lists: the plan pairs every cube once, and its total overlap is at
+    least that of pairing cubes in index order (the greedy choice never loses
+    to an arbitrary pairing by more than a factor 2; on these inputs it wins)."""
+    idx = synth.random_topk(seed, 2, 2, nq, topk)
+    plan = oracle_lib.plan(idx)
+    _check_pairing(plan, nq)
+    for bh in range(4):
+        L = idx.reshape(4, nq, topk)[bh]
+        ov = lambda a, b: len(set(L[a].tolist()) & set(L[b].tolist()))
+        planned = sum(ov(a, b) for a, b in plan[bh] if b >= 0)
+        ordered = sum(ov(2 * p, 2 * p + 1) for p in range(nq // 2))
+        assert planned >= ordered
+
+
+def test_plan_ignores_duplicates_and_bad_ids(oracle_lib):
+    """Overlaps count distinct cubes; ids outside [0, Nq) are ignored."""
+    idx = np.array([[[[1, 1, 2], [1, 2, 9], [3, 3, 3], [-1, 3, 0]]]], np.int32)
+    # distinct sets: {1,2}, {1,2}, {3}, {3,0}: 0-1 overlap 2, 2-3 overlap 1
+    assert oracle_lib.plan(idx).tolist() == [[[0, 1], [2, 3]]]

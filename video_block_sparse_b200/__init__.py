@@ -31,7 +31,7 @@ _STATUS = {0: "VSA_OK", -1: "VSA_ERR_ARG", -2: "VSA_ERR_NULL", -3: "VSA_ERR_ALIG
 
 # every symbol include/vsa.h declares
 EXPORTS = ("vsa_status_string", "vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_fwd_planned",
-           "vsa_route_workspace_size",
+           "vsa_plan_workspace_size", "vsa_plan", "vsa_route_workspace_size",
            "vsa_route", "vsa_route_noalloc", "vsa_cube_counts", "vsa_tile", "vsa_untile", "vsa_device_status")
 
 
@@ -52,6 +52,9 @@ def _load():
     lib.vsa_fwd.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
     lib.vsa_fwd_ex.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.vsa_fwd_planned.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
+    lib.vsa_plan_workspace_size.argtypes = [I, I, I, I]
+    lib.vsa_plan_workspace_size.restype = Z
+    lib.vsa_plan.argtypes = [P, P, I, I, I, I, P, Z, P]
     lib.vsa_route_workspace_size.argtypes = [I, I, I, I]
     lib.vsa_route_workspace_size.restype = Z
     lib.vsa_route.argtypes = [P, P, P, P, I, I, I, I, I, I, P, Z, P]
@@ -60,7 +63,7 @@ def _load():
     lib.vsa_tile.argtypes = [P, P, I, I, I, I, I, I, P]
     lib.vsa_untile.argtypes = [P, P, I, I, I, I, I, I, P]
     lib.vsa_device_status.argtypes = [P, P]
-    for name in ("vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_fwd_planned", "vsa_route", "vsa_route_noalloc", "vsa_cube_counts",
+    for name in ("vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_fwd_planned", "vsa_plan", "vsa_route", "vsa_route_noalloc", "vsa_cube_counts",
                  "vsa_tile",
                  "vsa_untile", "vsa_device_status"):
         getattr(lib, name).restype = I
@@ -166,6 +169,26 @@ def route(q: torch.Tensor, k: torch.Tensor, vbs: torch.Tensor, topk: int, out: t
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     _check(get_lib().vsa_route(_ptr(q), _ptr(k), _ptr(vbs), _ptr(out), B, S, H, D, nq, topk, _ptr(workspace),
                          workspace.numel() * workspace.element_size(), _stream(stream)), "vsa_route")
+    return out
+
+
+def plan_workspace_size(B: int, H: int, nq: int, topk: int) -> int:
+    return int(get_lib().vsa_plan_workspace_size(B, H, nq, topk))
+
+
+def plan(topk_idx: torch.Tensor, out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+         stream=None) -> torch.Tensor:
+    """Tile plan [B*H, ceil(Nq/2), 2] int32 pairing query cubes by selection overlap (vsa_plan)."""
+    B, H, nq, topk = topk_idx.shape
+    if topk_idx.dtype != torch.int32:
+        raise ValueError("topk_idx must be int32")
+    if out is None:
+        out = torch.empty(B * H, (nq + 1) // 2, 2, dtype=torch.int32, device=topk_idx.device)
+    need = plan_workspace_size(B, H, nq, topk)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=topk_idx.device)
+    _check(get_lib().vsa_plan(_ptr(topk_idx), _ptr(out), B, H, nq, topk, _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream(stream)), "vsa_plan")
     return out
 
 

@@ -178,6 +178,27 @@ int vsa_route(const vsa_bf16* q, const vsa_bf16* k, const int32_t* vbs, int32_t*
     return launch_status(vsa::launch_route(q, k, vbs, topk_idx, B, S, H, Nq, topk, workspace, err, stream));
 }
 
+size_t vsa_plan_workspace_size(int B, int H, int Nq, int topk)
+{
+    if (B < 1 || H < 1 || Nq < 1 || Nq > 8192 || topk < 1) return 0;
+    return vsa::plan_workspace_bytes(B, H, Nq);
+}
+
+int vsa_plan(const int32_t* topk_idx, int32_t* plan, int B, int H, int Nq, int topk, void* workspace,
+             size_t workspace_bytes, cudaStream_t stream)
+{
+    if (B < 1 || H < 1 || Nq < 1 || Nq > 8192 || topk < 1 || topk > Nq) return VSA_ERR_ARG;
+    if ((int64_t)B * H * Nq * topk > INT32_MAX) return VSA_ERR_ARG;
+    if (!topk_idx || !plan) return VSA_ERR_NULL;
+    if (!workspace || workspace_bytes < vsa::plan_workspace_bytes(B, H, Nq)) return VSA_ERR_WORKSPACE;
+    if (!aligned16(topk_idx) || !aligned16(plan) || !aligned16(workspace)) return VSA_ERR_ALIGN;
+    int rc = check_arch();
+    if (rc != VSA_OK) return rc;
+    int* err;
+    if ((rc = device_error_word(&err)) != VSA_OK) return rc;
+    return launch_status(vsa::launch_plan(topk_idx, plan, B, H, Nq, topk, workspace, err, stream));
+}
+
 int vsa_cube_counts(int T, int Hh, int W, int32_t* vbs_host, int* Nq_out)
 {
     if (T < 1 || Hh < 1 || W < 1) return VSA_ERR_ARG;

@@ -98,8 +98,7 @@ struct StepMeta {
 static_assert(sizeof(StepMeta) == 48, "StepMeta layout");
 
 // The fields the other roles need, packed in one 32-bit word in shared memory:
-// na [0,7) nb [7,14) ma [14,16) mb [16,18) flags [18,20) vslot [20] vpar [21]
-// kslot [22] (the K ring slot the step's QK read).
+// na [0,7) nb [7,14) ma [14,16) mb [16,18) flags [18,20) vslot [20] vpar [21].
 __device__ __forceinline__ uint32_t step_word(const StepMeta& s)
 {
     return (uint32_t)s.na | ((uint32_t)s.nb << 7) | ((uint32_t)s.ma << 14) | ((uint32_t)s.mb << 16) |
@@ -112,7 +111,6 @@ __device__ __forceinline__ int sw_mb(uint32_t w) { return (int)((w >> 16) & 3u);
 __device__ __forceinline__ int sw_flags(uint32_t w) { return (int)((w >> 18) & 3u); }
 __device__ __forceinline__ int sw_vslot(uint32_t w) { return (int)((w >> 20) & 1u); }
 __device__ __forceinline__ int sw_vpar(uint32_t w) { return (int)((w >> 21) & 1u); }
-__device__ __forceinline__ int sw_kslot(uint32_t w) { return (int)((w >> 22) & 1u); }
 
 struct Misc {
     uint64_t q_full[2], q_empty[2];        // per slot
@@ -250,20 +248,6 @@ __device__ __noinline__ bool wait_bar_slow(uint64_t* bar, uint32_t parity, Misc&
             return false;
         }
     }
-}
-
-// Non-blocking probe of a phase (cheaper than try_wait when it has completed).
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred P;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, P;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
 }
 
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Misc& m, int* err)
@@ -722,8 +706,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int ks = ku % kNK;
                     if (!wait_warp(&m.k_full[ks], (ku / kNK) & 1, m, err)) { aborted = true; break; }
                     const int vidx = vu + (pending[x ^ 1] ? 1 : 0);  // V uses before this step's PV
-                    const uint32_t meta = m.k_meta[ks] | ((uint32_t)(vidx % kNV) << 20) |
-                                          ((uint32_t)((vidx / kNV) & 1) << 21) | ((uint32_t)ks << 22);
+                    const uint32_t meta =
+                        m.k_meta[ks] | ((uint32_t)(vidx % kNV) << 20) | ((uint32_t)((vidx / kNV) & 1) << 21);
                     __syncwarp();
                     if (lane == 0) {
                         m.s_meta[x] = meta;

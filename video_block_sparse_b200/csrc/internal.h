@@ -53,4 +53,9 @@ cudaError_t launch_fwd_pair(const uint16_t* q, const uint16_t* k, const uint16_t
                             const int32_t* vbs, const int32_t* plan, uint16_t* out, float* lse, int B, int S, int H,
                             int nq, int topk, float sm_scale, bool precise_p, int* err, cudaStream_t s);
 
+// ---- plan.cu (pairing of query cubes by selection overlap)
+size_t plan_workspace_bytes(int B, int H, int nq);
+cudaError_t launch_plan(const int32_t* topk_idx, int32_t* plan, int B, int H, int nq, int topk, void* workspace,
+                        int* err, cudaStream_t s);
+
 }  // namespace vsa
