@@ -20,7 +20,9 @@
 //   score_topk_kernel  one CTA per (QB query cubes, head, batch): streams the
 //                      head's kc rows once, keeps QB score rows in shared
 //                      memory as order-preserving 64-bit keys, then one warp
-//                      per query cube bitonic-sorts (key, index) pairs.
+//                      per query cube selects the topk smallest keys exactly
+//                      (radix select on 8-bit digits, ties by index) and
+//                      sorts only the selected ones.
 #include "internal.h"
 
 namespace vsa {
@@ -104,15 +106,130 @@ __device__ __forceinline__ uint64_t score_key(double s)
     return ~ord;
 }
 
+// Exact top-k of one row by radix selection on the 64-bit keys (ascending key
+// = better), run by one warp: 8-bit digits from the most significant byte
+// fix the threshold key T; the selection is every key < T plus the
+// lowest-index entries equal to T; it is then sorted by (key, index).
+__device__ void select_row(const uint64_t* __restrict__ keys, int n, int topk, int* hist, uint64_t* sel_k,
+                           uint16_t* sel_i, int ns, int32_t* __restrict__ dst, int lane)
+{
+    uint64_t prefix = 0, pmask = 0;  // decided high bits of T and their mask
+    int need = topk;                 // how many still to take at or above the current prefix
+    bool done = false;
+    for (int byte = 7; byte >= 0 && !done; --byte) {
+        for (int b = lane; b < 256; b += 32) hist[b] = 0;
+        __syncwarp();
+        const int sh = 8 * byte;
+        for (int j = lane; j < n; j += 32) {
+            const uint64_t k = keys[j];
+            if ((k & pmask) == prefix) atomicAdd(&hist[(int)((k >> sh) & 255u)], 1);
+        }
+        __syncwarp();
+        // lane owns bins 8*lane .. 8*lane+7; exclusive prefix over lanes
+        int c[8], tot = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            c[e] = hist[8 * lane + e];
+            tot += c[e];
+        }
+        int incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const int excl = incl - tot;
+        // the bucket where the running count reaches `need`
+        int found = -1, below = 0, cnt = 0;
+        if (excl < need && need <= incl) {
+            int run = excl;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                if (found < 0 && run + c[e] >= need) {
+                    found = 8 * lane + e;
+                    below = run;
+                    cnt = c[e];
+                }
+                run += c[e];
+            }
+        }
+        const uint32_t owner = __ballot_sync(0xffffffffu, found >= 0);
+        const int src = __ffs(owner) - 1;
+        found = __shfl_sync(0xffffffffu, found, src);
+        below = __shfl_sync(0xffffffffu, below, src);
+        cnt = __shfl_sync(0xffffffffu, cnt, src);
+        prefix |= (uint64_t)found << sh;
+        pmask |= (uint64_t)255u << sh;
+        need -= below;
+        if (cnt == need) done = true;  // the whole bucket is taken: no tie to break
+        __syncwarp();
+    }
+    // gather: keys below the threshold prefix, plus `need` entries of the threshold
+    // bucket in index order (all of it when done early)
+    int taken_eq = 0, pos = 0;
+    for (int base = 0; base < n; base += 32) {
+        const int j = base + lane;
+        uint64_t k = 0;
+        bool lt = false, eq = false;
+        if (j < n) {
+            k = keys[j];
+            const uint64_t hk = k & pmask;
+            lt = hk < prefix;
+            eq = hk == prefix;
+        }
+        const uint32_t meq = __ballot_sync(0xffffffffu, eq);
+        const int eq_rank = taken_eq + __popc(meq & ((1u << lane) - 1u));
+        const bool take = lt || (eq && eq_rank < need);
+        const uint32_t mt = __ballot_sync(0xffffffffu, take);
+        if (take) {
+            const int p = pos + __popc(mt & ((1u << lane) - 1u));
+            sel_k[p] = k;
+            sel_i[p] = (uint16_t)j;
+        }
+        pos += __popc(mt);
+        taken_eq += __popc(meq);
+    }
+    for (int p = pos + lane; p < ns; p += 32) {
+        sel_k[p] = ~0ull;
+        sel_i[p] = 0xFFFFu;
+    }
+    __syncwarp();
+    // bitonic sort of the ns (power of two) selected entries by (key, index)
+    for (int len = 2; len <= ns; len <<= 1) {
+        for (int stride = len >> 1; stride > 0; stride >>= 1) {
+            for (int a = lane; a < ns; a += 32) {
+                const int q = a ^ stride;
+                if (q > a) {
+                    const uint64_t ka = sel_k[a], kq = sel_k[q];
+                    const uint16_t ia = sel_i[a], iq = sel_i[q];
+                    const bool a_after = (ka > kq) || (ka == kq && ia > iq);
+                    const bool ascending = (a & len) == 0;
+                    if (a_after == ascending) {
+                        sel_k[a] = kq;
+                        sel_k[q] = ka;
+                        sel_i[a] = iq;
+                        sel_i[q] = ia;
+                    }
+                }
+            }
+            __syncwarp();
+        }
+    }
+    for (int t = lane; t < topk; t += 32) dst[t] = sel_i[t];
+    __syncwarp();
+}
+
 template <int QB>
 __global__ void __launch_bounds__(256) score_topk_kernel(const uint16_t* __restrict__ qc,
                                                          const uint16_t* __restrict__ kc, int32_t* __restrict__ topk_idx,
-                                                         int H, int nq, int np, int topk)
+                                                         int H, int nq, int ns, int topk, int sel_warps)
 {
     extern __shared__ __align__(16) uint8_t smem[];
-    double* qd = reinterpret_cast<double*>(smem);                       // [QB][D]
-    uint64_t* keys = reinterpret_cast<uint64_t*>(qd + QB * kD);         // [QB][np]
-    uint16_t* ids = reinterpret_cast<uint16_t*>(keys + (size_t)QB * np);  // [QB][np]
+    double* qd = reinterpret_cast<double*>(smem);                          // [QB][D]
+    uint64_t* keys = reinterpret_cast<uint64_t*>(qd + QB * kD);            // [QB][nq]
+    uint64_t* sel_k = keys + (size_t)QB * nq;                                       // [sel_warps][ns]
+    uint16_t* sel_i = reinterpret_cast<uint16_t*>(sel_k + (size_t)sel_warps * ns);  // [sel_warps][ns]
+    int* hist = reinterpret_cast<int*>(sel_i + (size_t)sel_warps * ns);             // [sel_warps][256]
 
     const int i0 = blockIdx.x * QB, h = blockIdx.y, b = blockIdx.z;
     const int64_t head = (int64_t)b * H + h;
@@ -123,15 +240,7 @@ __global__ void __launch_bounds__(256) score_topk_kernel(const uint16_t* __restr
     __syncthreads();
 
     const uint4* krow = reinterpret_cast<const uint4*>(kc + head * nq * kD);
-    for (int j = threadIdx.x; j < np; j += blockDim.x) {
-        if (j >= nq) {
-#pragma unroll
-            for (int r = 0; r < QB; ++r) {
-                keys[r * np + j] = ~0ull;
-                ids[r * np + j] = 0xFFFFu;
-            }
-            continue;
-        }
+    for (int j = threadIdx.x; j < nq; j += blockDim.x) {
         double acc[QB];
 #pragma unroll
         for (int r = 0; r < QB; ++r) acc[r] = 0.0;
@@ -146,41 +255,17 @@ __global__ void __launch_bounds__(256) score_topk_kernel(const uint16_t* __restr
             }
         }
 #pragma unroll
-        for (int r = 0; r < QB; ++r) {
-            keys[r * np + j] = score_key(acc[r]);
-            ids[r * np + j] = (uint16_t)j;
-        }
+        for (int r = 0; r < QB; ++r) keys[r * nq + j] = score_key(acc[r]);
     }
     __syncthreads();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int r = warp; r < QB; r += blockDim.x / 32) {
+    if (warp >= sel_warps) return;
+    for (int r = warp; r < QB; r += sel_warps) {
         const int qi = i0 + r;
         if (qi >= nq) continue;
-        uint64_t* kk = keys + (size_t)r * np;
-        uint16_t* ii = ids + (size_t)r * np;
-        for (int len = 2; len <= np; len <<= 1) {
-            for (int stride = len >> 1; stride > 0; stride >>= 1) {
-                for (int a = lane; a < np; a += 32) {
-                    const int p = a ^ stride;
-                    if (p > a) {
-                        const uint64_t ka = kk[a], kp = kk[p];
-                        const uint16_t ia = ii[a], ip = ii[p];
-                        const bool a_after = (ka > kp) || (ka == kp && ia > ip);
-                        const bool ascending = (a & len) == 0;
-                        if (a_after == ascending) {
-                            kk[a] = kp;
-                            kk[p] = ka;
-                            ii[a] = ip;
-                            ii[p] = ia;
-                        }
-                    }
-                }
-                __syncwarp();
-            }
-        }
-        int32_t* dst = topk_idx + (head * nq + qi) * topk;
-        for (int t = lane; t < topk; t += 32) dst[t] = ii[t];
+        select_row(keys + (size_t)r * nq, nq, topk, hist + warp * 256, sel_k + (size_t)warp * ns,
+                   sel_i + (size_t)warp * ns, ns, topk_idx + (head * nq + qi) * topk, lane);
     }
 }
 
@@ -199,22 +284,32 @@ cudaError_t launch_route(const uint16_t* q, const uint16_t* k, const int32_t* vb
     cube_mean_kernel<<<dim3(nq, B, 2), 128, 0, s>>>(q, k, vbs, qc, kc, S, H, nq, err);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    int np = 32;
-    while (np < nq) np <<= 1;
-    if (np <= 2048) {
-        constexpr int QB = 8;
-        size_t smem = (size_t)QB * kD * 8 + (size_t)QB * np * 10;
-        auto kern = score_topk_kernel<QB>;
+    int ns = 32;  // selection buffer: topk rounded up to a power of two
+    while (ns < topk) ns <<= 1;
+    // rows per CTA and selecting warps sized to the shared-memory budget
+    auto smem_for = [&](int qb, int w) {
+        return (size_t)qb * kD * 8 + (size_t)qb * nq * 8 + (size_t)w * ns * 10 + (size_t)w * 256 * 4;
+    };
+    const size_t budget = 200 * 1024;
+    int qb = smem_for(8, 8) <= budget ? 8 : (smem_for(4, 1) <= budget ? 4 : 2);
+    int w = qb;
+    while (w > 1 && smem_for(qb, w) > budget) w >>= 1;
+    const size_t smem = smem_for(qb, w);
+    if (qb == 8) {
+        auto kern = score_topk_kernel<8>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kern<<<dim3((nq + QB - 1) / QB, H, B), 256, smem, s>>>(qc, kc, topk_idx, H, nq, np, topk);
+        kern<<<dim3((nq + 7) / 8, H, B), 256, smem, s>>>(qc, kc, topk_idx, H, nq, ns, topk, w);
+    } else if (qb == 4) {
+        auto kern = score_topk_kernel<4>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kern<<<dim3((nq + 3) / 4, H, B), 256, smem, s>>>(qc, kc, topk_idx, H, nq, ns, topk, w);
     } else {
-        constexpr int QB = 4;
-        size_t smem = (size_t)QB * kD * 8 + (size_t)QB * np * 10;
-        auto kern = score_topk_kernel<QB>;
+        auto kern = score_topk_kernel<2>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kern<<<dim3((nq + QB - 1) / QB, H, B), 256, smem, s>>>(qc, kc, topk_idx, H, nq, np, topk);
+        kern<<<dim3((nq + 1) / 2, H, B), 256, smem, s>>>(qc, kc, topk_idx, H, nq, ns, topk, w);
     }
     return cudaGetLastError();
 }
