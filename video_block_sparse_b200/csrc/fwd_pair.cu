@@ -1,145 +1,96 @@
-// VSA fine forward on the Blackwell tensor cores, queries on TMEM lanes,
-// two query cubes per 128-row tile.
+// VSA fine forward on the Blackwell tensor cores: two query cubes per
+// 128-row tile, queries on TMEM lanes, two tiles in flight per CTA, each tile
+// ("slot") with its own producer, MMA issuer and correction warps.
 //
 // Dataset card "wan2.2_production_values", section "Operator contract": for
 // query cube i of (batch b, head h) the keys are the first vbs[j] tokens of
 // every cube j in topk_idx[b, h, i, :]; out = softmax(q k^T * sm_scale) v.
 //
 // Shape of the work on sm_100a.  A query cube has only 64 rows, and an MMA
-// with M = 64 runs the tensor core at half rate.  This kernel stacks TWO
-// query cubes (i1 rows 0-63, i2 rows 64-127) of the same (b, h) into one
-// 128-row tile and walks the union of their two selection lists, two KV
-// cubes (128 keys) per step:
-//     S[128 q x 128 keys]  = Q_tile[128 x 128 d] . K_pair^T         (M=128, N=128)
+// with M = 64 runs the tensor core at half rate, so two query cubes (i1 rows
+// 0-63, i2 rows 64-127) of the same (b, h) share one 128-row tile that walks
+// the union of their selection lists, two KV cubes (128 keys) per step:
+//     S[128 q x 128 keys]  = Q_tile[128 x 128 d] . K_pair^T       (M=128, N=128)
 //     O[128 q x 128 d]    += P[128 x 128 keys] . V_pair[128 keys x 128 d]
-// Both are tcgen05.mma (bf16 in, fp32 accumulate in TMEM); P stays in TMEM
-// (bf16, written over S) and is the A operand of the second product.  A KV
-// cube that only one of the two query cubes selected is masked (weight 0)
-// for the other cube's rows.  Cubes both lists name are walked first, so a
-// tile whose query cubes select similar cubes (the pairing that vsa_plan
-// chooses) loads each shared K/V cube once for both: the L2->SM traffic of
-// the gather, the binding resource of this operator on B200, drops with the
-// overlap of the paired lists.
+// both tcgen05.mma (bf16 in, fp32 accumulate in TMEM); P is written over S
+// in TMEM as bf16 and is the A operand of the second product.  A KV cube
+// that only one of the two query cubes selected has weight 0 for the other
+// cube's rows.  Cubes both lists name are walked first and loaded once for
+// both; vsa_plan pairs query cubes whose lists overlap most.
 //
-// Each thread of a softmax warp owns one query row (one TMEM lane), so the
-// row maximum and the row sum are thread-local: no cross-lane reduction.
+// Each softmax thread owns one query row (one TMEM lane): row maximum and row
+// sum are thread-local.  Two tiles are in flight per CTA.  A slot's chain is
+// strictly serial (QK -> softmax -> PV -> next QK, S/P reuse), so the slots
+// are made fully independent: each has its own Q, K and V buffers, its own
+// producer warp, MMA-issuing warp and correction warps, and the tensor core
+// takes whichever slot's products are ready.  No warp ever waits on the other
+// slot's progress.
 //
-// Two tiles are in flight per CTA (slots A and B), each with its own S/P
-// (128 TMEM columns) and O (128 columns); the tensor core alternates
-//     QK_A(s)  PV_B(s-1)  QK_B(s)  PV_A(s)  QK_A(s+1) ...
-// so the softmax of one slot overlaps the products of the other.
+// Roles (640 threads, one persistent CTA per SM):
+//   warps 0-3 / 4-7    softmax + epilogue of slot 0 / 1 (thread = row = lane)
+//   warps 8-11 / 12-15 O correction of slot 0 / 1: rescale the rows whose
+//                      running offset rose (thread = row)
+//   warp 16 / 18       TMA producer of slot 0 / 1: builds each tile's step list
+//                      (shared cubes first) and streams its Q, K and V tiles
+//   warp 17 / 19       MMA issuer of slot 0 / 1 (the whole warp runs the
+//                      schedule, one elected lane issues); zeroes V pad rows
+//                      inside a partial k-step before the product.  Warp 17
+//                      also owns the TMEM allocation.
 //
-// Roles (512 threads = 4 warpgroups, one persistent CTA per SM):
-//   WG0 (warps 0-3)   softmax + epilogue of slot A (thread = row = TMEM lane)
-//   WG1 (warps 4-7)   softmax + epilogue of slot B
-//   WG2 (warps 8-11)  O correction of both slots (rescale rows whose offset
-//                     rose), zeroing of V pad rows inside a partial k-step, and
-//                     the check that the step's V pair has landed
-//   WG3 warp 12       TMA producer: builds each tile's step list (shared
-//                     cubes first) and streams Q, K and V tiles
-//       warp 13       TMEM allocator and MMA issuer (one thread)
-//       warps 14-15   idle
-//
-// Softmax.  Logits are taken in base 2 (x = s * sm_scale * log2 e).  Keys at
-// or beyond vbs of their cube, and cubes the row's query cube did not
-// select, are replaced by -inf (a select, so NaN/Inf there never
-// propagates).  The running offset m of a row is raised only when the
-// step's maximum exceeds it by more than kTau (so P <= 2^kTau); only then
-// are O's row and the row sum rescaled.  The result does not depend on the
-// offsets used.  PV k-steps (16 keys) beyond ceil16(vbs) of a cube are not
-// issued; V rows between vbs and that boundary are zeroed in shared memory
-// before the product, so 0 * NaN cannot occur.
-//
-// Precise mode (VSA_FWD_PRECISE_P): P is carried as a bf16 pair hi + lo in
-// the two halves of the S columns, and the P.V product runs twice.
+// Softmax.  Logits in base 2 (x = s * sm_scale * log2 e).  Keys at or beyond
+// vbs of their cube and cubes the row's query cube did not select are
+// replaced by -inf (a select: NaN/Inf there never propagates).  The running
+// offset of a row is raised only when the step maximum exceeds it by more
+// than kTau (so P <= 2^kTau); only then are the row of O and the row sum
+// rescaled.  PV k-steps (16 keys) beyond ceil16(vbs) of a cube are not issued;
+// V rows between vbs and that boundary are zeroed before the product, so
+// 0 * NaN cannot occur.
 //
 // Every mbarrier wait is bounded (~2 s of clock): on expiry the kernel
-// latches kErrWaitTimeout, raises a CTA-wide abort flag, every role leaves
-// its loop, the producer and the MMA issuer wait (bounded) for their own
-// copies and products in flight, and TMEM is freed before exit.
-#include "internal.h"
-#include "sm100_ptx.cuh"
-
-#include <cstddef>
-#include <cuda.h>
-#include <cudaTypedefs.h>
-#include <cuda_bf16.h>
+// latches kErrWaitTimeout and raises a CTA-wide abort flag; every role leaves
+// its loop, producers and MMA issuers wait (bounded) for their own copies and
+// products in flight, and TMEM is freed before exit.
+#include "fwd_pair_common.cuh"
 
 namespace vsa {
 namespace {
 
 using namespace ptx;
 
-constexpr int kD = 128;
-constexpr int kThreads = 512;
-constexpr int kWarpProducer = 12;
-constexpr int kWarpMma = 13;
-constexpr float kTau = 8.0f;
-constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
+constexpr int kThreads = 640;
+constexpr int kWarpCorr0 = 8;  // warps 8-11 correct slot 0, 12-15 slot 1
+constexpr int kWarpRole0 = 16; // warp 16 + 2x: producer of slot x, 17 + 2x: MMA issuer of slot x
 
-constexpr uint32_t kHalfBox = 64 * 128;        // 8 KiB: 64 rows x 64 bf16 (one TMA box)
-constexpr uint32_t kTileBytes = 4 * kHalfBox;  // 128 rows x 128 d: Q tile, K pair or V pair (32 KiB)
-constexpr int kNK = 2;                         // K ring slots
-constexpr int kNV = 2;                         // V ring slots
-
-constexpr int kMaxTopk = 1024;  // per-slot list staging in shared memory
-constexpr int kMaxNq = 8192;    // per-slot membership bitmaps in shared memory
-
-// Per-step description, produced by the producer warp with each K pair.
-struct StepMeta {
-    int32_t ja, jb;   // cube ids of key halves 0 (keys 0-63) and 1 (keys 64-127)
-    int32_t na, nb;   // valid keys of each half (0: nothing loaded)
-    int32_t ma, mb;   // membership: bit 0 = query cube i1 selects it, bit 1 = i2
-    int32_t flags;    // bit 0 first step of the tile, bit 1 last step
-    int32_t vslot;    // V ring slot of this step's V pair (set by the MMA issuer)
-    int32_t vpar;     // its phase parity
-    int32_t pad[3];
+struct SlotBars {
+    uint64_t q_full, q_empty;  // Q tile landed / last QK of the tile done
+    uint64_t k_full, k_empty;  // K pair landed / QK done
+    uint64_t v_full, v_empty;  // V pair landed / PV done
+    uint64_t s_full;           // step word published + QK done (2 arrivals)
+    uint64_t a_full;           // offsets decided (128 softmax threads)
+    uint64_t p_full;           // P written and O corrected (128 softmax + 128 correction threads)
+    uint64_t o_full;           // last PV of a tile done
+    uint64_t drain;
 };
-static_assert(sizeof(StepMeta) == 48, "StepMeta layout");
-
-// The fields the other roles need, packed in one 32-bit word in shared memory:
-// na [0,7) nb [7,14) ma [14,16) mb [16,18) flags [18,20) vslot [20] vpar [21].
-__device__ __forceinline__ uint32_t step_word(const StepMeta& s)
-{
-    return (uint32_t)s.na | ((uint32_t)s.nb << 7) | ((uint32_t)s.ma << 14) | ((uint32_t)s.mb << 16) |
-           ((uint32_t)s.flags << 18);
-}
-__device__ __forceinline__ int sw_na(uint32_t w) { return (int)(w & 127u); }
-__device__ __forceinline__ int sw_nb(uint32_t w) { return (int)((w >> 7) & 127u); }
-__device__ __forceinline__ int sw_ma(uint32_t w) { return (int)((w >> 14) & 3u); }
-__device__ __forceinline__ int sw_mb(uint32_t w) { return (int)((w >> 16) & 3u); }
-__device__ __forceinline__ int sw_flags(uint32_t w) { return (int)((w >> 18) & 3u); }
-__device__ __forceinline__ int sw_vslot(uint32_t w) { return (int)((w >> 20) & 1u); }
-__device__ __forceinline__ int sw_vpar(uint32_t w) { return (int)((w >> 21) & 1u); }
 
 struct Misc {
-    uint64_t q_full[2], q_empty[2];        // per slot
-    uint64_t k_full[kNK], k_empty[kNK];
-    uint64_t v_full[kNV], v_empty[kNV];
-    uint64_t s_full[2];                    // per slot: QK done (count 2: MMA meta + commit)
-    uint64_t p_full[2];                    // per slot: P in TMEM, O corrected, V landed and its pads
-                                           // zeroed (every softmax and correction thread)
-    uint64_t a_full[2];                    // per slot: offsets decided (every softmax thread)
-    uint64_t o_full[2];                    // per slot: last PV of a tile done (commit)
-    uint64_t drain;
-    uint32_t k_meta[kNK];                  // step word of the K pair in each K slot
-    uint32_t s_meta[2];                    // step word whose S sits in each slot
+    SlotBars bar[2];
+    uint32_t k_meta[2];  // step word of the K pair in each slot's K buffer
+    uint32_t s_meta[2];  // step word of the S in each slot
     uint32_t tmem_base;
     int abort;
-    alignas(16) float alpha[2][128];       // per slot, row: O rescale factor of the current step
-    int rflag[2][4];                       // per slot, warp: some row of the warp rescales
-    uint32_t bits1[2][kMaxNq / 32];        // per slot: membership bitmap of list 1
-    uint32_t bits2[2][kMaxNq / 32];        //                           and of list 2
-    int32_t list1[2][kMaxTopk];            // per slot: the two selection lists
+    alignas(16) float alpha[2][128];  // per slot, row: O rescale factor of the current step
+    int rflag[2][4];                  // per slot, warp: some row of the warp rescales
+    uint32_t bits1[2][kMaxNq / 32];   // per slot: membership bitmap of list 1
+    uint32_t bits2[2][kMaxNq / 32];   //                           and of list 2
+    int32_t list1[2][kMaxTopk];       // per slot: the two selection lists
     int32_t list2[2][kMaxTopk];
 };
 
-template <bool PRECISE>
 struct Layout {
-    static constexpr uint32_t Q_OFF = 0;                         // two Q tiles (slots A, B)
-    static constexpr uint32_t K_OFF = Q_OFF + 2 * kTileBytes;
-    static constexpr uint32_t V_OFF = K_OFF + kNK * kTileBytes;
-    static constexpr uint32_t TILE_BYTES = V_OFF + kNV * kTileBytes;
+    static constexpr uint32_t Q_OFF = 0;                       // Q tile of slot x at Q_OFF + x * 32 KiB
+    static constexpr uint32_t K_OFF = Q_OFF + 2 * kTileBytes;  // K pair of slot x
+    static constexpr uint32_t V_OFF = K_OFF + 2 * kTileBytes;  // V pair of slot x
+    static constexpr uint32_t TILE_BYTES = V_OFF + 2 * kTileBytes;
     static constexpr uint32_t MISC_BYTES = (sizeof(Misc) + 1023) / 1024 * 1024;
     static constexpr uint32_t SMEM_BYTES = MISC_BYTES + TILE_BYTES + 1024;  // + alignment slack
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -149,348 +100,7 @@ struct Layout {
 __device__ __forceinline__ uint32_t s_col(int x) { return 256u * x; }
 __device__ __forceinline__ uint32_t o_col(int x) { return 256u * x + 128u; }
 
-__device__ __forceinline__ float ex2(float x)
-{
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
-{
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
-}
-
-__device__ __forceinline__ float max3(float a, float b, float c)
-{
-    float r;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
-}
-
-__device__ __forceinline__ float min3(float a, float b, float c)
-{
-    float r;
-    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
-}
-
-// tcgen05.mma / commit issued by one elected lane of a converged warp: the
-// operands are warp-uniform values, the predicate picks a single issuer.
-__device__ __forceinline__ void umma_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                              uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-__device__ __forceinline__ void umma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                              uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-__device__ __forceinline__ void umma_commit_elect(uint64_t* bar)
-{
-    asm volatile(
-        "{\n\t.reg .pred e;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
-            smem_u32(bar))
-        : "memory");
-}
-
-// Packed pair arithmetic (one instruction for two fp32 lanes on sm_100).
-__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0, float c1)
-{
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d0), "=f"(d1)
-        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
-}
-
-__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1)
-{
-    asm("{\n\t.reg .b64 ra, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rd, {%0, %1};\n\t"
-        "add.rn.f32x2 rd, rd, ra;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "+f"(d0), "+f"(d1)
-        : "f"(a0), "f"(a1));
-}
-
-__device__ __forceinline__ bool aborted_flag(Misc& m) { return *reinterpret_cast<volatile int*>(&m.abort) != 0; }
-
-// Bounded mbarrier wait that also gives up when another role aborted.  The
-// slow path is a real call: it is reached from many sites, and inlining it
-// everywhere would bloat the instruction footprint of the hot loops.
-__device__ __noinline__ bool wait_bar_slow(uint64_t* bar, uint32_t parity, Misc& m, int* err)
-{
-    const long long t0 = clock64();
-    for (;;) {
-        if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
-        if (aborted_flag(m)) return false;
-        if (clock64() - t0 > kWaitCycles) {
-            atomicCAS(err, 0, (int)kErrWaitTimeout);
-            *reinterpret_cast<volatile int*>(&m.abort) = 1;
-            return false;
-        }
-    }
-}
-
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Misc& m, int* err)
-{
-    if (mbar_try_wait(bar, parity)) return true;
-    return wait_bar_slow(bar, parity, m, err);
-}
-
-// The same wait fully inlined, for the softmax warps: code that runs under a
-// raised setmaxnreg budget makes no calls.
-__device__ __forceinline__ bool wait_bar_inl(uint64_t* bar, uint32_t parity, Misc& m, int* err)
-{
-    if (mbar_try_wait(bar, parity)) return true;
-    const long long t0 = clock64();
-    for (;;) {
-        if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
-        if (aborted_flag(m)) return false;
-        if (clock64() - t0 > kWaitCycles) {
-            atomicCAS(err, 0, (int)kErrWaitTimeout);
-            *reinterpret_cast<volatile int*>(&m.abort) = 1;
-            return false;
-        }
-    }
-}
-
-// Warp-uniform bounded wait: true only if every lane saw the phase complete.
-__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, Misc& m, int* err)
-{
-    const bool ok = wait_bar(bar, parity, m, err);
-    return __all_sync(0xffffffffu, ok);
-}
-
-__device__ __forceinline__ bool wait_warp_inl(uint64_t* bar, uint32_t parity, Misc& m, int* err)
-{
-    const bool ok = wait_bar_inl(bar, parity, m, err);
-    return __all_sync(0xffffffffu, ok);
-}
-
-// Short bounded wait used while draining after an abort.
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity)
-{
-    const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity))
-        if (clock64() - t0 > kWaitCycles / 4) return;
-}
-
-// 32x32b TMEM load of 32 consecutive columns of this thread's lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r)
-{
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32"
-        " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15,"
-        " %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r)
-{
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32"
-        " [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16,"
-        " %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
-        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
-        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]), "r"(r[32])
-        : "memory");
-}
-
-__device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
-{
-    asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
-}
-
-__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
-{
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-                 : "memory");
-}
-
-// The CTA's tiles are t = blockIdx.x + n * gridDim.x; tile n goes to slot n & 1.
-struct TileRef {
-    int b, h, i1, i2;  // i2 = -1: a single query cube (rows 64-127 unused)
-};
-
-__device__ __forceinline__ TileRef tile_ref(int t, int H, int nq, int tiles_per_bh, const int32_t* plan)
-{
-    TileRef r;
-    const int bh = t / tiles_per_bh, p = t - bh * tiles_per_bh;
-    r.b = bh / H;
-    r.h = bh - r.b * H;
-    if (plan != nullptr) {
-        r.i1 = __ldg(plan + 2 * (int64_t)t);
-        r.i2 = __ldg(plan + 2 * (int64_t)t + 1);
-    } else {
-        r.i1 = 2 * p;
-        r.i2 = 2 * p + 1 < nq ? 2 * p + 1 : -1;
-    }
-    return r;
-}
-
-// ------------------------------------------------------------------ step lists
-//
-// The union of a tile's two selection lists, walked in three phases:
-//   0: entries of list 2 whose cube list 1 also names   (both query cubes)
-//   1: entries of list 1 whose cube list 2 does not name (query cube i1 only)
-//   2: entries of list 2 whose cube list 1 does not name (query cube i2 only)
-// A list that names a cube twice disables the sharing (phase 0 is empty and
-// phases 1/2 take every entry), which keeps every multiplicity.  Entries
-// whose cube has no valid token are skipped.  The generator is run by the
-// whole producer warp; `next` keeps a one-entry lookahead so that each step
-// knows whether it is the tile's last.
-struct Entry {
-    int j, n, mem;  // cube, valid tokens, membership bits; mem = 0: none
-};
-
-struct ListGen {
-    int phase, base;
-    uint32_t mask;   // qualifying entries of the 32-entry window at `base`
-    bool dedupe;
-    int len1, len2;  // list lengths (0 if the query cube is absent)
-    Entry next;
-};
-
-__device__ __forceinline__ bool test_bit(const uint32_t* bits, int j) { return (bits[j >> 5] >> (j & 31)) & 1u; }
-
-// Scan forward to the next qualifying entry (warp-uniform result).
-__device__ Entry gen_pull(ListGen& g, const int32_t* l1, const int32_t* l2, const uint32_t* b1, const uint32_t* b2,
-                          const int32_t* __restrict__ vbs, uint32_t lane)
-{
-    Entry e{0, 0, 0};
-    for (;;) {
-        if (g.phase > 2) return e;
-        const int len = g.phase == 1 ? g.len1 : g.len2;
-        const int32_t* list = g.phase == 1 ? l1 : l2;
-        if (g.mask == 0) {
-            if (g.base >= len) {
-                ++g.phase;
-                g.base = 0;
-                continue;
-            }
-            const int idx = g.base + (int)lane;
-            bool q = false;
-            if (idx < len) {
-                const int j = list[idx];
-                const int n = j >= 0 ? __ldg(vbs + j) : 0;
-                if (n > 0 && n <= 64) {
-                    if (g.phase == 0)
-                        q = g.dedupe && test_bit(b1, j);
-                    else if (g.phase == 1)
-                        q = !g.dedupe || !test_bit(b2, j);
-                    else
-                        q = !g.dedupe || !test_bit(b1, j);
-                }
-            }
-            g.mask = __ballot_sync(0xffffffffu, q);
-            g.base += 32;
-            if (g.mask == 0) continue;
-        }
-        const int l = __ffs(g.mask) - 1;
-        g.mask &= g.mask - 1;
-        const int idx = g.base - 32 + l;
-        const int j = list[idx];
-        e.j = j;
-        e.n = __ldg(vbs + j);
-        e.mem = g.phase == 0 ? 3 : (g.phase == 1 ? 1 : 2);
-        return e;
-    }
-}
-
-// Stage a tile's lists and membership bitmaps in shared memory and prime the
-// generator.  Invalid cube ids latch an error and are dropped (stored as -1);
-// invalid vbs values latch an error and count as empty cubes.
-__device__ void gen_start(ListGen& g, const TileRef& t, const int32_t* __restrict__ topk_idx,
-                          const int32_t* __restrict__ vbs, int H, int nq, int topk, int32_t* l1, int32_t* l2,
-                          uint32_t* b1, uint32_t* b2, int* err, uint32_t lane)
-{
-    const int words = (nq + 31) >> 5;
-    for (int w = lane; w < words; w += 32) {
-        b1[w] = 0u;
-        b2[w] = 0u;
-    }
-    g.len1 = t.i1 >= 0 ? topk : 0;
-    g.len2 = t.i2 >= 0 ? topk : 0;
-    __syncwarp();
-    bool dup = false;
-    for (int s = 0; s < 2; ++s) {
-        const int len = s == 0 ? g.len1 : g.len2;
-        if (len == 0) continue;
-        const int i = s == 0 ? t.i1 : t.i2;
-        const int32_t* src = topk_idx + (((int64_t)t.b * H + t.h) * nq + i) * topk;
-        int32_t* dst = s == 0 ? l1 : l2;
-        uint32_t* bits = s == 0 ? b1 : b2;
-        for (int e = lane; e < len; e += 32) {
-            int j = __ldg(src + e);
-            if (j < 0 || j >= nq) {
-                atomicCAS(err, 0, (int)kErrTopkIdx);
-                j = -1;
-            } else {
-                const int n = __ldg(vbs + j);
-                if (n < 0 || n > 64) atomicCAS(err, 0, (int)kErrVbs);
-                const uint32_t old = atomicOr(&bits[j >> 5], 1u << (j & 31));
-                if (old & (1u << (j & 31))) dup = true;
-            }
-            dst[e] = j;
-        }
-    }
-    __syncwarp();
-    g.dedupe = !__any_sync(0xffffffffu, dup) && g.len1 > 0 && g.len2 > 0;
-    g.phase = g.dedupe ? 0 : 1;
-    g.base = 0;
-    g.mask = 0;
-    g.next = gen_pull(g, l1, l2, b1, b2, vbs, lane);
-}
-
-// A tile with an out-of-range plan entry latches an error; the bad cube is dropped.
-__device__ __forceinline__ TileRef checked_tile(int t, int H, int nq, int tiles_per_bh, const int32_t* plan, int* err)
-{
-    TileRef r = tile_ref(t, H, nq, tiles_per_bh, plan);
-    if (r.i1 < 0 || r.i1 >= nq) {
-        if (err != nullptr) atomicCAS(err, 0, (int)kErrPlan);
-        r.i1 = -1;
-    }
-    if (r.i2 < -1 || r.i2 >= nq) {
-        if (err != nullptr) atomicCAS(err, 0, (int)kErrPlan);
-        r.i2 = -1;
-    }
-    return r;
-}
-
-// TMA copy of one 64-token cube (both 64-wide d halves) into rows 64*part of a 128-row tile.
-__device__ __forceinline__ void load_cube(const CUtensorMap* map, uint64_t* bar, uint8_t* dst, int part, int h,
-                                          int tok)
-{
-    tma_load_3d(map, bar, dst + part * kHalfBox, 0, h, tok);
-    tma_load_3d(map, bar, dst + 2 * kHalfBox + part * kHalfBox, 64, h, tok);
-}
-
-template <bool PRECISE, bool NEG>
+template <bool NEG>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv, const int32_t* __restrict__ topk_idx,
@@ -498,7 +108,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float* __restrict__ lse, int S, int H, int nq, int topk, int tiles_per_bh, int n_tiles,
                     float scale_log2, int* err)
 {
-    using L = Layout<PRECISE>;
+    using L = Layout;
     extern __shared__ uint8_t smem_raw[];
     Misc& m = *reinterpret_cast<Misc*>(smem_raw);
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -512,30 +122,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ set-up
     if (threadIdx.x == 0) {
         for (int x = 0; x < 2; ++x) {
-            mbar_init(&m.q_full[x], 1);
-            mbar_init(&m.q_empty[x], 1);
-            mbar_init(&m.s_full[x], 2);    // MMA thread (metadata) + QK completion
-            mbar_init(&m.p_full[x], 256);  // every softmax thread of the slot + every correction thread
-            mbar_init(&m.a_full[x], 128);
-            mbar_init(&m.o_full[x], 1);
+            SlotBars& sb = m.bar[x];
+            mbar_init(&sb.q_full, 1);
+            mbar_init(&sb.q_empty, 1);
+            mbar_init(&sb.k_full, 1);
+            mbar_init(&sb.k_empty, 1);
+            mbar_init(&sb.v_full, 1);
+            mbar_init(&sb.v_empty, 1);
+            mbar_init(&sb.s_full, 2);    // MMA warp (step word) + QK completion
+            mbar_init(&sb.a_full, 128);  // every softmax thread of the slot
+            mbar_init(&sb.p_full, 256);  // every softmax and every correction thread of the slot
+            mbar_init(&sb.o_full, 1);
+            mbar_init(&sb.drain, 1);
         }
-        for (int i = 0; i < kNK; ++i) {
-            mbar_init(&m.k_full[i], 1);
-            mbar_init(&m.k_empty[i], 1);
-        }
-        for (int i = 0; i < kNV; ++i) {
-            mbar_init(&m.v_full[i], 1);
-            mbar_init(&m.v_empty[i], 1);
-        }
-        mbar_init(&m.drain, 1);
         m.abort = 0;
         fence_mbar_init();
     }
-    if (warp == kWarpMma) {
+    if (warp == kWarpRole0 + 1) {
         tmem_alloc(&m.tmem_base, 512);
         tmem_relinquish();
     }
-    if (warp == kWarpProducer && lane == 0) {
+    if (warp == kWarpRole0 && lane == 0) {
         prefetch_tmap(&tmq);
         prefetch_tmap(&tmk);
         prefetch_tmap(&tmv);
@@ -545,67 +152,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tbase = m.tmem_base;
 
-    // Registers: the softmax warpgroups hold a 128-column row of S per thread.
-    // Each warpgroup sets its budget before it splits into roles, so that the
-    // code of every role is dominated by its warpgroup's setmaxnreg.
-    if (warp >= 8) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 72;" ::: "memory");
-    if (warp == kWarpProducer) {
-        // -------------------------------------------------------- TMA producer
-        ListGen gen[2];
-        int tn[2] = {0, 1};
-        bool active[2] = {my_tiles > 0, my_tiles > 1};
-        bool need_start[2] = {true, true};
-        bool pend_v[2] = {false, false};
-        StepMeta pend[2];
-        int h_of[2] = {0, 0}, tok0_of[2] = {0, 0};
-        int ku = 0, vu = 0, qn[2] = {0, 0};
-        int armed_q[2] = {-1, -1}, armed_k[kNK], armed_v[kNV];
-        for (int i = 0; i < kNK; ++i) armed_k[i] = -1;
-        for (int i = 0; i < kNV; ++i) armed_v[i] = -1;
-        bool aborted = false;
-        while (!aborted) {
-#pragma unroll 1
-            for (int e = 0; e < 4 && !aborted; ++e) {
-                const int x = (e == 0 || e == 3) ? 0 : 1;
-                if (e == 0 || e == 2) {
-                    // ---- K pair of slot x's next step (and Q at a tile start)
-                    if (!active[x]) continue;
-                    bool first = false;
-                    if (need_start[x]) {
-                        const TileRef t =
-                            checked_tile(blockIdx.x + tn[x] * gridDim.x, H, nq, tiles_per_bh, plan, lane == 0 ? err : nullptr);
-                        gen_start(gen[x], t, topk_idx, vbs, H, nq, topk, m.list1[x], m.list2[x], m.bits1[x],
-                                  m.bits2[x], err, lane);
-                        h_of[x] = t.h;
-                        tok0_of[x] = t.b * S;
-                        if (lane == 0) {
-                            if (wait_bar(&m.q_empty[x], (qn[x] & 1) ^ 1, m, err)) {
-                                const uint32_t bytes = 2 * kHalfBox * ((t.i1 >= 0) + (t.i2 >= 0));
-                                mbar_expect_tx(&m.q_full[x], bytes);
-                                armed_q[x] = qn[x] & 1;
-                                uint8_t* qdst = tiles_ptr + L::Q_OFF + x * kTileBytes;
-                                if (t.i1 >= 0) load_cube(&tmq, &m.q_full[x], qdst, 0, t.h, t.b * S + 64 * t.i1);
-                                if (t.i2 >= 0) load_cube(&tmq, &m.q_full[x], qdst, 1, t.h, t.b * S + 64 * t.i2);
-                            } else {
-                                aborted = true;
-                            }
-                        }
-                        aborted = __shfl_sync(0xffffffffu, aborted, 0);
-                        if (aborted) break;
-                        ++qn[x];
-                        need_start[x] = false;
-                        first = true;
+    if (warp >= kWarpRole0) {
+        const int x = (warp - kWarpRole0) >> 1;
+        SlotBars& sb = m.bar[x];
+        uint8_t* qdst = tiles_ptr + L::Q_OFF + x * kTileBytes;
+        uint8_t* kdst = tiles_ptr + L::K_OFF + x * kTileBytes;
+        uint8_t* vdst = tiles_ptr + L::V_OFF + x * kTileBytes;
+        if (((warp - kWarpRole0) & 1) == 0) {
+            // ---------------------------------------------------- TMA producer of slot x
+            ListGen gen;
+            int qn = 0, kc = 0;
+            int armed_q = -1, armed_k = -1, armed_v = -1;
+            bool aborted = false;
+            for (int n = x; n < my_tiles && !aborted; n += 2) {
+                const TileRef t =
+                    checked_tile(blockIdx.x + n * gridDim.x, H, nq, tiles_per_bh, plan, lane == 0 ? err : nullptr);
+                gen_start(gen, t, topk_idx, vbs, H, nq, topk, m.list1[x], m.list2[x], m.bits1[x], m.bits2[x], err,
+                          lane);
+                const int tok0 = t.b * S;
+                if (lane == 0) {
+                    if (wait_bar(&sb.q_empty, (qn & 1) ^ 1, &m.abort, err)) {
+                        mbar_expect_tx(&sb.q_full, 2 * kHalfBox * ((t.i1 >= 0) + (t.i2 >= 0)));
+                        armed_q = qn & 1;
+                        if (t.i1 >= 0) load_cube(&tmq, &sb.q_full, qdst, 0, t.h, tok0 + 64 * t.i1);
+                        if (t.i2 >= 0) load_cube(&tmq, &sb.q_full, qdst, 1, t.h, tok0 + 64 * t.i2);
+                    } else {
+                        aborted = true;
                     }
-                    ListGen& G = gen[x];
-                    const Entry ea = G.next;
+                }
+                aborted = __shfl_sync(0xffffffffu, aborted, 0);
+                ++qn;
+                bool first = true;
+                while (!aborted) {
+                    const Entry ea = gen.next;
                     Entry eb{0, 0, 0};
                     if (ea.mem != 0) {
-                        G.next = gen_pull(G, m.list1[x], m.list2[x], m.bits1[x], m.bits2[x], vbs, lane);
-                        eb = G.next;
-                        if (eb.mem != 0) G.next = gen_pull(G, m.list1[x], m.list2[x], m.bits1[x], m.bits2[x], vbs, lane);
+                        gen.next = gen_pull(gen, m.list1[x], m.list2[x], m.bits1[x], m.bits2[x], vbs, lane);
+                        eb = gen.next;
+                        if (eb.mem != 0) gen.next = gen_pull(gen, m.list1[x], m.list2[x], m.bits1[x], m.bits2[x], vbs, lane);
                     }
-                    const bool last = G.next.mem == 0;
+                    const bool last = gen.next.mem == 0;
                     StepMeta meta;
                     meta.ja = ea.j;
                     meta.jb = eb.j;
@@ -614,186 +200,133 @@ __global__ void __launch_bounds__(kThreads, 1)
                     meta.ma = ea.mem;
                     meta.mb = eb.mem;
                     meta.flags = (first ? 1 : 0) | (last ? 2 : 0);
-                    meta.vslot = 0;
-                    meta.vpar = 0;
+                    first = false;
+                    const uint32_t bytes = 2 * kHalfBox * ((meta.na > 0) + (meta.nb > 0));
                     if (lane == 0) {
-                        const int ks = ku % kNK;
-                        if (wait_bar(&m.k_empty[ks], ((ku / kNK) & 1) ^ 1, m, err)) {
-                            m.k_meta[ks] = step_word(meta);
-                            const uint32_t bytes = 2 * kHalfBox * ((meta.na > 0) + (meta.nb > 0));
-                            mbar_expect_tx(&m.k_full[ks], bytes);
-                            armed_k[ks] = (ku / kNK) & 1;
-                            uint8_t* kdst = tiles_ptr + L::K_OFF + ks * kTileBytes;
-                            if (meta.na > 0) load_cube(&tmk, &m.k_full[ks], kdst, 0, h_of[x], tok0_of[x] + 64 * meta.ja);
-                            if (meta.nb > 0) load_cube(&tmk, &m.k_full[ks], kdst, 1, h_of[x], tok0_of[x] + 64 * meta.jb);
+                        // K pair of the step: the buffer is free once the previous QK finished
+                        if (wait_bar(&sb.k_empty, (kc & 1) ^ 1, &m.abort, err)) {
+                            m.k_meta[x] = step_word(meta);
+                            mbar_expect_tx(&sb.k_full, bytes);
+                            armed_k = kc & 1;
+                            if (meta.na > 0) load_cube(&tmk, &sb.k_full, kdst, 0, t.h, tok0 + 64 * meta.ja);
+                            if (meta.nb > 0) load_cube(&tmk, &sb.k_full, kdst, 1, t.h, tok0 + 64 * meta.jb);
+                        } else {
+                            aborted = true;
+                        }
+                        // V pair of the step: free once the previous PV finished
+                        if (!aborted && wait_bar(&sb.v_empty, (kc & 1) ^ 1, &m.abort, err)) {
+                            mbar_expect_tx(&sb.v_full, bytes);
+                            armed_v = kc & 1;
+                            if (meta.na > 0) load_cube(&tmv, &sb.v_full, vdst, 0, t.h, tok0 + 64 * meta.ja);
+                            if (meta.nb > 0) load_cube(&tmv, &sb.v_full, vdst, 1, t.h, tok0 + 64 * meta.jb);
                         } else {
                             aborted = true;
                         }
                     }
                     aborted = __shfl_sync(0xffffffffu, aborted, 0);
-                    ++ku;
-                    pend[x] = meta;
-                    pend_v[x] = true;
-                    if (last) {
-                        tn[x] += 2;
-                        need_start[x] = true;
-                        active[x] = tn[x] < my_tiles;
-                    }
-                } else {
-                    // ---- V pair of slot x's pending step
-                    if (!pend_v[x]) continue;
-                    if (lane == 0) {
-                        const int vs = vu % kNV;
-                        if (wait_bar(&m.v_empty[vs], ((vu / kNV) & 1) ^ 1, m, err)) {
-                            const StepMeta& p = pend[x];
-                            const uint32_t bytes = 2 * kHalfBox * ((p.na > 0) + (p.nb > 0));
-                            mbar_expect_tx(&m.v_full[vs], bytes);
-                            armed_v[vs] = (vu / kNV) & 1;
-                            uint8_t* vdst = tiles_ptr + L::V_OFF + vs * kTileBytes;
-                            if (p.na > 0) load_cube(&tmv, &m.v_full[vs], vdst, 0, h_of[x], tok0_of[x] + 64 * p.ja);
-                            if (p.nb > 0) load_cube(&tmv, &m.v_full[vs], vdst, 1, h_of[x], tok0_of[x] + 64 * p.jb);
-                        } else {
-                            aborted = true;
-                        }
-                    }
-                    aborted = __shfl_sync(0xffffffffu, aborted, 0);
-                    ++vu;
-                    pend_v[x] = false;
+                    ++kc;
+                    if (last) break;
                 }
             }
-            if (!active[0] && !active[1] && !pend_v[0] && !pend_v[1]) break;
-        }
-        if (aborted && lane == 0) {
-            // copies issued by this thread must land before the CTA's shared memory goes away
-            for (int x = 0; x < 2; ++x)
-                if (armed_q[x] >= 0) drain_wait(&m.q_full[x], armed_q[x]);
-            for (int i = 0; i < kNK; ++i)
-                if (armed_k[i] >= 0) drain_wait(&m.k_full[i], armed_k[i]);
-            for (int i = 0; i < kNV; ++i)
-                if (armed_v[i] >= 0) drain_wait(&m.v_full[i], armed_v[i]);
-        }
-    } else if (warp == kWarpMma) {
-        // -------------------------------------------------------- MMA issuer
-        // The whole warp runs the schedule (every value below is warp-uniform);
-        // each tcgen05.mma / commit is issued by one elected lane.
-        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);
-        // Descriptors of every operand tile, built once; a k-step only adds its
-        // byte offset / 16 to the start-address field (no carry: smem < 256 KiB).
-        const uint64_t d_hi = smem_desc_sw128(0, 0, 1024);  // SBO, version, swizzle: shared by all
-        const uint32_t q_lo0 = (uint32_t)smem_desc_sw128(tiles + L::Q_OFF, 16, 1024);
-        const uint32_t k_lo0 = (uint32_t)smem_desc_sw128(tiles + L::K_OFF, 16, 1024);
-        const uint32_t v_lo0 = (uint32_t)smem_desc_sw128(tiles + L::V_OFF, 2 * kHalfBox, 1024);
-        int tn[2] = {0, 1}, g[2] = {0, 0}, qn[2] = {0, 0};
-        bool active[2] = {my_tiles > 0, my_tiles > 1};
-        bool pending[2] = {false, false}, new_tile[2] = {true, true}, o_init[2] = {false, false};
-        uint32_t cur[2] = {0u, 0u};
-        int ku = 0, vu = 0;
-        bool aborted = false;
-        while (!aborted) {
-#pragma unroll
-            for (int e = 0; e < 4 && !aborted; ++e) {
-                const int x = (e == 0 || e == 3) ? 0 : 1;
-                if (e == 0 || e == 2) {
-                    // ---- S_x = Q_x . K^T
-                    if (!active[x]) continue;
-                    if (new_tile[x]) {
-                        if (!wait_warp(&m.q_full[x], qn[x] & 1, m, err)) { aborted = true; break; }
-                        ++qn[x];
-                        new_tile[x] = false;
-                        o_init[x] = false;
-                    }
-                    const int ks = ku % kNK;
-                    if (!wait_warp(&m.k_full[ks], (ku / kNK) & 1, m, err)) { aborted = true; break; }
-                    const int vidx = vu + (pending[x ^ 1] ? 1 : 0);  // V uses before this step's PV
-                    const uint32_t meta =
-                        m.k_meta[ks] | ((uint32_t)(vidx % kNV) << 20) | ((uint32_t)((vidx / kNV) & 1) << 21);
+            if (aborted && lane == 0) {
+                // copies issued by this thread must land before the CTA's shared memory goes away
+                if (armed_q >= 0) drain_wait(&sb.q_full, armed_q);
+                if (armed_k >= 0) drain_wait(&sb.k_full, armed_k);
+                if (armed_v >= 0) drain_wait(&sb.v_full, armed_v);
+            }
+        } else {
+            // ---------------------------------------------------- MMA issuer of slot x
+            constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);
+            // operand descriptors built once; a k-step adds its byte offset / 16
+            const uint64_t d_hi = smem_desc_sw128(0, 0, 1024);
+            const uint32_t ql = (uint32_t)smem_desc_sw128(smem_u32(qdst), 16, 1024);
+            const uint32_t kl = (uint32_t)smem_desc_sw128(smem_u32(kdst), 16, 1024);
+            const uint32_t vl = (uint32_t)smem_desc_sw128(smem_u32(vdst), 2 * kHalfBox, 1024);
+            const uint32_t s_tmem = tbase + s_col(x), o_tmem = tbase + o_col(x);
+            int qn = 0, kc = 0;
+            bool aborted = false;
+            for (int n = x; n < my_tiles && !aborted; n += 2) {
+                if (!wait_warp(&sb.q_full, qn & 1, &m.abort, err)) { aborted = true; break; }
+                ++qn;
+                bool o_init = false;
+                for (;;) {
+                    // ---- S = Q . K^T
+                    if (!wait_warp(&sb.k_full, kc & 1, &m.abort, err)) { aborted = true; break; }
+                    const uint32_t meta = m.k_meta[x];
                     __syncwarp();
                     if (lane == 0) {
                         m.s_meta[x] = meta;
-                        mbar_arrive(&m.s_full[x]);  // publishes s_meta (release)
+                        mbar_arrive(&sb.s_full);  // publishes the step word (release)
                     }
                     __syncwarp();
                     tc_fence_after();
-                    const uint32_t ql = q_lo0 + x * (kTileBytes >> 4), kl = k_lo0 + ks * (kTileBytes >> 4);
-                    const uint32_t s_tmem = tbase + s_col(x);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t off = ((kk >> 2) * (2 * kHalfBox) + (kk & 3) * 32u) >> 4;
                         umma_ss_elect(s_tmem, d_hi | (ql + off), d_hi | (kl + off), idesc_qk, kk > 0 ? 1u : 0u);
                     }
-                    umma_commit_elect(&m.s_full[x]);
-                    umma_commit_elect(&m.k_empty[ks]);
-                    ++ku;
-                    cur[x] = meta;
-                    pending[x] = true;
-                    if (sw_flags(meta) & 2) {
-                        umma_commit_elect(&m.q_empty[x]);
-                        tn[x] += 2;
-                        new_tile[x] = true;
-                        active[x] = tn[x] < my_tiles;
+                    umma_commit_elect(&sb.s_full);
+                    umma_commit_elect(&sb.k_empty);
+                    const bool last = (sw_flags(meta) & 2) != 0;
+                    if (last) umma_commit_elect(&sb.q_empty);
+                    // ---- O += P . V
+                    if (!wait_warp(&sb.p_full, kc & 1, &m.abort, err)) { aborted = true; break; }
+                    if (!wait_warp(&sb.v_full, kc & 1, &m.abort, err)) { aborted = true; break; }
+                    const int na = sw_na(meta), nb = sw_nb(meta);
+                    const int za = (na & 15) ? 16 - (na & 15) : 0, zb = (nb & 15) ? 16 - (nb & 15) : 0;
+                    if (za + zb > 0) {
+                        // V rows between vbs and the next multiple of 16 are read by the last
+                        // k-step of their cube: zero them (both d halves) before the product
+                        const uint32_t vb = smem_u32(vdst);
+                        for (int w = lane; w < (za + zb) * 16; w += 32) {
+                            const int zr = w >> 4, chunk = w & 15;
+                            const int row = zr < za ? na + zr : 64 + nb + (zr - za);
+                            sts128(vb + (chunk >> 3) * (2 * kHalfBox) + row * 128 + (chunk & 7) * 16, 0u, 0u, 0u, 0u);
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
                     }
-                } else {
-                    // ---- O_x += P_x . V
-                    if (!pending[x]) continue;
-                    const uint32_t c = cur[x];
-                    // one wait: P written, O corrected, V landed (the correction waited for it)
-                    if (!wait_warp(&m.p_full[x], g[x] & 1, m, err)) { aborted = true; break; }
                     tc_fence_after();
-                    const uint32_t vl = v_lo0 + sw_vslot(c) * (kTileBytes >> 4);
-                    const uint32_t p_tmem = tbase + s_col(x), o_tmem = tbase + o_col(x);
                     // k-steps (16 keys) 0..ceil16(na)-1 of half 0 and 4..4+ceil16(nb)-1 of half 1
-                    const uint32_t kmask =
-                        ((1u << ((sw_na(c) + 15) >> 4)) - 1u) | (((1u << ((sw_nb(c) + 15) >> 4)) - 1u) << 4);
-                    uint32_t acc = o_init[x] ? 1u : 0u;
+                    const uint32_t kmask = ((1u << ((na + 15) >> 4)) - 1u) | (((1u << ((nb + 15) >> 4)) - 1u) << 4);
+                    uint32_t acc = o_init ? 1u : 0u;
 #pragma unroll
                     for (int kstep = 0; kstep < 8; ++kstep) {
                         if (kmask & (1u << kstep)) {
-                            const uint64_t bd = d_hi | (vl + ((kstep * 2048) >> 4));
-                            umma_ts_elect(o_tmem, p_tmem + kstep * 8, bd, idesc_pv, acc);
+                            umma_ts_elect(o_tmem, s_tmem + kstep * 8, d_hi | (vl + ((kstep * 2048) >> 4)), idesc_pv, acc);
                             acc = 1u;
-                            if (PRECISE) umma_ts_elect(o_tmem, p_tmem + 64 + kstep * 8, bd, idesc_pv, 1u);
                         }
                     }
-                    o_init[x] = o_init[x] || kmask != 0;
-                    umma_commit_elect(&m.v_empty[sw_vslot(c)]);
-                    if (sw_flags(c) & 2) umma_commit_elect(&m.o_full[x]);
-                    ++vu;
-                    ++g[x];
-                    pending[x] = false;
+                    o_init = o_init || kmask != 0;
+                    umma_commit_elect(&sb.v_empty);
+                    if (last) umma_commit_elect(&sb.o_full);
+                    ++kc;
+                    if (last) break;
                 }
             }
-            if (!active[0] && !active[1] && !pending[0] && !pending[1]) break;
+            if (aborted) {
+                umma_commit_elect(&sb.drain);
+                if (lane == 0) drain_wait(&sb.drain, 0);
+                __syncwarp();
+            }
         }
-        if (aborted) {
-            umma_commit_elect(&m.drain);
-            if (lane == 0) drain_wait(&m.drain, 0);
-            __syncwarp();
-        }
-    } else if (warp < kWarpProducer) {
-        // -------------------------------------------------------- correction (warps 8-11)
-        const int wq = warp & 3;
+    } else if (warp >= kWarpCorr0) {
+        // -------------------------------------------------------- O correction of slot x
+        const int x = (warp - kWarpCorr0) >> 2, wq = warp & 3;
         const int r = 32 * wq + (int)lane;
-        const uint32_t lane_base = tbase + ((uint32_t)(32 * wq) << 16);
-        int tn[2] = {0, 1}, g[2] = {0, 0};
-        bool active[2] = {my_tiles > 0, my_tiles > 1};
-        bool pending[2] = {false, false};
-        for (;;) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int x = (e == 0 || e == 3) ? 0 : 1;
-                if (e == 0 || e == 2) {
-                    pending[x] = active[x];  // the MMA issues QK_x here
-                    continue;
-                }
-                if (!pending[x]) continue;
-                if (!wait_warp(&m.a_full[x], g[x] & 1, m, err)) goto corr_exit;
+        SlotBars& sb = m.bar[x];
+        const uint32_t oa = tbase + ((uint32_t)(32 * wq) << 16) + o_col(x);
+        int g = 0;
+        for (int n = x; n < my_tiles; n += 2) {
+            for (;;) {
+                if (!wait_warp(&sb.a_full, g & 1, &m.abort, err)) goto corr_exit;
                 const uint32_t meta = m.s_meta[x];
                 tc_fence_after();
                 if (!(sw_flags(meta) & 1) && m.rflag[x][wq] != 0) {
-                    // O row r *= alpha (1 for rows whose offset stayed)
+                    // O row r *= alpha (1 for rows whose offset stayed); the previous
+                    // P.V of the slot finished before this step's S was published
                     const float a = m.alpha[x][r];
-                    const uint32_t oa = lane_base + o_col(x);
 #pragma unroll 1
                     for (int c4 = 0; c4 < 4; ++c4) {
                         uint32_t o[32];
@@ -805,40 +338,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tmem_st_wait();
                 }
-                // V rows between vbs and the next multiple of 16 are read by the last
-                // k-step of their cube: zero them (both d halves) before the product
-                const int mna = sw_na(meta), mnb = sw_nb(meta);
-                const int za = (mna & 15) ? 16 - (mna & 15) : 0;
-                const int zb = (mnb & 15) ? 16 - (mnb & 15) : 0;
-                if (!wait_warp(&m.v_full[sw_vslot(meta)], sw_vpar(meta), m, err)) goto corr_exit;
-                if (za + zb > 0) {
-                    const uint32_t vb = tiles + L::V_OFF + sw_vslot(meta) * kTileBytes;
-                    for (int w = r; w < (za + zb) * 16; w += 128) {
-                        const int zr = w >> 4, chunk = w & 15;
-                        const int row = zr < za ? mna + zr : 64 + mnb + (zr - za);
-                        sts128(vb + (chunk >> 3) * (2 * kHalfBox) + row * 128 + (chunk & 7) * 16, 0u, 0u, 0u, 0u);
-                    }
-                    fence_proxy_async_smem();
-                }
                 tc_fence_before();
-                mbar_arrive(&m.p_full[x]);
-                ++g[x];
-                pending[x] = false;
-                if (sw_flags(meta) & 2) {
-                    tn[x] += 2;
-                    active[x] = tn[x] < my_tiles;
-                }
+                mbar_arrive(&sb.p_full);
+                ++g;
+                if (sw_flags(meta) & 2) break;
             }
-            if (!active[0] && !active[1] && !pending[0] && !pending[1]) break;
         }
     corr_exit:;
-    }
     } else {
-        // -------------------------------------------------------- softmax + epilogue (warps 0-7)
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 184;" ::: "memory");
+        // -------------------------------------------------------- softmax + epilogue of slot x
         const int x = warp >> 2, wq = warp & 3;
         const int r = 32 * wq + (int)lane;  // query row of the tile == TMEM lane
         const int qbit = r >> 6;            // 0: query cube i1, 1: i2
+        SlotBars& sb = m.bar[x];
         const uint32_t lane_base = tbase + ((uint32_t)(32 * wq) << 16);
         const uint32_t s_addr = lane_base + s_col(x), o_addr = lane_base + o_col(x);
         constexpr float kNeutral = NEG ? INFINITY : -INFINITY;  // a masked logit
@@ -847,115 +359,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int n = x; n < my_tiles; n += 2, ++tc) {
             const TileRef t = checked_tile(blockIdx.x + n * gridDim.x, H, nq, tiles_per_bh, plan, nullptr);
             for (;;) {
-                if (!wait_warp_inl(&m.s_full[x], g & 1, m, err)) goto softmax_exit;
+                if (!wait_warp_inl(&sb.s_full, g & 1, &m.abort, err)) goto softmax_exit;
                 const uint32_t meta = m.s_meta[x];
                 const int na = sw_na(meta), nb = sw_nb(meta), ma = sw_ma(meta), mb = sw_mb(meta), flags = sw_flags(meta);
-                const int myn[2] = {((ma >> qbit) & 1) ? na : 0, ((mb >> qbit) & 1) ? nb : 0};
+                const int myn0 = ((ma >> qbit) & 1) ? na : 0, myn1 = ((mb >> qbit) & 1) ? nb : 0;
                 if (flags & 1) {
                     m_run = -INFINITY;
                     l_run = 0.f;
                 }
                 tc_fence_after();
-                if constexpr (!PRECISE) {
-                    // pass 1: row extreme over the selected keys, one 32-column TMEM load
-                    // at a time (small loop bodies keep the hot code in the instruction cache)
-                    float e4[4] = {kNeutral, kNeutral, kNeutral, kNeutral};
-#pragma unroll 1
-                    for (int ch = 0; ch < 4; ++ch) {
-                        const int nv = ch < 2 ? myn[0] : myn[1];
-                        const int cb = (ch & 1) * 32;  // first column of the chunk in its 64-key half
-                        if (nv <= cb) continue;        // no selected key in this chunk
-                        float sc[32];
-                        tmem_ld32(s_addr + 32 * ch, reinterpret_cast<uint32_t*>(sc));
-                        tmem_ld_wait();
-                        if (nv < cb + 32) {
-#pragma unroll
-                            for (int c = 0; c < 32; ++c) sc[c] = cb + c < nv ? sc[c] : kNeutral;
-                        }
-#pragma unroll
-                        for (int c = 0; c < 32; c += 8) {
-#pragma unroll
-                            for (int u = 0; u < 4; ++u)
-                                e4[u] = NEG ? min3(e4[u], sc[c + 2 * u], sc[c + 2 * u + 1])
-                                            : max3(e4[u], sc[c + 2 * u], sc[c + 2 * u + 1]);
-                        }
-                    }
-                    const float ext = NEG ? min3(fminf(e4[0], e4[1]), e4[2], e4[3]) : max3(fmaxf(e4[0], e4[1]), e4[2], e4[3]);
-                    const bool any_valid = (myn[0] | myn[1]) != 0;
-                    const float m_step = any_valid ? ext * scale_log2 : -INFINITY;  // base-2 units
-                    const bool raise = m_step > m_run + kTau;                    // false for -inf
-                    float alpha = 1.f;
-                    if (raise) {
-                        alpha = m_run == -INFINITY ? 0.f : ex2(m_run - m_step);
-                        m_run = m_step;
-                        l_run *= alpha;
-                    }
-                    m.alpha[x][r] = alpha;
-                    const bool warp_raise = __any_sync(0xffffffffu, raise && !(flags & 1));
-                    if (lane == 0) m.rflag[x][wq] = warp_raise ? 1 : 0;
-                    mbar_arrive(&m.a_full[x]);
-
-                    // pass 2: P = exp2(x - m) as bf16 pairs over S's first 64 columns; the
-                    // chunk's P lands on columns whose logits were already consumed
-                    const float mu = m_run == -INFINITY ? 0.f : m_run;
-                    float ls0 = 0.f, ls1 = 0.f;
-#pragma unroll 1
-                    for (int ch = 0; ch < 4; ++ch) {
-                        const int nv = ch < 2 ? myn[0] : myn[1];
-                        const int cb = (ch & 1) * 32;
-                        uint32_t pk[16];
-                        if (nv <= cb) {
-#pragma unroll
-                            for (int c = 0; c < 16; ++c) pk[c] = 0u;
-                        } else {
-                            float sc[32];
-                            tmem_ld32(s_addr + 32 * ch, reinterpret_cast<uint32_t*>(sc));
-                            tmem_ld_wait();
-                            if (nv < cb + 32) {
-#pragma unroll
-                                for (int c = 0; c < 32; ++c) sc[c] = cb + c < nv ? sc[c] : kNeutral;
-                            }
-#pragma unroll
-                            for (int c = 0; c < 16; ++c) {
-                                float x0, x1;
-                                ffma2(x0, x1, sc[2 * c], sc[2 * c + 1], scale_log2, scale_log2, -mu, -mu);
-                                const float p0 = ex2(x0), p1 = ex2(x1);
-                                fadd2(ls0, ls1, p0, p1);
-                                pk[c] = pack_bf16(p0, p1);
-                            }
-                        }
-                        tmem_st16(s_addr + 16 * ch, pk);
-                    }
-                    l_run += ls0 + ls1;
-                } else {
-                float s[128];
-                tmem_ld32(s_addr, reinterpret_cast<uint32_t*>(&s[0]));
-                tmem_ld32(s_addr + 32, reinterpret_cast<uint32_t*>(&s[32]));
-                tmem_ld32(s_addr + 64, reinterpret_cast<uint32_t*>(&s[64]));
-                tmem_ld32(s_addr + 96, reinterpret_cast<uint32_t*>(&s[96]));
-                tmem_ld_wait();
-
-                // keys outside the row's selection take the neutral value (a select:
-                // NaN/Inf from unselected or padded keys never propagates)
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    const int nv = myn[hf];
-                    if (nv < 64) {
-#pragma unroll
-                        for (int c = 0; c < 64; ++c) s[64 * hf + c] = c < nv ? s[64 * hf + c] : kNeutral;
-                    }
-                }
-                // row extreme of the raw logits (max for a positive scale, min for a negative one)
+                // pass 1: row extreme over the selected keys, one 32-column TMEM load at a
+                // time (small loop bodies keep the hot code in the instruction cache)
                 float e4[4] = {kNeutral, kNeutral, kNeutral, kNeutral};
+#pragma unroll 1
+                for (int ch = 0; ch < 4; ++ch) {
+                    const int nv = ch < 2 ? myn0 : myn1;
+                    const int cb = (ch & 1) * 32;  // first column of the chunk in its 64-key half
+                    if (nv <= cb) continue;        // no selected key in this chunk
+                    float sc[32];
+                    tmem_ld32(s_addr + 32 * ch, reinterpret_cast<uint32_t*>(sc));
+                    tmem_ld_wait();
+                    if (nv < cb + 32) {
 #pragma unroll
-                for (int c = 0; c < 128; c += 8) {
+                        for (int c = 0; c < 32; ++c) sc[c] = cb + c < nv ? sc[c] : kNeutral;
+                    }
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        e4[u] = NEG ? min3(e4[u], s[c + 2 * u], s[c + 2 * u + 1])
-                                    : max3(e4[u], s[c + 2 * u], s[c + 2 * u + 1]);
+                    for (int c = 0; c < 32; c += 8) {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            e4[u] = NEG ? min3(e4[u], sc[c + 2 * u], sc[c + 2 * u + 1])
+                                        : max3(e4[u], sc[c + 2 * u], sc[c + 2 * u + 1]);
+                    }
                 }
                 const float ext = NEG ? min3(fminf(e4[0], e4[1]), e4[2], e4[3]) : max3(fmaxf(e4[0], e4[1]), e4[2], e4[3]);
-                const bool any_valid = (myn[0] | myn[1]) != 0;
+                const bool any_valid = (myn0 | myn1) != 0;
                 const float m_step = any_valid ? ext * scale_log2 : -INFINITY;  // base-2 units
                 const bool raise = m_step > m_run + kTau;                    // false for -inf
                 float alpha = 1.f;
@@ -967,59 +404,56 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m.alpha[x][r] = alpha;
                 const bool warp_raise = __any_sync(0xffffffffu, raise && !(flags & 1));
                 if (lane == 0) m.rflag[x][wq] = warp_raise ? 1 : 0;
-                mbar_arrive(&m.a_full[x]);
+                mbar_arrive(&sb.a_full);
 
-                // P = exp2(x - m) as bf16 pairs over S's first 64 columns (hi part
-                // of the precise mode; its lo part goes to columns 64-127)
+                // pass 2: P = exp2(x - m) as bf16 pairs over S's first 64 columns; the
+                // chunk's P lands on columns whose logits were already consumed
                 const float mu = m_run == -INFINITY ? 0.f : m_run;
-                float ls[4] = {0.f, 0.f, 0.f, 0.f};
-                // 16 columns of P (32 keys) per TMEM store; S is already in registers,
-                // so writing P over S's leading columns is safe
-#pragma unroll
+                float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll 1
                 for (int ch = 0; ch < 4; ++ch) {
+                    const int nv = ch < 2 ? myn0 : myn1;
+                    const int cb = (ch & 1) * 32;
                     uint32_t pk[16];
-                    uint32_t pl[16];
-                    if (myn[ch >> 1] == 0) {
+                    if (nv <= cb) {
 #pragma unroll
-                        for (int c = 0; c < 16; ++c) {
-                            pk[c] = 0u;
-                            pl[c] = 0u;
-                        }
+                        for (int c = 0; c < 16; ++c) pk[c] = 0u;
                     } else {
+                        float sc[32];
+                        tmem_ld32(s_addr + 32 * ch, reinterpret_cast<uint32_t*>(sc));
+                        tmem_ld_wait();
+                        if (nv < cb + 32) {
+#pragma unroll
+                            for (int c = 0; c < 32; ++c) sc[c] = cb + c < nv ? sc[c] : kNeutral;
+                        }
 #pragma unroll
                         for (int c = 0; c < 16; ++c) {
-                            const float p0 = ex2(fmaf(s[32 * ch + 2 * c], scale_log2, -mu));
-                            const float p1 = ex2(fmaf(s[32 * ch + 2 * c + 1], scale_log2, -mu));
-                            ls[c & 3] += p0 + p1;
-                            const uint32_t hb = pack_bf16(p0, p1);
-                            pk[c] = hb;
-                            if (PRECISE) {
-                                const float a0 = __uint_as_float(hb << 16), a1 = __uint_as_float(hb & 0xFFFF0000u);
-                                pl[c] = pack_bf16(p0 - a0, p1 - a1);
-                            }
+                            float x0, x1;
+                            ffma2(x0, x1, sc[2 * c], sc[2 * c + 1], scale_log2, scale_log2, -mu, -mu);
+                            const float p0 = ex2(x0), p1 = ex2(x1);
+                            fadd2(ls0, ls1, p0, p1);
+                            pk[c] = pack_bf16(p0, p1);
                         }
                     }
                     tmem_st16(s_addr + 16 * ch, pk);
-                    if (PRECISE) tmem_st16(s_addr + 64 + 16 * ch, pl);
                 }
-                l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-                }
+                l_run += ls0 + ls1;
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(&m.p_full[x]);
+                mbar_arrive(&sb.p_full);
                 ++g;
                 if (flags & 2) break;
             }
 
             // ---- epilogue: out[b, 64 i + (r % 64), h, :] = O[r, :] / l; lse = (m + log2 l) ln 2
-            if (!wait_warp_inl(&m.o_full[x], tc & 1, m, err)) goto softmax_exit;
+            if (!wait_warp_inl(&sb.o_full, tc & 1, &m.abort, err)) goto softmax_exit;
             tc_fence_after();
             {
                 const int cube = qbit == 0 ? t.i1 : t.i2;
                 const float inv = l_run > 0.f ? __frcp_rn(l_run) : 0.f;
                 const int64_t token = (int64_t)t.b * S + 64LL * cube + (r & 63);
                 uint16_t* dst = out + (token * H + t.h) * kD;
-#pragma unroll
+#pragma unroll 1
                 for (int c4 = 0; c4 < 4; ++c4) {
                     uint32_t o[32];
                     tmem_ld32(o_addr + 32 * c4, o);
@@ -1048,44 +482,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == kWarpMma) tmem_dealloc(tbase, 512);
+    if (warp == kWarpRole0 + 1) tmem_dealloc(tbase, 512);
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
-{
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (fn == nullptr) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
-
-// [B*S tokens][H][D] bf16 viewed as a 3-D tensor; box = 64 d x 1 head x 64 tokens.
-bool make_map(CUtensorMap* map, const void* base, int64_t tokens, int H)
-{
-    auto enc = encode_fn();
-    if (enc == nullptr) return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)tokens};
-    const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2};
-    const cuuint32_t box[3] = {64, 1, 64};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-template <bool PRECISE, bool NEG>
+template <bool NEG>
 cudaError_t launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const int32_t* topk_idx,
                    const int32_t* vbs, const int32_t* plan, uint16_t* out, float* lse, int B, int S, int H, int nq,
                    int topk, float scale_log2, int* err, cudaStream_t s)
 {
-    using L = Layout<PRECISE>;
-    auto kern = fwd_pair_kernel<PRECISE, NEG>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::SMEM_BYTES);
+    auto kern = fwd_pair_kernel<NEG>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Layout::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -1093,8 +499,8 @@ cudaError_t launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
     const int tiles_per_bh = (nq + 1) / 2;
     const int n_tiles = B * H * tiles_per_bh;
     const int grid = n_tiles < sms ? n_tiles : sms;
-    kern<<<grid, kThreads, L::SMEM_BYTES, s>>>(mq, mk, mv, topk_idx, vbs, plan, out, lse, S, H, nq, topk,
-                                               tiles_per_bh, n_tiles, scale_log2, err);
+    kern<<<grid, kThreads, Layout::SMEM_BYTES, s>>>(mq, mk, mv, topk_idx, vbs, plan, out, lse, S, H, nq, topk,
+                                                    tiles_per_bh, n_tiles, scale_log2, err);
     return cudaGetLastError();
 }
 
@@ -1106,17 +512,16 @@ cudaError_t launch_fwd_pair(const uint16_t* q, const uint16_t* k, const uint16_t
                             const int32_t* vbs, const int32_t* plan, uint16_t* out, float* lse, int B, int S, int H,
                             int nq, int topk, float sm_scale, bool precise_p, int* err, cudaStream_t s)
 {
+    if (precise_p)
+        return launch_fwd_pair_shared(q, k, v, topk_idx, vbs, plan, out, lse, B, S, H, nq, topk, sm_scale, true, err, s);
     CUtensorMap mq, mk, mv;
     const int64_t tokens = (int64_t)B * S;
     if (!make_map(&mq, q, tokens, H) || !make_map(&mk, k, tokens, H) || !make_map(&mv, v, tokens, H))
         return cudaErrorInvalidValue;
     const float scale_log2 = sm_scale * 1.4426950408889634f;
-    const bool neg = scale_log2 < 0.f;
-    if (precise_p)
-        return neg ? launch<true, true>(mq, mk, mv, topk_idx, vbs, plan, out, lse, B, S, H, nq, topk, scale_log2, err, s)
-                   : launch<true, false>(mq, mk, mv, topk_idx, vbs, plan, out, lse, B, S, H, nq, topk, scale_log2, err, s);
-    return neg ? launch<false, true>(mq, mk, mv, topk_idx, vbs, plan, out, lse, B, S, H, nq, topk, scale_log2, err, s)
-               : launch<false, false>(mq, mk, mv, topk_idx, vbs, plan, out, lse, B, S, H, nq, topk, scale_log2, err, s);
+    return scale_log2 < 0.f
+               ? launch<true>(mq, mk, mv, topk_idx, vbs, plan, out, lse, B, S, H, nq, topk, scale_log2, err, s)
+               : launch<false>(mq, mk, mv, topk_idx, vbs, plan, out, lse, B, S, H, nq, topk, scale_log2, err, s);
 }
 
 }  // namespace vsa

@@ -1,0 +1,433 @@
+// Device helpers shared by the paired-tile forward kernels (fwd_pair.cu and
+// fwd_pair_precise.cu): step descriptors, bounded mbarrier waits, tcgen05 /
+// TMEM wrappers, packed fp32 pair arithmetic, the tile list generator (the
+// union of two selection lists, shared cubes first) and the TMA tensor maps.
+// Everything lives in an anonymous namespace: each kernel file gets its own
+// copy.
+#pragma once
+
+#include "internal.h"
+#include "sm100_ptx.cuh"
+
+#include <cstddef>
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+namespace vsa {
+namespace {
+
+using namespace ptx;
+
+constexpr int kD = 128;
+constexpr float kTau = 8.0f;
+constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
+
+constexpr uint32_t kHalfBox = 64 * 128;        // 8 KiB: 64 rows x 64 bf16 (one TMA box)
+constexpr uint32_t kTileBytes = 4 * kHalfBox;  // 128 rows x 128 d: Q tile, K pair or V pair (32 KiB)
+
+constexpr int kMaxTopk = 1024;  // per-slot list staging in shared memory
+constexpr int kMaxNq = 8192;    // per-slot membership bitmaps in shared memory
+
+// Per-step description, produced by the producer warp with each K pair.
+struct StepMeta {
+    int32_t ja, jb;   // cube ids of key halves 0 (keys 0-63) and 1 (keys 64-127)
+    int32_t na, nb;   // valid keys of each half (0: nothing loaded)
+    int32_t ma, mb;   // membership: bit 0 = query cube i1 selects it, bit 1 = i2
+    int32_t flags;    // bit 0 first step of the tile, bit 1 last step
+    int32_t vslot;    // V ring slot of this step's V pair (set by the MMA issuer)
+    int32_t vpar;     // its phase parity
+    int32_t pad[3];
+};
+static_assert(sizeof(StepMeta) == 48, "StepMeta layout");
+
+// The fields the other roles need, packed in one 32-bit word in shared memory:
+// na [0,7) nb [7,14) ma [14,16) mb [16,18) flags [18,20) vslot [20] vpar [21].
+__device__ __forceinline__ uint32_t step_word(const StepMeta& s)
+{
+    return (uint32_t)s.na | ((uint32_t)s.nb << 7) | ((uint32_t)s.ma << 14) | ((uint32_t)s.mb << 16) |
+           ((uint32_t)s.flags << 18);
+}
+__device__ __forceinline__ int sw_na(uint32_t w) { return (int)(w & 127u); }
+__device__ __forceinline__ int sw_nb(uint32_t w) { return (int)((w >> 7) & 127u); }
+__device__ __forceinline__ int sw_ma(uint32_t w) { return (int)((w >> 14) & 3u); }
+__device__ __forceinline__ int sw_mb(uint32_t w) { return (int)((w >> 16) & 3u); }
+__device__ __forceinline__ int sw_flags(uint32_t w) { return (int)((w >> 18) & 3u); }
+__device__ __forceinline__ int sw_vslot(uint32_t w) { return (int)((w >> 20) & 1u); }
+__device__ __forceinline__ int sw_vpar(uint32_t w) { return (int)((w >> 21) & 1u); }
+
+
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+__device__ __forceinline__ float min3(float a, float b, float c)
+{
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// tcgen05.mma / commit issued by one elected lane of a converged warp: the
+// operands are warp-uniform values, the predicate picks a single issuer.
+__device__ __forceinline__ void umma_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit_elect(uint64_t* bar)
+{
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+
+// Packed pair arithmetic (one instruction for two fp32 lanes on sm_100).
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0, float c1)
+{
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1)
+{
+    asm("{\n\t.reg .b64 ra, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rd, {%0, %1};\n\t"
+        "add.rn.f32x2 rd, rd, ra;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(a0), "f"(a1));
+}
+
+
+__device__ __forceinline__ bool aborted_flag(int* abort) { return *reinterpret_cast<volatile int*>(abort) != 0; }
+
+// Bounded mbarrier wait that also gives up when another role aborted.  The
+// slow path is a real call: it is reached from many sites, and inlining it
+// everywhere would bloat the instruction footprint of the hot loops.
+__device__ __noinline__ bool wait_bar_slow(uint64_t* bar, uint32_t parity, int* abort, int* err)
+{
+    const long long t0 = clock64();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+        if (aborted_flag(abort)) return false;
+        if (clock64() - t0 > kWaitCycles) {
+            atomicCAS(err, 0, (int)kErrWaitTimeout);
+            *reinterpret_cast<volatile int*>(abort) = 1;
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, int* abort, int* err)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait_bar_slow(bar, parity, abort, err);
+}
+
+// The same wait fully inlined, for the softmax warps: code that runs under a
+// raised setmaxnreg budget makes no calls.
+__device__ __forceinline__ bool wait_bar_inl(uint64_t* bar, uint32_t parity, int* abort, int* err)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+        if (aborted_flag(abort)) return false;
+        if (clock64() - t0 > kWaitCycles) {
+            atomicCAS(err, 0, (int)kErrWaitTimeout);
+            *reinterpret_cast<volatile int*>(abort) = 1;
+            return false;
+        }
+    }
+}
+
+// Warp-uniform bounded wait: true only if every lane saw the phase complete.
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, int* abort, int* err)
+{
+    const bool ok = wait_bar(bar, parity, abort, err);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ bool wait_warp_inl(uint64_t* bar, uint32_t parity, int* abort, int* err)
+{
+    const bool ok = wait_bar_inl(bar, parity, abort, err);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Short bounded wait used while draining after an abort.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity)
+{
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > kWaitCycles / 4) return;
+}
+
+
+// 32x32b TMEM load of 32 consecutive columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r)
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32"
+        " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15,"
+        " %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r)
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32"
+        " [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16,"
+        " %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]), "r"(r[32])
+        : "memory");
+}
+
+__device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
+// The CTA's tiles are t = blockIdx.x + n * gridDim.x; tile n goes to slot n & 1.
+struct TileRef {
+    int b, h, i1, i2;  // i2 = -1: a single query cube (rows 64-127 unused)
+};
+
+__device__ __forceinline__ TileRef tile_ref(int t, int H, int nq, int tiles_per_bh, const int32_t* plan)
+{
+    TileRef r;
+    const int bh = t / tiles_per_bh, p = t - bh * tiles_per_bh;
+    r.b = bh / H;
+    r.h = bh - r.b * H;
+    if (plan != nullptr) {
+        r.i1 = __ldg(plan + 2 * (int64_t)t);
+        r.i2 = __ldg(plan + 2 * (int64_t)t + 1);
+    } else {
+        r.i1 = 2 * p;
+        r.i2 = 2 * p + 1 < nq ? 2 * p + 1 : -1;
+    }
+    return r;
+}
+
+// ------------------------------------------------------------------ step lists
+//
+// The union of a tile's two selection lists, walked in three phases:
+//   0: entries of list 2 whose cube list 1 also names   (both query cubes)
+//   1: entries of list 1 whose cube list 2 does not name (query cube i1 only)
+//   2: entries of list 2 whose cube list 1 does not name (query cube i2 only)
+// A list that names a cube twice disables the sharing (phase 0 is empty and
+// phases 1/2 take every entry), which keeps every multiplicity.  Entries
+// whose cube has no valid token are skipped.  The generator is run by the
+// whole producer warp; `next` keeps a one-entry lookahead so that each step
+// knows whether it is the tile's last.
+struct Entry {
+    int j, n, mem;  // cube, valid tokens, membership bits; mem = 0: none
+};
+
+struct ListGen {
+    int phase, base;
+    uint32_t mask;   // qualifying entries of the 32-entry window at `base`
+    bool dedupe;
+    int len1, len2;  // list lengths (0 if the query cube is absent)
+    Entry next;
+};
+
+__device__ __forceinline__ bool test_bit(const uint32_t* bits, int j) { return (bits[j >> 5] >> (j & 31)) & 1u; }
+
+// Scan forward to the next qualifying entry (warp-uniform result).
+__device__ Entry gen_pull(ListGen& g, const int32_t* l1, const int32_t* l2, const uint32_t* b1, const uint32_t* b2,
+                          const int32_t* __restrict__ vbs, uint32_t lane)
+{
+    Entry e{0, 0, 0};
+    for (;;) {
+        if (g.phase > 2) return e;
+        const int len = g.phase == 1 ? g.len1 : g.len2;
+        const int32_t* list = g.phase == 1 ? l1 : l2;
+        if (g.mask == 0) {
+            if (g.base >= len) {
+                ++g.phase;
+                g.base = 0;
+                continue;
+            }
+            const int idx = g.base + (int)lane;
+            bool q = false;
+            if (idx < len) {
+                const int j = list[idx];
+                const int n = j >= 0 ? __ldg(vbs + j) : 0;
+                if (n > 0 && n <= 64) {
+                    if (g.phase == 0)
+                        q = g.dedupe && test_bit(b1, j);
+                    else if (g.phase == 1)
+                        q = !g.dedupe || !test_bit(b2, j);
+                    else
+                        q = !g.dedupe || !test_bit(b1, j);
+                }
+            }
+            g.mask = __ballot_sync(0xffffffffu, q);
+            g.base += 32;
+            if (g.mask == 0) continue;
+        }
+        const int l = __ffs(g.mask) - 1;
+        g.mask &= g.mask - 1;
+        const int idx = g.base - 32 + l;
+        const int j = list[idx];
+        e.j = j;
+        e.n = __ldg(vbs + j);
+        e.mem = g.phase == 0 ? 3 : (g.phase == 1 ? 1 : 2);
+        return e;
+    }
+}
+
+// Stage a tile's lists and membership bitmaps in shared memory and prime the
+// generator.  Invalid cube ids latch an error and are dropped (stored as -1);
+// invalid vbs values latch an error and count as empty cubes.
+__device__ void gen_start(ListGen& g, const TileRef& t, const int32_t* __restrict__ topk_idx,
+                          const int32_t* __restrict__ vbs, int H, int nq, int topk, int32_t* l1, int32_t* l2,
+                          uint32_t* b1, uint32_t* b2, int* err, uint32_t lane)
+{
+    const int words = (nq + 31) >> 5;
+    for (int w = lane; w < words; w += 32) {
+        b1[w] = 0u;
+        b2[w] = 0u;
+    }
+    g.len1 = t.i1 >= 0 ? topk : 0;
+    g.len2 = t.i2 >= 0 ? topk : 0;
+    __syncwarp();
+    bool dup = false;
+    for (int s = 0; s < 2; ++s) {
+        const int len = s == 0 ? g.len1 : g.len2;
+        if (len == 0) continue;
+        const int i = s == 0 ? t.i1 : t.i2;
+        const int32_t* src = topk_idx + (((int64_t)t.b * H + t.h) * nq + i) * topk;
+        int32_t* dst = s == 0 ? l1 : l2;
+        uint32_t* bits = s == 0 ? b1 : b2;
+        for (int e = lane; e < len; e += 32) {
+            int j = __ldg(src + e);
+            if (j < 0 || j >= nq) {
+                atomicCAS(err, 0, (int)kErrTopkIdx);
+                j = -1;
+            } else {
+                const int n = __ldg(vbs + j);
+                if (n < 0 || n > 64) atomicCAS(err, 0, (int)kErrVbs);
+                const uint32_t old = atomicOr(&bits[j >> 5], 1u << (j & 31));
+                if (old & (1u << (j & 31))) dup = true;
+            }
+            dst[e] = j;
+        }
+    }
+    __syncwarp();
+    g.dedupe = !__any_sync(0xffffffffu, dup) && g.len1 > 0 && g.len2 > 0;
+    g.phase = g.dedupe ? 0 : 1;
+    g.base = 0;
+    g.mask = 0;
+    g.next = gen_pull(g, l1, l2, b1, b2, vbs, lane);
+}
+
+// A tile with an out-of-range plan entry latches an error; the bad cube is dropped.
+__device__ __forceinline__ TileRef checked_tile(int t, int H, int nq, int tiles_per_bh, const int32_t* plan, int* err)
+{
+    TileRef r = tile_ref(t, H, nq, tiles_per_bh, plan);
+    if (r.i1 < 0 || r.i1 >= nq) {
+        if (err != nullptr) atomicCAS(err, 0, (int)kErrPlan);
+        r.i1 = -1;
+    }
+    if (r.i2 < -1 || r.i2 >= nq) {
+        if (err != nullptr) atomicCAS(err, 0, (int)kErrPlan);
+        r.i2 = -1;
+    }
+    return r;
+}
+
+// TMA copy of one 64-token cube (both 64-wide d halves) into rows 64*part of a 128-row tile.
+__device__ __forceinline__ void load_cube(const CUtensorMap* map, uint64_t* bar, uint8_t* dst, int part, int h,
+                                          int tok)
+{
+    tma_load_3d(map, bar, dst + part * kHalfBox, 0, h, tok);
+    tma_load_3d(map, bar, dst + 2 * kHalfBox + part * kHalfBox, 64, h, tok);
+}
+
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// [B*S tokens][H][D] bf16 viewed as a 3-D tensor; box = 64 d x 1 head x 64 tokens.
+bool make_map(CUtensorMap* map, const void* base, int64_t tokens, int H)
+{
+    auto enc = encode_fn();
+    if (enc == nullptr) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)tokens};
+    const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2};
+    const cuuint32_t box[3] = {64, 1, 64};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+
+}  // namespace
+}  // namespace vsa

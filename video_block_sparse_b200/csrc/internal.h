@@ -49,6 +49,10 @@ cudaError_t launch_fwd_tc(const uint16_t* q, const uint16_t* k, const uint16_t* 
 
 // ---- fwd_pair.cu (tcgen05 kernel, two query cubes per 128-row tile)
 bool fwd_pair_supported(int nq, int topk);
+// the variant with one MMA issuer shared by both tiles (fwd_pair_precise.cu); runs the precise mode
+cudaError_t launch_fwd_pair_shared(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* topk_idx,
+                                   const int32_t* vbs, const int32_t* plan, uint16_t* out, float* lse, int B, int S,
+                                   int H, int nq, int topk, float sm_scale, bool precise_p, int* err, cudaStream_t s);
 cudaError_t launch_fwd_pair(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* topk_idx,
                             const int32_t* vbs, const int32_t* plan, uint16_t* out, float* lse, int B, int S, int H,
                             int nq, int topk, float sm_scale, bool precise_p, int* err, cudaStream_t s);
