@@ -58,6 +58,13 @@ namespace {
 using namespace ptx;
 
 constexpr int kThreads = 640;
+
+// Pairs (bit c: columns 2c, 2c+1 of each 32-column chunk) whose exp2 runs on
+// the FMA pipe instead of the multi-function unit.
+#ifndef VSA_POLY_PAIRS
+#define VSA_POLY_PAIRS 0x5252
+#endif
+constexpr uint32_t kPolyPairs = VSA_POLY_PAIRS;
 constexpr int kWarpCorr0 = 8;  // warps 8-11 correct slot 0, 12-15 slot 1
 constexpr int kWarpRole0 = 16; // warp 16 + 2x: producer of slot x, 17 + 2x: MMA issuer of slot x
 
@@ -428,9 +435,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
 #pragma unroll
                         for (int c = 0; c < 16; ++c) {
-                            float x0, x1;
+                            float x0, x1, p0, p1;
                             ffma2(x0, x1, sc[2 * c], sc[2 * c + 1], scale_log2, scale_log2, -mu, -mu);
-                            const float p0 = ex2(x0), p1 = ex2(x1);
+                            if ((kPolyPairs >> c) & 1) {
+                                // weights below 2^-125 (masked keys included) become 2^-125
+                                const float2 pp = ex2_fma2(make_float2(fmaxf(x0, -125.f), fmaxf(x1, -125.f)));
+                                p0 = pp.x;
+                                p1 = pp.y;
+                            } else {
+                                p0 = ex2(x0);
+                                p1 = ex2(x1);
+                            }
                             fadd2(ls0, ls1, p0, p1);
                             pk[c] = pack_bf16(p0, p1);
                         }

@@ -7,6 +7,7 @@
 #pragma once
 
 #include "internal.h"
+#include "exp2_poly.h"
 #include "sm100_ptx.cuh"
 
 #include <cstddef>
@@ -62,6 +63,31 @@ __device__ __forceinline__ float ex2(float x)
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// Adding kRound = 1.5 * 2^23 to a float of magnitude below 2^22 rounds it to
+// an integer n (the sum has unit spacing) and leaves n, in two's complement,
+// in the sum's low mantissa bits; kRound's own low 9 bits are zero.
+constexpr float kRound = 12582912.f;
+
+// 2^x for a pair of exponents x in [-125, 126] on the FMA pipe.  The
+// multi-function unit's exp2 rate (16 per clock per SM) equals the tensor
+// cores' rate at this tile shape, so a share of the exponentials is evaluated
+// here instead:
+//   t = x + kRound = kRound + n,  n = round(x);   f = x - n in [-1/2, 1/2] (exact)
+//   2^f ~ 1 + f (C1 + C2 f + C3 f^2), the fit of exp2_poly.h (relative error
+//   1.0e-4, exact at f = 0), and 2^x = 2^f with n added to its exponent
+//   field: n << 23 is t's bit pattern shifted left by 23.
+__device__ __forceinline__ float2 ex2_fma2(float2 x)
+{
+    const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+    const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
+    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+    float2 p = __ffma2_rn(make_float2(VSA_EXP2_C3, VSA_EXP2_C3), f, make_float2(VSA_EXP2_C2, VSA_EXP2_C2));
+    p = __ffma2_rn(p, f, make_float2(VSA_EXP2_C1, VSA_EXP2_C1));
+    p = __ffma2_rn(p, f, make_float2(1.f, 1.f));
+    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
