@@ -1,6 +1,5 @@
 // VSA fine forward on the Blackwell tensor cores: two query cubes per
-// 128-row tile, queries on TMEM lanes, two tiles in flight per CTA, each tile
-// ("slot") with its own producer, MMA issuer and correction warps.
+// 128-row tile, queries on TMEM lanes, the logits of three steps in flight.
 //
 // Dataset card "wan2.2_production_values", section "Operator contract": for
 // query cube i of (batch b, head h) the keys are the first vbs[j] tokens of
@@ -18,38 +17,43 @@
 // cube's rows.  Cubes both lists name are walked first and loaded once for
 // both; vsa_plan pairs query cubes whose lists overlap most.
 //
-// Each softmax thread owns one query row (one TMEM lane): row maximum and row
-// sum are thread-local.  Two tiles are in flight per CTA.  A slot's chain is
-// strictly serial (QK -> softmax -> PV -> next QK, S/P reuse), so the slots
-// are made fully independent: each has its own Q, K and V buffers, its own
-// producer warp, MMA-issuing warp and correction warps, and the tensor core
-// takes whichever slot's products are ready.  No warp ever waits on the other
-// slot's progress.
+// Pipeline.  TMEM holds three S/P buffers (columns 0, 128, 256) and O
+// (columns 384-511).  Step g uses buffer g % 3, and the MMA issuer runs the
+// products in the order  ..., PV(g), QK(g + 3), PV(g + 1), QK(g + 4), ...
+// so the logits of the next two steps are ready while the softmax of step g
+// runs; the softmax, not the QK -> softmax -> PV chain, sets the pace, and the
+// tensor core sees one PV and one QK per softmax step.  Steps run on across
+// tile boundaries; the tile's offsets and sums restart at its first step.
 //
-// Roles (640 threads, one persistent CTA per SM):
-//   warps 0-3 / 4-7    softmax + epilogue of slot 0 / 1 (thread = row = lane)
-//   warps 8-11 / 12-15 O correction of slot 0 / 1: rescale the rows whose
-//                      running offset rose (thread = row)
-//   warp 16 / 18       TMA producer of slot 0 / 1: builds each tile's step list
-//                      (shared cubes first) and streams its Q, K and V tiles
-//   warp 17 / 19       MMA issuer of slot 0 / 1 (the whole warp runs the
-//                      schedule, one elected lane issues); zeroes V pad rows
-//                      inside a partial k-step before the product.  Warp 17
-//                      also owns the TMEM allocation.
+// Roles (448 threads, one persistent CTA per SM):
+//   warps 0-7   softmax: warp w owns TMEM lanes 32 (w % 4) .. +31 (query rows)
+//               and key half w / 4 (columns 0-63: the step's first KV cube,
+//               64-127: the second).  The two warps of a lane quarter share
+//               each row's step maximum through shared memory, so both halves
+//               use the same offset; each keeps the sum of its own half.
+//   warps 8-11  O correction and epilogue (thread = row): rescale the rows
+//               whose running offset rose, once the previous PV has finished;
+//               at a tile's end, O / l -> out and the log-sum-exp -> lse
+//   warp 12     TMA producer: builds each tile's step list (shared cubes
+//               first) and streams Q (one buffer), K pairs (ring of 2) and
+//               V pairs (ring of 3)
+//   warp 13     MMA issuer (the whole warp runs the schedule, one elected lane
+//               issues); zeroes V pad rows inside a partial k-step before the
+//               product; owns the TMEM allocation.
 //
 // Softmax.  Logits in base 2 (x = s * sm_scale * log2 e).  Keys at or beyond
 // vbs of their cube and cubes the row's query cube did not select are
 // replaced by -inf (a select: NaN/Inf there never propagates).  The running
 // offset of a row is raised only when the step maximum exceeds it by more
-// than kTau (so P <= 2^kTau); only then are the row of O and the row sum
+// than kTau (so P <= 2^kTau); only then are the row of O and the row sums
 // rescaled.  PV k-steps (16 keys) beyond ceil16(vbs) of a cube are not issued;
 // V rows between vbs and that boundary are zeroed before the product, so
 // 0 * NaN cannot occur.
 //
 // Every mbarrier wait is bounded (~2 s of clock): on expiry the kernel
 // latches kErrWaitTimeout and raises a CTA-wide abort flag; every role leaves
-// its loop, producers and MMA issuers wait (bounded) for their own copies and
-// products in flight, and TMEM is freed before exit.
+// its loop, the producer and the MMA issuer wait (bounded) for their own
+// copies and products in flight, and TMEM is freed before exit.
 #include "fwd_pair_common.cuh"
 
 namespace vsa {
@@ -57,7 +61,17 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kThreads = 640;
+constexpr int kSoftWarps = 12;  // warps 0-11: softmax, three per SMSP
+constexpr int kWarpCorr0 = 12;  // warps 12-15: correction and epilogue
+constexpr int kWarpProd = 16;
+constexpr int kWarpMma = 17;
+constexpr int kWarpVProd = 18;
+constexpr int kThreads = 19 * 32;
+constexpr int kVReq = 4;  // ring of V load requests from the K producer to the V producer
+constexpr int kSBuf = 3;  // S/P buffers in TMEM (also the V ring depth)
+constexpr int kKBuf = 2;  // K ring depth
+constexpr uint32_t kOCol = 384;
+constexpr uint32_t kFinal = 1u << 22;  // step word: last step of the CTA's last tile
 
 // Pairs (bit c: columns 2c, 2c+1 of each 32-column chunk) whose exp2 runs on
 // the FMA pipe instead of the multi-function unit.
@@ -65,47 +79,61 @@ constexpr int kThreads = 640;
 #define VSA_POLY_PAIRS 0x5252
 #endif
 constexpr uint32_t kPolyPairs = VSA_POLY_PAIRS;
-constexpr int kWarpCorr0 = 8;  // warps 8-11 correct slot 0, 12-15 slot 1
-constexpr int kWarpRole0 = 16; // warp 16 + 2x: producer of slot x, 17 + 2x: MMA issuer of slot x
 
-struct SlotBars {
-    uint64_t q_full, q_empty;  // Q tile landed / last QK of the tile done
-    uint64_t k_full, k_empty;  // K pair landed / QK done
-    uint64_t v_full, v_empty;  // V pair landed / PV done
-    uint64_t s_full;           // step word published + QK done (2 arrivals)
-    uint64_t a_full;           // offsets decided (128 softmax threads)
-    uint64_t p_full;           // P written and O corrected (128 softmax + 128 correction threads)
-    uint64_t o_full;           // last PV of a tile done
+struct Bars {
+    uint64_t q_full, q_empty;                // Q tile landed / last QK of the tile done
+    uint64_t k_full[kKBuf], k_empty[kKBuf];  // K pair landed / its QK done
+    uint64_t v_full[kSBuf], v_empty[kSBuf];  // V pair landed / its PV done
+    uint64_t s_full[kSBuf];  // step word published + QK done (2 arrivals)
+    uint64_t a_full[kSBuf];  // offsets decided (the 128 threads of the step's softmax warps)
+    uint64_t p_full[kSBuf];  // P written (128 softmax threads) and O corrected (128)
+    uint64_t pv_done[2];     // PV of step j done: pv_done[j & 1]
+    uint64_t o_full;         // last PV of a tile done
+    uint64_t l_full[2];      // tile parity: row sums and offsets written (128)
+    uint64_t l_empty[2];     // tile parity: the epilogue has read them (128)
+    uint64_t dec[kSBuf][4];   // [step % 3][lane quarter]: offsets after the step decided (32)
+    uint64_t lsum[kSBuf][4];  // [step % 3][lane quarter]: row sums after the step written (32)
+    uint64_t vr_full[kVReq], vr_empty[kVReq];  // V load request posted / taken
     uint64_t drain;
 };
 
 struct Misc {
-    SlotBars bar[2];
-    uint32_t k_meta[2];  // step word of the K pair in each slot's K buffer
-    uint32_t s_meta[2];  // step word of the S in each slot
+    Bars bar;
+    int4 vreq[kVReq];        // V load request: first token of cube a (-1: none), of cube b, head, last
+    uint32_t k_meta[kKBuf];  // step word of the K pair in each K buffer
+    uint32_t s_meta[kSBuf];  // step word of each S buffer
     uint32_t tmem_base;
     int abort;
-    alignas(16) float alpha[2][128];  // per slot, row: O rescale factor of the current step
-    int rflag[2][4];                  // per slot, warp: some row of the warp rescales
-    uint32_t bits1[2][kMaxNq / 32];   // per slot: membership bitmap of list 1
-    uint32_t bits2[2][kMaxNq / 32];   //                           and of list 2
-    int32_t list1[2][kMaxTopk];       // per slot: the two selection lists
-    int32_t list2[2][kMaxTopk];
+    alignas(16) float alpha[kSBuf][128];  // per S buffer, row: O rescale factor of that step
+    int rflag[kSBuf][4];                  // per S buffer, lane quarter: some row rescales
+    float m_state[2][128];                // [step parity][row]: offset after the step's decision
+    float l_state[2][128];                // [step parity][row]: row sum after the step
+    int n_state[2][4];                    // [step parity][lane quarter]: tiles finished after the step
+    float lfin[2][128];                   // [tile parity][row]: row sum at the tile's end
+    float mfin[2][128];                   // [tile parity][row]: running offset at the tile's end
+    uint32_t bits1[kMaxNq / 32];          // membership bitmaps of the tile's two lists
+    uint32_t bits2[kMaxNq / 32];
+    int32_t list1[kMaxTopk];              // the tile's two selection lists
+    int32_t list2[kMaxTopk];
 };
 
 struct Layout {
-    static constexpr uint32_t Q_OFF = 0;                       // Q tile of slot x at Q_OFF + x * 32 KiB
-    static constexpr uint32_t K_OFF = Q_OFF + 2 * kTileBytes;  // K pair of slot x
-    static constexpr uint32_t V_OFF = K_OFF + 2 * kTileBytes;  // V pair of slot x
-    static constexpr uint32_t TILE_BYTES = V_OFF + 2 * kTileBytes;
+    static constexpr uint32_t Q_OFF = 0;                           // Q tile
+    static constexpr uint32_t K_OFF = Q_OFF + kTileBytes;          // K ring
+    static constexpr uint32_t V_OFF = K_OFF + kKBuf * kTileBytes;  // V ring
+    static constexpr uint32_t TILE_BYTES = V_OFF + kSBuf * kTileBytes;
     static constexpr uint32_t MISC_BYTES = (sizeof(Misc) + 1023) / 1024 * 1024;
     static constexpr uint32_t SMEM_BYTES = MISC_BYTES + TILE_BYTES + 1024;  // + alignment slack
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-// TMEM columns of slot x: S/P at 256x, O at 256x + 128.
-__device__ __forceinline__ uint32_t s_col(int x) { return 256u * x; }
-__device__ __forceinline__ uint32_t o_col(int x) { return 256u * x + 128u; }
+// Non-blocking check of a phase by lane 0, made warp-uniform.
+__device__ __forceinline__ bool probe_warp(uint64_t* bar, uint32_t parity)
+{
+    uint32_t ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_test_wait(bar, parity) ? 1u : 0u;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
 
 template <bool NEG>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -118,6 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     using L = Layout;
     extern __shared__ uint8_t smem_raw[];
     Misc& m = *reinterpret_cast<Misc*>(smem_raw);
+    Bars& bb = m.bar;
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t tiles = (raw_addr + L::MISC_BYTES + 1023u) & ~1023u;  // 1 KiB aligned for 128B swizzle
     uint8_t* tiles_ptr = smem_raw + (tiles - raw_addr);
@@ -128,28 +157,43 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ------------------------------------------------------------ set-up
     if (threadIdx.x == 0) {
-        for (int x = 0; x < 2; ++x) {
-            SlotBars& sb = m.bar[x];
-            mbar_init(&sb.q_full, 1);
-            mbar_init(&sb.q_empty, 1);
-            mbar_init(&sb.k_full, 1);
-            mbar_init(&sb.k_empty, 1);
-            mbar_init(&sb.v_full, 1);
-            mbar_init(&sb.v_empty, 1);
-            mbar_init(&sb.s_full, 2);    // MMA warp (step word) + QK completion
-            mbar_init(&sb.a_full, 128);  // every softmax thread of the slot
-            mbar_init(&sb.p_full, 256);  // every softmax and every correction thread of the slot
-            mbar_init(&sb.o_full, 1);
-            mbar_init(&sb.drain, 1);
+        mbar_init(&bb.q_full, 1);
+        mbar_init(&bb.q_empty, 1);
+        for (int i = 0; i < kKBuf; ++i) {
+            mbar_init(&bb.k_full[i], 1);
+            mbar_init(&bb.k_empty[i], 1);
         }
+        for (int i = 0; i < kSBuf; ++i) {
+            mbar_init(&bb.v_full[i], 1);
+            mbar_init(&bb.v_empty[i], 1);
+            mbar_init(&bb.s_full[i], 2);    // MMA warp (step word) + QK completion
+            mbar_init(&bb.a_full[i], 128);  // the four softmax warps of the step
+            mbar_init(&bb.p_full[i], 256);  // those and every correction thread
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bb.pv_done[i], 1);
+            mbar_init(&bb.l_full[i], 128);
+            mbar_init(&bb.l_empty[i], 128);
+        }
+        for (int i = 0; i < kVReq; ++i) {
+            mbar_init(&bb.vr_full[i], 1);
+            mbar_init(&bb.vr_empty[i], 1);
+        }
+        for (int i = 0; i < kSBuf; ++i)
+            for (int j = 0; j < 4; ++j) {
+                mbar_init(&bb.dec[i][j], 32);
+                mbar_init(&bb.lsum[i][j], 32);
+            }
+        mbar_init(&bb.o_full, 1);
+        mbar_init(&bb.drain, 1);
         m.abort = 0;
         fence_mbar_init();
     }
-    if (warp == kWarpRole0 + 1) {
+    if (warp == kWarpMma) {
         tmem_alloc(&m.tmem_base, 512);
         tmem_relinquish();
     }
-    if (warp == kWarpRole0 && lane == 0) {
+    if (warp == kWarpProd && lane == 0) {
         prefetch_tmap(&tmq);
         prefetch_tmap(&tmk);
         prefetch_tmap(&tmv);
@@ -159,181 +203,219 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tbase = m.tmem_base;
 
-    if (warp >= kWarpRole0) {
-        const int x = (warp - kWarpRole0) >> 1;
-        SlotBars& sb = m.bar[x];
-        uint8_t* qdst = tiles_ptr + L::Q_OFF + x * kTileBytes;
-        uint8_t* kdst = tiles_ptr + L::K_OFF + x * kTileBytes;
-        uint8_t* vdst = tiles_ptr + L::V_OFF + x * kTileBytes;
-        if (((warp - kWarpRole0) & 1) == 0) {
-            // ---------------------------------------------------- TMA producer of slot x
-            ListGen gen;
-            int qn = 0, kc = 0;
-            int armed_q = -1, armed_k = -1, armed_v = -1;
-            bool aborted = false;
-            for (int n = x; n < my_tiles && !aborted; n += 2) {
-                const TileRef t =
-                    checked_tile(blockIdx.x + n * gridDim.x, H, nq, tiles_per_bh, plan, lane == 0 ? err : nullptr);
-                gen_start(gen, t, topk_idx, vbs, H, nq, topk, m.list1[x], m.list2[x], m.bits1[x], m.bits2[x], err,
-                          lane);
-                const int tok0 = t.b * S;
+    if (warp == kWarpProd) {
+        // ------------------------------------------------------------ TMA producer of Q and K
+        // (it posts each step's V pair to the V producer, so that K loads never wait
+        // behind a V buffer)
+        ListGen gen;
+        int kc = 0;
+        int armed_q = -1, armed_k = -1, armed_kb = 0;
+        bool aborted = false;
+        uint8_t* qdst = tiles_ptr + L::Q_OFF;
+        for (int n = 0; n < my_tiles && !aborted; ++n) {
+            const TileRef t =
+                checked_tile(blockIdx.x + n * gridDim.x, H, nq, tiles_per_bh, plan, lane == 0 ? err : nullptr);
+            gen_start(gen, t, topk_idx, vbs, H, nq, topk, m.list1, m.list2, m.bits1, m.bits2, err, lane);
+            const int tok0 = t.b * S;
+            if (lane == 0) {
+                if (wait_bar(&bb.q_empty, (n & 1) ^ 1, &m.abort, err)) {
+                    mbar_expect_tx(&bb.q_full, 2 * kHalfBox * ((t.i1 >= 0) + (t.i2 >= 0)));
+                    armed_q = n & 1;
+                    if (t.i1 >= 0) load_cube(&tmq, &bb.q_full, qdst, 0, t.h, tok0 + 64 * t.i1);
+                    if (t.i2 >= 0) load_cube(&tmq, &bb.q_full, qdst, 1, t.h, tok0 + 64 * t.i2);
+                } else {
+                    aborted = true;
+                }
+            }
+            aborted = __shfl_sync(0xffffffffu, aborted, 0);
+            bool first = true;
+            while (!aborted) {
+                const Entry ea = gen.next;
+                Entry eb{0, 0, 0};
+                if (ea.mem != 0) {
+                    gen.next = gen_pull(gen, m.list1, m.list2, m.bits1, m.bits2, vbs, lane);
+                    eb = gen.next;
+                    if (eb.mem != 0) gen.next = gen_pull(gen, m.list1, m.list2, m.bits1, m.bits2, vbs, lane);
+                }
+                const bool last = gen.next.mem == 0;
+                StepMeta meta;
+                meta.ja = ea.j;
+                meta.jb = eb.j;
+                meta.na = ea.n;
+                meta.nb = eb.n;
+                meta.ma = ea.mem;
+                meta.mb = eb.mem;
+                meta.flags = (first ? 1 : 0) | (last ? 2 : 0);
+                first = false;
+                const uint32_t word = step_word(meta) | (last && n == my_tiles - 1 ? kFinal : 0u);
+                const uint32_t bytes = 2 * kHalfBox * ((meta.na > 0) + (meta.nb > 0));
+                const int kb = kc % kKBuf, vr = kc % kVReq;
                 if (lane == 0) {
-                    if (wait_bar(&sb.q_empty, (qn & 1) ^ 1, &m.abort, err)) {
-                        mbar_expect_tx(&sb.q_full, 2 * kHalfBox * ((t.i1 >= 0) + (t.i2 >= 0)));
-                        armed_q = qn & 1;
-                        if (t.i1 >= 0) load_cube(&tmq, &sb.q_full, qdst, 0, t.h, tok0 + 64 * t.i1);
-                        if (t.i2 >= 0) load_cube(&tmq, &sb.q_full, qdst, 1, t.h, tok0 + 64 * t.i2);
+                    // K pair of the step: its buffer is free once the QK two steps back finished
+                    if (wait_bar(&bb.k_empty[kb], ((kc / kKBuf) & 1) ^ 1, &m.abort, err)) {
+                        m.k_meta[kb] = word;
+                        mbar_expect_tx(&bb.k_full[kb], bytes);
+                        armed_k = (kc / kKBuf) & 1;
+                        armed_kb = kb;
+                        uint8_t* kdst = tiles_ptr + L::K_OFF + kb * kTileBytes;
+                        if (meta.na > 0) load_cube(&tmk, &bb.k_full[kb], kdst, 0, t.h, tok0 + 64 * meta.ja);
+                        if (meta.nb > 0) load_cube(&tmk, &bb.k_full[kb], kdst, 1, t.h, tok0 + 64 * meta.jb);
+                    } else {
+                        aborted = true;
+                    }
+                    // the step's V pair, for the V producer
+                    if (!aborted && wait_bar(&bb.vr_empty[vr], ((kc / kVReq) & 1) ^ 1, &m.abort, err)) {
+                        m.vreq[vr] = make_int4(meta.na > 0 ? tok0 + 64 * meta.ja : -1,
+                                               meta.nb > 0 ? tok0 + 64 * meta.jb : -1, t.h,
+                                               (word & kFinal) ? 1 : 0);
+                        mbar_arrive(&bb.vr_full[vr]);
                     } else {
                         aborted = true;
                     }
                 }
                 aborted = __shfl_sync(0xffffffffu, aborted, 0);
-                ++qn;
-                bool first = true;
-                while (!aborted) {
-                    const Entry ea = gen.next;
-                    Entry eb{0, 0, 0};
-                    if (ea.mem != 0) {
-                        gen.next = gen_pull(gen, m.list1[x], m.list2[x], m.bits1[x], m.bits2[x], vbs, lane);
-                        eb = gen.next;
-                        if (eb.mem != 0) gen.next = gen_pull(gen, m.list1[x], m.list2[x], m.bits1[x], m.bits2[x], vbs, lane);
-                    }
-                    const bool last = gen.next.mem == 0;
-                    StepMeta meta;
-                    meta.ja = ea.j;
-                    meta.jb = eb.j;
-                    meta.na = ea.n;
-                    meta.nb = eb.n;
-                    meta.ma = ea.mem;
-                    meta.mb = eb.mem;
-                    meta.flags = (first ? 1 : 0) | (last ? 2 : 0);
-                    first = false;
-                    const uint32_t bytes = 2 * kHalfBox * ((meta.na > 0) + (meta.nb > 0));
-                    if (lane == 0) {
-                        // K pair of the step: the buffer is free once the previous QK finished
-                        if (wait_bar(&sb.k_empty, (kc & 1) ^ 1, &m.abort, err)) {
-                            m.k_meta[x] = step_word(meta);
-                            mbar_expect_tx(&sb.k_full, bytes);
-                            armed_k = kc & 1;
-                            if (meta.na > 0) load_cube(&tmk, &sb.k_full, kdst, 0, t.h, tok0 + 64 * meta.ja);
-                            if (meta.nb > 0) load_cube(&tmk, &sb.k_full, kdst, 1, t.h, tok0 + 64 * meta.jb);
-                        } else {
-                            aborted = true;
-                        }
-                        // V pair of the step: free once the previous PV finished
-                        if (!aborted && wait_bar(&sb.v_empty, (kc & 1) ^ 1, &m.abort, err)) {
-                            mbar_expect_tx(&sb.v_full, bytes);
-                            armed_v = kc & 1;
-                            if (meta.na > 0) load_cube(&tmv, &sb.v_full, vdst, 0, t.h, tok0 + 64 * meta.ja);
-                            if (meta.nb > 0) load_cube(&tmv, &sb.v_full, vdst, 1, t.h, tok0 + 64 * meta.jb);
-                        } else {
-                            aborted = true;
-                        }
-                    }
-                    aborted = __shfl_sync(0xffffffffu, aborted, 0);
-                    ++kc;
-                    if (last) break;
-                }
-            }
-            if (aborted && lane == 0) {
-                // copies issued by this thread must land before the CTA's shared memory goes away
-                if (armed_q >= 0) drain_wait(&sb.q_full, armed_q);
-                if (armed_k >= 0) drain_wait(&sb.k_full, armed_k);
-                if (armed_v >= 0) drain_wait(&sb.v_full, armed_v);
-            }
-        } else {
-            // ---------------------------------------------------- MMA issuer of slot x
-            constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);
-            // operand descriptors built once; a k-step adds its byte offset / 16
-            const uint64_t d_hi = smem_desc_sw128(0, 0, 1024);
-            const uint32_t ql = (uint32_t)smem_desc_sw128(smem_u32(qdst), 16, 1024);
-            const uint32_t kl = (uint32_t)smem_desc_sw128(smem_u32(kdst), 16, 1024);
-            const uint32_t vl = (uint32_t)smem_desc_sw128(smem_u32(vdst), 2 * kHalfBox, 1024);
-            const uint32_t s_tmem = tbase + s_col(x), o_tmem = tbase + o_col(x);
-            int qn = 0, kc = 0;
-            bool aborted = false;
-            for (int n = x; n < my_tiles && !aborted; n += 2) {
-                if (!wait_warp(&sb.q_full, qn & 1, &m.abort, err)) { aborted = true; break; }
-                ++qn;
-                bool o_init = false;
-                for (;;) {
-                    // ---- S = Q . K^T
-                    if (!wait_warp(&sb.k_full, kc & 1, &m.abort, err)) { aborted = true; break; }
-                    const uint32_t meta = m.k_meta[x];
-                    __syncwarp();
-                    if (lane == 0) {
-                        m.s_meta[x] = meta;
-                        mbar_arrive(&sb.s_full);  // publishes the step word (release)
-                    }
-                    __syncwarp();
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t off = ((kk >> 2) * (2 * kHalfBox) + (kk & 3) * 32u) >> 4;
-                        umma_ss_elect(s_tmem, d_hi | (ql + off), d_hi | (kl + off), idesc_qk, kk > 0 ? 1u : 0u);
-                    }
-                    umma_commit_elect(&sb.s_full);
-                    umma_commit_elect(&sb.k_empty);
-                    const bool last = (sw_flags(meta) & 2) != 0;
-                    if (last) umma_commit_elect(&sb.q_empty);
-                    // ---- O += P . V
-                    if (!wait_warp(&sb.p_full, kc & 1, &m.abort, err)) { aborted = true; break; }
-                    if (!wait_warp(&sb.v_full, kc & 1, &m.abort, err)) { aborted = true; break; }
-                    const int na = sw_na(meta), nb = sw_nb(meta);
-                    const int za = (na & 15) ? 16 - (na & 15) : 0, zb = (nb & 15) ? 16 - (nb & 15) : 0;
-                    if (za + zb > 0) {
-                        // V rows between vbs and the next multiple of 16 are read by the last
-                        // k-step of their cube: zero them (both d halves) before the product
-                        const uint32_t vb = smem_u32(vdst);
-                        for (int w = lane; w < (za + zb) * 16; w += 32) {
-                            const int zr = w >> 4, chunk = w & 15;
-                            const int row = zr < za ? na + zr : 64 + nb + (zr - za);
-                            sts128(vb + (chunk >> 3) * (2 * kHalfBox) + row * 128 + (chunk & 7) * 16, 0u, 0u, 0u, 0u);
-                        }
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                    }
-                    tc_fence_after();
-                    // k-steps (16 keys) 0..ceil16(na)-1 of half 0 and 4..4+ceil16(nb)-1 of half 1
-                    const uint32_t kmask = ((1u << ((na + 15) >> 4)) - 1u) | (((1u << ((nb + 15) >> 4)) - 1u) << 4);
-                    uint32_t acc = o_init ? 1u : 0u;
-#pragma unroll
-                    for (int kstep = 0; kstep < 8; ++kstep) {
-                        if (kmask & (1u << kstep)) {
-                            umma_ts_elect(o_tmem, s_tmem + kstep * 8, d_hi | (vl + ((kstep * 2048) >> 4)), idesc_pv, acc);
-                            acc = 1u;
-                        }
-                    }
-                    o_init = o_init || kmask != 0;
-                    umma_commit_elect(&sb.v_empty);
-                    if (last) umma_commit_elect(&sb.o_full);
-                    ++kc;
-                    if (last) break;
-                }
-            }
-            if (aborted) {
-                umma_commit_elect(&sb.drain);
-                if (lane == 0) drain_wait(&sb.drain, 0);
-                __syncwarp();
+                ++kc;
+                if (last) break;
             }
         }
-    } else if (warp >= kWarpCorr0) {
-        // -------------------------------------------------------- O correction of slot x
-        const int x = (warp - kWarpCorr0) >> 2, wq = warp & 3;
-        const int r = 32 * wq + (int)lane;
-        SlotBars& sb = m.bar[x];
-        const uint32_t oa = tbase + ((uint32_t)(32 * wq) << 16) + o_col(x);
-        int g = 0;
-        for (int n = x; n < my_tiles; n += 2) {
-            for (;;) {
-                if (!wait_warp(&sb.a_full, g & 1, &m.abort, err)) goto corr_exit;
-                const uint32_t meta = m.s_meta[x];
+        if (aborted && lane == 0) {
+            // copies issued by this thread must land before the CTA's shared memory goes away
+            if (armed_q >= 0) drain_wait(&bb.q_full, armed_q);
+            if (armed_k >= 0) drain_wait(&bb.k_full[armed_kb], armed_k);
+        }
+    } else if (warp == kWarpVProd) {
+        // ------------------------------------------------------------ TMA producer of V
+        int armed_v = -1, armed_vb = 0;
+        for (int vc = 0; my_tiles > 0 && lane == 0; ++vc) {
+            const int vr = vc % kVReq, vb = vc % kSBuf;
+            if (!wait_bar(&bb.vr_full[vr], (vc / kVReq) & 1, &m.abort, err)) break;
+            const int4 rq = m.vreq[vr];
+            mbar_arrive(&bb.vr_empty[vr]);
+            // the V buffer is free once the PV three steps back finished
+            if (!wait_bar(&bb.v_empty[vb], ((vc / kSBuf) & 1) ^ 1, &m.abort, err)) break;
+            mbar_expect_tx(&bb.v_full[vb], 2 * kHalfBox * ((rq.x >= 0) + (rq.y >= 0)));
+            armed_v = (vc / kSBuf) & 1;
+            armed_vb = vb;
+            uint8_t* vdst = tiles_ptr + L::V_OFF + vb * kTileBytes;
+            if (rq.x >= 0) load_cube(&tmv, &bb.v_full[vb], vdst, 0, rq.z, rq.x);
+            if (rq.y >= 0) load_cube(&tmv, &bb.v_full[vb], vdst, 1, rq.z, rq.y);
+            if (rq.w) break;  // the CTA's last step
+        }
+        if (lane == 0 && armed_v >= 0 && aborted_flag(&m.abort)) drain_wait(&bb.v_full[armed_vb], armed_v);
+        __syncwarp();
+    } else if (warp == kWarpMma) {
+        // ------------------------------------------------------------ MMA issuer
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);
+        // operand descriptors built once; a k-step adds its byte offset / 16
+        const uint64_t d_hi = smem_desc_sw128(0, 0, 1024);
+        const uint32_t ql = (uint32_t)smem_desc_sw128(tiles + L::Q_OFF, 16, 1024);
+        const uint32_t kl0 = (uint32_t)smem_desc_sw128(tiles + L::K_OFF, 16, 1024);
+        const uint32_t vl0 = (uint32_t)smem_desc_sw128(tiles + L::V_OFF, 2 * kHalfBox, 1024);
+        const uint32_t o_tmem = tbase + kOCol;
+        int j_qk = 0, j_pv = 0, qn = 0;
+        bool qk_done = my_tiles == 0, o_init = false, aborted = false;
+        for (;;) {
+            // ---- QK of the steps up to two ahead of the next PV (S buffers are free)
+            while (!qk_done && j_qk < j_pv + kSBuf) {
+                const int kb = j_qk % kKBuf;
+                const uint32_t kpar = (j_qk / kKBuf) & 1;
+                // with a PV pending, a QK whose operands are not there yet waits for later
+                if (j_pv < j_qk && !probe_warp(&bb.k_full[kb], kpar)) break;
+                if (!wait_warp(&bb.k_full[kb], kpar, &m.abort, err)) { aborted = true; break; }
+                const uint32_t meta = m.k_meta[kb];
+                if (sw_flags(meta) & 1) {
+                    if (j_pv < j_qk && !probe_warp(&bb.q_full, qn & 1)) break;
+                    if (!wait_warp(&bb.q_full, qn & 1, &m.abort, err)) { aborted = true; break; }
+                    ++qn;
+                }
+                const int sb = j_qk % kSBuf;
+                __syncwarp();
+                if (lane == 0) {
+                    m.s_meta[sb] = meta;
+                    mbar_arrive(&bb.s_full[sb]);  // publishes the step word (release)
+                }
+                __syncwarp();
                 tc_fence_after();
-                if (!(sw_flags(meta) & 1) && m.rflag[x][wq] != 0) {
-                    // O row r *= alpha (1 for rows whose offset stayed); the previous
-                    // P.V of the slot finished before this step's S was published
-                    const float a = m.alpha[x][r];
+                const uint32_t kl = kl0 + ((uint32_t)kb * kTileBytes >> 4);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = ((kk >> 2) * (2 * kHalfBox) + (kk & 3) * 32u) >> 4;
+                    umma_ss_elect(tbase + 128u * sb, d_hi | (ql + off), d_hi | (kl + off), idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                umma_commit_elect(&bb.s_full[sb]);
+                umma_commit_elect(&bb.k_empty[kb]);
+                if (sw_flags(meta) & 2) umma_commit_elect(&bb.q_empty);
+                if (meta & kFinal) qk_done = true;
+                ++j_qk;
+            }
+            if (aborted || j_pv == j_qk) break;  // aborted, or every step done
+            // ---- O += P . V for step j_pv
+            const int sb = j_pv % kSBuf;
+            const uint32_t par = (j_pv / kSBuf) & 1;
+            if (!wait_warp(&bb.p_full[sb], par, &m.abort, err)) { aborted = true; break; }
+            if (!wait_warp(&bb.v_full[sb], par, &m.abort, err)) { aborted = true; break; }
+            const uint32_t meta = m.s_meta[sb];
+            const int na = sw_na(meta), nb = sw_nb(meta);
+            const uint32_t vl = vl0 + ((uint32_t)sb * kTileBytes >> 4);
+            const int za = (na & 15) ? 16 - (na & 15) : 0, zb = (nb & 15) ? 16 - (nb & 15) : 0;
+            if (za + zb > 0) {
+                // V rows between vbs and the next multiple of 16 are read by the last
+                // k-step of their cube: zero them (both d halves) before the product
+                const uint32_t vbase = tiles + L::V_OFF + sb * kTileBytes;
+                for (int w = lane; w < (za + zb) * 16; w += 32) {
+                    const int zr = w >> 4, chunk = w & 15;
+                    const int row = zr < za ? na + zr : 64 + nb + (zr - za);
+                    sts128(vbase + (chunk >> 3) * (2 * kHalfBox) + row * 128 + (chunk & 7) * 16, 0u, 0u, 0u, 0u);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
+            tc_fence_after();
+            // k-steps (16 keys) 0..ceil16(na)-1 of half 0 and 4..4+ceil16(nb)-1 of half 1; the
+            // bf16 P of key half h sits in the first 32 columns of that half's 64
+            const uint32_t kmask = ((1u << ((na + 15) >> 4)) - 1u) | (((1u << ((nb + 15) >> 4)) - 1u) << 4);
+            const uint32_t p_tmem = tbase + 128u * sb;
+            if (sw_flags(meta) & 1) o_init = false;
+            uint32_t acc = o_init ? 1u : 0u;
+#pragma unroll
+            for (int kstep = 0; kstep < 8; ++kstep) {
+                if (kmask & (1u << kstep)) {
+                    const uint32_t a_col = kstep < 4 ? 8u * kstep : 64u + 8u * (kstep - 4);
+                    umma_ts_elect(o_tmem, p_tmem + a_col, d_hi | (vl + ((kstep * 2048) >> 4)), idesc_pv, acc);
+                    acc = 1u;
+                }
+            }
+            o_init = o_init || kmask != 0;
+            umma_commit_elect(&bb.v_empty[sb]);
+            umma_commit_elect(&bb.pv_done[j_pv & 1]);
+            if (sw_flags(meta) & 2) umma_commit_elect(&bb.o_full);
+            ++j_pv;
+        }
+        if (aborted) {
+            umma_commit_elect(&bb.drain);
+            if (lane == 0) drain_wait(&bb.drain, 0);
+            __syncwarp();
+        }
+    } else if (warp >= kWarpCorr0) {
+        // ------------------------------------------------------------ O correction and epilogue
+        const int wq = warp & 3;
+        const int r = 32 * wq + (int)lane;
+        const int qbit = r >> 6;
+        const uint32_t oa = tbase + ((uint32_t)(32 * wq) << 16) + kOCol;
+        int g = 0;
+        for (int n = 0; n < my_tiles; ++n) {
+            for (;;) {
+                const int b = g % kSBuf;
+                if (!wait_warp(&bb.a_full[b], (g / kSBuf) & 1, &m.abort, err)) goto corr_exit;
+                const uint32_t meta = m.s_meta[b];
+                if (!(sw_flags(meta) & 1) && m.rflag[b][wq] != 0) {
+                    // O row r *= alpha (1 for rows whose offset stayed), once the
+                    // previous step's PV has finished
+                    const int jp = g - 1;
+                    if (!wait_warp(&bb.pv_done[jp & 1], (jp >> 1) & 1, &m.abort, err)) goto corr_exit;
+                    tc_fence_after();
+                    const float a = m.alpha[b][r];
 #pragma unroll 1
                     for (int c4 = 0; c4 < 4; ++c4) {
                         uint32_t o[32];
@@ -346,132 +428,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_st_wait();
                 }
                 tc_fence_before();
-                mbar_arrive(&sb.p_full);
+                mbar_arrive(&bb.p_full[b]);
                 ++g;
                 if (sw_flags(meta) & 2) break;
             }
-        }
-    corr_exit:;
-    } else {
-        // -------------------------------------------------------- softmax + epilogue of slot x
-        const int x = warp >> 2, wq = warp & 3;
-        const int r = 32 * wq + (int)lane;  // query row of the tile == TMEM lane
-        const int qbit = r >> 6;            // 0: query cube i1, 1: i2
-        SlotBars& sb = m.bar[x];
-        const uint32_t lane_base = tbase + ((uint32_t)(32 * wq) << 16);
-        const uint32_t s_addr = lane_base + s_col(x), o_addr = lane_base + o_col(x);
-        constexpr float kNeutral = NEG ? INFINITY : -INFINITY;  // a masked logit
-        int g = 0, tc = 0;
-        float m_run = -INFINITY, l_run = 0.f;
-        for (int n = x; n < my_tiles; n += 2, ++tc) {
-            const TileRef t = checked_tile(blockIdx.x + n * gridDim.x, H, nq, tiles_per_bh, plan, nullptr);
-            for (;;) {
-                if (!wait_warp_inl(&sb.s_full, g & 1, &m.abort, err)) goto softmax_exit;
-                const uint32_t meta = m.s_meta[x];
-                const int na = sw_na(meta), nb = sw_nb(meta), ma = sw_ma(meta), mb = sw_mb(meta), flags = sw_flags(meta);
-                const int myn0 = ((ma >> qbit) & 1) ? na : 0, myn1 = ((mb >> qbit) & 1) ? nb : 0;
-                if (flags & 1) {
-                    m_run = -INFINITY;
-                    l_run = 0.f;
-                }
-                tc_fence_after();
-                // pass 1: row extreme over the selected keys, one 32-column TMEM load at a
-                // time (small loop bodies keep the hot code in the instruction cache)
-                float e4[4] = {kNeutral, kNeutral, kNeutral, kNeutral};
-#pragma unroll 1
-                for (int ch = 0; ch < 4; ++ch) {
-                    const int nv = ch < 2 ? myn0 : myn1;
-                    const int cb = (ch & 1) * 32;  // first column of the chunk in its 64-key half
-                    if (nv <= cb) continue;        // no selected key in this chunk
-                    float sc[32];
-                    tmem_ld32(s_addr + 32 * ch, reinterpret_cast<uint32_t*>(sc));
-                    tmem_ld_wait();
-                    if (nv < cb + 32) {
-#pragma unroll
-                        for (int c = 0; c < 32; ++c) sc[c] = cb + c < nv ? sc[c] : kNeutral;
-                    }
-#pragma unroll
-                    for (int c = 0; c < 32; c += 8) {
-#pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            e4[u] = NEG ? min3(e4[u], sc[c + 2 * u], sc[c + 2 * u + 1])
-                                        : max3(e4[u], sc[c + 2 * u], sc[c + 2 * u + 1]);
-                    }
-                }
-                const float ext = NEG ? min3(fminf(e4[0], e4[1]), e4[2], e4[3]) : max3(fmaxf(e4[0], e4[1]), e4[2], e4[3]);
-                const bool any_valid = (myn0 | myn1) != 0;
-                const float m_step = any_valid ? ext * scale_log2 : -INFINITY;  // base-2 units
-                const bool raise = m_step > m_run + kTau;                    // false for -inf
-                float alpha = 1.f;
-                if (raise) {
-                    alpha = m_run == -INFINITY ? 0.f : ex2(m_run - m_step);
-                    m_run = m_step;
-                    l_run *= alpha;
-                }
-                m.alpha[x][r] = alpha;
-                const bool warp_raise = __any_sync(0xffffffffu, raise && !(flags & 1));
-                if (lane == 0) m.rflag[x][wq] = warp_raise ? 1 : 0;
-                mbar_arrive(&sb.a_full);
-
-                // pass 2: P = exp2(x - m) as bf16 pairs over S's first 64 columns; the
-                // chunk's P lands on columns whose logits were already consumed
-                const float mu = m_run == -INFINITY ? 0.f : m_run;
-                float ls0 = 0.f, ls1 = 0.f;
-#pragma unroll 1
-                for (int ch = 0; ch < 4; ++ch) {
-                    const int nv = ch < 2 ? myn0 : myn1;
-                    const int cb = (ch & 1) * 32;
-                    uint32_t pk[16];
-                    if (nv <= cb) {
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) pk[c] = 0u;
-                    } else {
-                        float sc[32];
-                        tmem_ld32(s_addr + 32 * ch, reinterpret_cast<uint32_t*>(sc));
-                        tmem_ld_wait();
-                        if (nv < cb + 32) {
-#pragma unroll
-                            for (int c = 0; c < 32; ++c) sc[c] = cb + c < nv ? sc[c] : kNeutral;
-                        }
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) {
-                            float x0, x1, p0, p1;
-                            ffma2(x0, x1, sc[2 * c], sc[2 * c + 1], scale_log2, scale_log2, -mu, -mu);
-                            if ((kPolyPairs >> c) & 1) {
-                                // weights below 2^-125 (masked keys included) become 2^-125
-                                const float2 pp = ex2_fma2(make_float2(fmaxf(x0, -125.f), fmaxf(x1, -125.f)));
-                                p0 = pp.x;
-                                p1 = pp.y;
-                            } else {
-                                p0 = ex2(x0);
-                                p1 = ex2(x1);
-                            }
-                            fadd2(ls0, ls1, p0, p1);
-                            pk[c] = pack_bf16(p0, p1);
-                        }
-                    }
-                    tmem_st16(s_addr + 16 * ch, pk);
-                }
-                l_run += ls0 + ls1;
-                tmem_st_wait();
-                tc_fence_before();
-                mbar_arrive(&sb.p_full);
-                ++g;
-                if (flags & 2) break;
-            }
 
             // ---- epilogue: out[b, 64 i + (r % 64), h, :] = O[r, :] / l; lse = (m + log2 l) ln 2
-            if (!wait_warp_inl(&sb.o_full, tc & 1, &m.abort, err)) goto softmax_exit;
+            if (!wait_warp(&bb.o_full, n & 1, &m.abort, err)) goto corr_exit;
+            if (!wait_warp(&bb.l_full[n & 1], (n >> 1) & 1, &m.abort, err)) goto corr_exit;
             tc_fence_after();
             {
+                const TileRef t = checked_tile(blockIdx.x + n * gridDim.x, H, nq, tiles_per_bh, plan, nullptr);
+                const float l = m.lfin[n & 1][r];
+                const float m_row = m.mfin[n & 1][r];
+                mbar_arrive(&bb.l_empty[n & 1]);
                 const int cube = qbit == 0 ? t.i1 : t.i2;
-                const float inv = l_run > 0.f ? __frcp_rn(l_run) : 0.f;
+                const bool has = l > 0.f;
+                const float inv = has ? __frcp_rn(l) : 0.f;
                 const int64_t token = (int64_t)t.b * S + 64LL * cube + (r & 63);
                 uint16_t* dst = out + (token * H + t.h) * kD;
 #pragma unroll 1
                 for (int c4 = 0; c4 < 4; ++c4) {
                     uint32_t o[32];
-                    tmem_ld32(o_addr + 32 * c4, o);
+                    tmem_ld32(oa + 32 * c4, o);
                     tmem_ld_wait();
                     if (cube >= 0) {
 #pragma unroll
@@ -479,25 +458,186 @@ __global__ void __launch_bounds__(kThreads, 1)
                             uint32_t w[4];
 #pragma unroll
                             for (int e = 0; e < 4; ++e)
-                                w[e] = pack_bf16(__uint_as_float(o[8 * v + 2 * e]) * inv,
-                                                 __uint_as_float(o[8 * v + 2 * e + 1]) * inv);
+                                w[e] = has ? pack_bf16(__uint_as_float(o[8 * v + 2 * e]) * inv,
+                                                       __uint_as_float(o[8 * v + 2 * e + 1]) * inv)
+                                           : 0u;
                             st_global_v4(dst + 32 * c4 + 8 * v, w[0], w[1], w[2], w[3]);
                         }
                     }
                 }
                 if (lse != nullptr && cube >= 0)
                     lse[((int64_t)t.b * H + t.h) * S + 64LL * cube + (r & 63)] =
-                        l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+                        has ? (m_row + __log2f(l)) * 0.69314718055994531f : -INFINITY;
             }
             tc_fence_before();
+        }
+    corr_exit:;
+    } else {
+        // ------------------------------------------------------------ softmax: steps in turn
+        //
+        // Warp w owns TMEM lanes 32 (w % 4) .. +31 (query rows, thread = row) and
+        // the steps g with g % 3 == w / 4, all 128 columns.  The three warps of a
+        // lane quarter share an SMSP and work on three consecutive steps at once
+        // (one per S buffer), so the SMSP's exp2 units always have work while
+        // any one warp waits for TMEM or a barrier.  A row's running offset and
+        // running sum pass from step to step through shared memory (dec: offset
+        // and tile count after the decision of step g; lsum: row sum after step g).
+        // Those barriers come in three sets by step % 3: the warp of step g waits
+        // for step g - 1 only after its own step g - 3, which waited for g - 4,
+        // so a barrier is never two phases behind its waiter.
+        const int wq = warp & 3, par = warp >> 2;
+        const int r = 32 * wq + (int)lane;  // query row of the tile == TMEM lane
+        const int qbit = r >> 6;            // 0: query cube i1, 1: i2
+        const uint32_t lane_base = tbase + ((uint32_t)(32 * wq) << 16);
+        constexpr float kNeutral = NEG ? INFINITY : -INFINITY;  // a masked logit
+        for (int g = par;; g += kSBuf) {
+            const int b = g % kSBuf;
+            const uint32_t spar = (g / kSBuf) & 1;
+            int n_before = 0;
+            float m_prev = -INFINITY;
+            bool got_dec = false;
+            if (my_tiles == 0) break;
+            if (g > 0 && !probe_warp(&bb.s_full[b], spar)) {
+                // step g may not exist: the previous step's hand-off says
+                if (!wait_warp_inl(&bb.dec[(g - 1) % kSBuf][wq], ((g - 1) / kSBuf) & 1, &m.abort, err))
+                    goto softmax_exit;
+                n_before = m.n_state[(g - 1) & 1][wq];
+                if (n_before >= my_tiles) {
+                    // no step g: pass the end on to the warp of step g + 1
+                    if (lane == 0) m.n_state[g & 1][wq] = n_before;
+                    mbar_arrive(&bb.dec[b][wq]);
+                    break;
+                }
+                m_prev = m.m_state[(g - 1) & 1][r];
+                got_dec = true;
+            }
+            if (!wait_warp_inl(&bb.s_full[b], spar, &m.abort, err)) goto softmax_exit;
+            const uint32_t meta = m.s_meta[b];
+            tc_fence_after();
+            const int na = sw_na(meta), nb = sw_nb(meta), flags = sw_flags(meta);
+            const int nv0 = ((sw_ma(meta) >> qbit) & 1) ? na : 0;  // valid keys of each half
+            const int nv1 = ((sw_mb(meta) >> qbit) & 1) ? nb : 0;  // for this row (warp-uniform)
+            const uint32_t s_addr = lane_base + 128u * b;
+
+            // pass 1: extreme of the selected logits, one 32-column chunk at a time
+            // (chunk ch: columns 32 ch .. +31, key half ch / 2)
+            float e4[4] = {kNeutral, kNeutral, kNeutral, kNeutral};
+#pragma unroll 1
+            for (int ch = 0; ch < 4; ++ch) {
+                const int nv = (ch < 2 ? nv0 : nv1) - 32 * (ch & 1);  // valid columns of the chunk
+                if (nv <= 0) continue;
+                float sc[32];
+                tmem_ld32(s_addr + 32 * ch, reinterpret_cast<uint32_t*>(sc));
+                tmem_ld_wait();
+                if (nv < 32) {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) sc[c] = c < nv ? sc[c] : kNeutral;
+                }
+#pragma unroll
+                for (int c = 0; c < 32; c += 8) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        e4[u] = NEG ? min3(e4[u], sc[c + 2 * u], sc[c + 2 * u + 1])
+                                    : max3(e4[u], sc[c + 2 * u], sc[c + 2 * u + 1]);
+                }
+            }
+            const float ext = NEG ? min3(fminf(e4[0], e4[1]), e4[2], e4[3]) : max3(fmaxf(e4[0], e4[1]), e4[2], e4[3]);
+
+            // decision: the row's offset after this step (lazy: raised by more than kTau only)
+            if (g > 0 && !got_dec) {
+                if (!wait_warp_inl(&bb.dec[(g - 1) % kSBuf][wq], ((g - 1) / kSBuf) & 1, &m.abort, err))
+                    goto softmax_exit;
+                n_before = m.n_state[(g - 1) & 1][wq];
+                m_prev = m.m_state[(g - 1) & 1][r];
+            }
+            if (flags & 1) m_prev = -INFINITY;  // a tile's first step starts afresh
+            const float m_step = (nv0 | nv1) != 0 ? ext * scale_log2 : -INFINITY;  // base-2 units
+            const bool raise = m_step > m_prev + kTau;                            // false for -inf
+            const float m_run = raise ? m_step : m_prev;
+            // alpha scales O and the running sum; 0 at a tile's first step (nothing before)
+            const float alpha = (flags & 1) ? 0.f : (raise ? (m_prev == -INFINITY ? 0.f : ex2(m_prev - m_step)) : 1.f);
+            const int n_after = n_before + ((flags & 2) ? 1 : 0);
+            m.alpha[b][r] = alpha;
+            m.m_state[g & 1][r] = m_run;
+            const bool warp_raise = __any_sync(0xffffffffu, raise && !(flags & 1));
+            if (lane == 0) {
+                m.rflag[b][wq] = warp_raise ? 1 : 0;
+                m.n_state[g & 1][wq] = n_after;
+            }
+            mbar_arrive(&bb.a_full[b]);
+            mbar_arrive(&bb.dec[b][wq]);
+
+            // pass 2: P = exp2(x - m) as bf16 pairs; chunk ch's P goes to columns
+            // 64 (ch / 2) + 16 (ch % 2): each half's P fills the half's first 32
+            // columns, over logits already consumed
+            const float mu = m_run == -INFINITY ? 0.f : m_run;
+            float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll 1
+            for (int ch = 0; ch < 4; ++ch) {
+                const int nv = (ch < 2 ? nv0 : nv1) - 32 * (ch & 1);
+                uint32_t pk[16];
+                if (nv > 0) {
+                    float sc[32];
+                    tmem_ld32(s_addr + 32 * ch, reinterpret_cast<uint32_t*>(sc));
+                    tmem_ld_wait();
+                    if (nv < 32) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) sc[c] = c < nv ? sc[c] : kNeutral;
+                    }
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        float x0, x1, p0, p1;
+                        ffma2(x0, x1, sc[2 * c], sc[2 * c + 1], scale_log2, scale_log2, -mu, -mu);
+                        if ((kPolyPairs >> (c & 15)) & 1) {
+                            // weights below 2^-125 (masked keys included) become 2^-125
+                            const float2 pp = ex2_fma2(make_float2(fmaxf(x0, -125.f), fmaxf(x1, -125.f)));
+                            p0 = pp.x;
+                            p1 = pp.y;
+                        } else {
+                            p0 = ex2(x0);
+                            p1 = ex2(x1);
+                        }
+                        fadd2(ls0, ls1, p0, p1);
+                        pk[c] = pack_bf16(p0, p1);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) pk[c] = 0u;
+                }
+                tmem_st16(s_addr + 64 * (ch >> 1) + 16 * (ch & 1), pk);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&bb.p_full[b]);
+
+            // running row sum: l(g) = l(g - 1) * alpha(g) + sum of P(g)
+            float l_prev = 0.f;
+            if (g > 0) {
+                if (!wait_warp_inl(&bb.lsum[(g - 1) % kSBuf][wq], ((g - 1) / kSBuf) & 1, &m.abort, err))
+                    goto softmax_exit;
+                if (!(flags & 1)) l_prev = m.l_state[(g - 1) & 1][r];
+            }
+            const float l_run = l_prev * alpha + (ls0 + ls1);
+            m.l_state[g & 1][r] = l_run;
+            mbar_arrive(&bb.lsum[b][wq]);
+            if (flags & 2) {
+                // the tile's row sum and offset for the epilogue (ring of two tiles)
+                const int n = n_before;
+                if (!wait_warp_inl(&bb.l_empty[n & 1], ((n >> 1) & 1) ^ 1, &m.abort, err)) goto softmax_exit;
+                m.lfin[n & 1][r] = l_run;
+                m.mfin[n & 1][r] = m_run;
+                mbar_arrive(&bb.l_full[n & 1]);
+            }
+            if (meta & kFinal) break;
         }
     softmax_exit:;
     }
 
+    // ------------------------------------------------------------ teardown
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == kWarpRole0 + 1) tmem_dealloc(tbase, 512);
+    if (warp == kWarpMma) tmem_dealloc(tbase, 512);
 }
 
 template <bool NEG>
