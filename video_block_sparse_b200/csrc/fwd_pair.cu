@@ -74,9 +74,12 @@ constexpr uint32_t kOCol = 384;
 constexpr uint32_t kFinal = 1u << 22;  // step word: last step of the CTA's last tile
 
 // Pairs (bit c: columns 2c, 2c+1 of each 32-column chunk) whose exp2 runs on
-// the FMA pipe instead of the multi-function unit.
+// the FMA pipe instead of the multi-function unit.  None by default: with three
+// softmax warps per SMSP the exp pass is bound by latency and instruction issue,
+// not by the multi-function unit, and the FMA-pipe exp2 costs eight more
+// instructions a pair (Wan 832x480: 5.94 ms without, 6.16 ms with 6 of 16 pairs).
 #ifndef VSA_POLY_PAIRS
-#define VSA_POLY_PAIRS 0x5252
+#define VSA_POLY_PAIRS 0
 #endif
 constexpr uint32_t kPolyPairs = VSA_POLY_PAIRS;
 
