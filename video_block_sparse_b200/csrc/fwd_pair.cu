@@ -66,7 +66,8 @@ constexpr int kWarpCorr0 = 12;  // warps 12-15: correction and epilogue
 constexpr int kWarpProd = 16;
 constexpr int kWarpMma = 17;
 constexpr int kWarpVProd = 18;
-constexpr int kThreads = 19 * 32;
+constexpr int kWarpQk = 19;  // kWarpMma issues the PV products, kWarpQk the QK products
+constexpr int kThreads = 20 * 32;
 constexpr int kVReq = 4;  // ring of V load requests from the K producer to the V producer
 constexpr int kSBuf = 3;  // S/P buffers in TMEM (also the V ring depth)
 constexpr int kKBuf = 2;  // K ring depth
@@ -97,7 +98,8 @@ struct Bars {
     uint64_t dec[kSBuf][4];   // [step % 3][lane quarter]: offsets after the step decided (32)
     uint64_t lsum[kSBuf][4];  // [step % 3][lane quarter]: row sums after the step written (32)
     uint64_t vr_full[kVReq], vr_empty[kVReq];  // V load request posted / taken
-    uint64_t drain;
+    uint64_t pv_issued[kSBuf];  // PV of the step in S buffer b issued (after a tcgen05 before-fence)
+    uint64_t drain[2];
 };
 
 struct Misc {
@@ -188,7 +190,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_init(&bb.lsum[i][j], 32);
             }
         mbar_init(&bb.o_full, 1);
-        mbar_init(&bb.drain, 1);
+        for (int i = 0; i < kSBuf; ++i) mbar_init(&bb.pv_issued[i], 1);
+        mbar_init(&bb.drain[0], 1);
+        mbar_init(&bb.drain[1], 1);
         m.abort = 0;
         fence_mbar_init();
     }
@@ -306,33 +310,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (lane == 0 && armed_v >= 0 && aborted_flag(&m.abort)) drain_wait(&bb.v_full[armed_vb], armed_v);
         __syncwarp();
-    } else if (warp == kWarpMma) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == kWarpMma || warp == kWarpQk) {
+        // ------------------------------------------------------------ MMA issuers
+        // Two warps feed the tensor core: warp kWarpQk issues the QK products, warp
+        // kWarpMma the PV products.  While one is blocked issuing a group (the
+        // tensor core's queue is short), the other does the barrier checks for
+        // its next group, so the groups reach the tensor core back to back.  The
+        // order QK(j) after PV(j - 3) (they share S buffer j % 3) is kept by
+        // barrier pv_issued: the PV warp arrives after issuing PV(j) (after a
+        // tcgen05 before-fence), the QK warp waits for it before QK(j + 3).
+        // In each warp the whole warp runs the schedule and one elected lane issues.
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);
         // operand descriptors built once; a k-step adds its byte offset / 16
         const uint64_t d_hi = smem_desc_sw128(0, 0, 1024);
-        const uint32_t ql = (uint32_t)smem_desc_sw128(tiles + L::Q_OFF, 16, 1024);
-        const uint32_t kl0 = (uint32_t)smem_desc_sw128(tiles + L::K_OFF, 16, 1024);
-        const uint32_t vl0 = (uint32_t)smem_desc_sw128(tiles + L::V_OFF, 2 * kHalfBox, 1024);
-        const uint32_t o_tmem = tbase + kOCol;
-        int j_qk = 0, j_pv = 0, qn = 0;
-        bool qk_done = my_tiles == 0, o_init = false, aborted = false;
-        for (;;) {
-            // ---- QK of the steps up to two ahead of the next PV (S buffers are free)
-            while (!qk_done && j_qk < j_pv + kSBuf) {
-                const int kb = j_qk % kKBuf;
-                const uint32_t kpar = (j_qk / kKBuf) & 1;
-                // with a PV pending, a QK whose operands are not there yet waits for later
-                if (j_pv < j_qk && !probe_warp(&bb.k_full[kb], kpar)) break;
-                if (!wait_warp(&bb.k_full[kb], kpar, &m.abort, err)) { aborted = true; break; }
+        bool aborted = false;
+        if (warp == kWarpQk) {
+            const uint32_t ql = (uint32_t)smem_desc_sw128(tiles + L::Q_OFF, 16, 1024);
+            const uint32_t kl0 = (uint32_t)smem_desc_sw128(tiles + L::K_OFF, 16, 1024);
+            int qn = 0;
+            for (int j = 0; my_tiles > 0; ++j) {
+                const int kb = j % kKBuf, sb = j % kSBuf;
+                if (!wait_warp(&bb.k_full[kb], (j / kKBuf) & 1, &m.abort, err)) { aborted = true; break; }
                 const uint32_t meta = m.k_meta[kb];
                 if (sw_flags(meta) & 1) {
-                    if (j_pv < j_qk && !probe_warp(&bb.q_full, qn & 1)) break;
                     if (!wait_warp(&bb.q_full, qn & 1, &m.abort, err)) { aborted = true; break; }
                     ++qn;
                 }
-                const int sb = j_qk % kSBuf;
+                // S buffer sb is free once PV(j - 3) has been issued
+                if (j >= kSBuf && !wait_warp(&bb.pv_issued[sb], ((j - kSBuf) / kSBuf) & 1, &m.abort, err)) {
+                    aborted = true;
+                    break;
+                }
                 __syncwarp();
                 if (lane == 0) {
                     m.s_meta[sb] = meta;
@@ -349,55 +358,62 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma_commit_elect(&bb.s_full[sb]);
                 umma_commit_elect(&bb.k_empty[kb]);
                 if (sw_flags(meta) & 2) umma_commit_elect(&bb.q_empty);
-                if (meta & kFinal) qk_done = true;
-                ++j_qk;
+                if (meta & kFinal) break;
             }
-            if (aborted || j_pv == j_qk) break;  // aborted, or every step done
-            // ---- O += P . V for step j_pv
-            const int sb = j_pv % kSBuf;
-            const uint32_t par = (j_pv / kSBuf) & 1;
-            if (!wait_warp(&bb.p_full[sb], par, &m.abort, err)) { aborted = true; break; }
-            if (!wait_warp(&bb.v_full[sb], par, &m.abort, err)) { aborted = true; break; }
-            const uint32_t meta = m.s_meta[sb];
-            const int na = sw_na(meta), nb = sw_nb(meta);
-            const uint32_t vl = vl0 + ((uint32_t)sb * kTileBytes >> 4);
-            const int za = (na & 15) ? 16 - (na & 15) : 0, zb = (nb & 15) ? 16 - (nb & 15) : 0;
-            if (za + zb > 0) {
-                // V rows between vbs and the next multiple of 16 are read by the last
-                // k-step of their cube: zero them (both d halves) before the product
-                const uint32_t vbase = tiles + L::V_OFF + sb * kTileBytes;
-                for (int w = lane; w < (za + zb) * 16; w += 32) {
-                    const int zr = w >> 4, chunk = w & 15;
-                    const int row = zr < za ? na + zr : 64 + nb + (zr - za);
-                    sts128(vbase + (chunk >> 3) * (2 * kHalfBox) + row * 128 + (chunk & 7) * 16, 0u, 0u, 0u, 0u);
+        } else {
+            const uint32_t vl0 = (uint32_t)smem_desc_sw128(tiles + L::V_OFF, 2 * kHalfBox, 1024);
+            const uint32_t o_tmem = tbase + kOCol;
+            bool o_init = false;
+            for (int j = 0; my_tiles > 0; ++j) {
+                const int sb = j % kSBuf;
+                const uint32_t par = (j / kSBuf) & 1;
+                if (!wait_warp(&bb.v_full[sb], par, &m.abort, err)) { aborted = true; break; }
+                if (!wait_warp(&bb.p_full[sb], par, &m.abort, err)) { aborted = true; break; }
+                const uint32_t meta = m.s_meta[sb];
+                const int na = sw_na(meta), nb = sw_nb(meta);
+                const uint32_t vl = vl0 + ((uint32_t)sb * kTileBytes >> 4);
+                const int za = (na & 15) ? 16 - (na & 15) : 0, zb = (nb & 15) ? 16 - (nb & 15) : 0;
+                if (za + zb > 0) {
+                    // V rows between vbs and the next multiple of 16 are read by the last
+                    // k-step of their cube: zero them (both d halves) before the product
+                    const uint32_t vbase = tiles + L::V_OFF + sb * kTileBytes;
+                    for (int w = lane; w < (za + zb) * 16; w += 32) {
+                        const int zr = w >> 4, chunk = w & 15;
+                        const int row = zr < za ? na + zr : 64 + nb + (zr - za);
+                        sts128(vbase + (chunk >> 3) * (2 * kHalfBox) + row * 128 + (chunk & 7) * 16, 0u, 0u, 0u, 0u);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-            }
-            tc_fence_after();
-            // k-steps (16 keys) 0..ceil16(na)-1 of half 0 and 4..4+ceil16(nb)-1 of half 1; the
-            // bf16 P of key half h sits in the first 32 columns of that half's 64
-            const uint32_t kmask = ((1u << ((na + 15) >> 4)) - 1u) | (((1u << ((nb + 15) >> 4)) - 1u) << 4);
-            const uint32_t p_tmem = tbase + 128u * sb;
-            if (sw_flags(meta) & 1) o_init = false;
-            uint32_t acc = o_init ? 1u : 0u;
+                tc_fence_after();
+                // k-steps (16 keys) 0..ceil16(na)-1 of half 0 and 4..4+ceil16(nb)-1 of half 1; the
+                // bf16 P of key half h sits in the first 32 columns of that half's 64
+                const uint32_t kmask = ((1u << ((na + 15) >> 4)) - 1u) | (((1u << ((nb + 15) >> 4)) - 1u) << 4);
+                const uint32_t p_tmem = tbase + 128u * sb;
+                if (sw_flags(meta) & 1) o_init = false;
+                uint32_t acc = o_init ? 1u : 0u;
 #pragma unroll
-            for (int kstep = 0; kstep < 8; ++kstep) {
-                if (kmask & (1u << kstep)) {
-                    const uint32_t a_col = kstep < 4 ? 8u * kstep : 64u + 8u * (kstep - 4);
-                    umma_ts_elect(o_tmem, p_tmem + a_col, d_hi | (vl + ((kstep * 2048) >> 4)), idesc_pv, acc);
-                    acc = 1u;
+                for (int kstep = 0; kstep < 8; ++kstep) {
+                    if (kmask & (1u << kstep)) {
+                        const uint32_t a_col = kstep < 4 ? 8u * kstep : 64u + 8u * (kstep - 4);
+                        umma_ts_elect(o_tmem, p_tmem + a_col, d_hi | (vl + ((kstep * 2048) >> 4)), idesc_pv, acc);
+                        acc = 1u;
+                    }
                 }
+                o_init = o_init || kmask != 0;
+                umma_commit_elect(&bb.v_empty[sb]);
+                umma_commit_elect(&bb.pv_done[j & 1]);
+                if (sw_flags(meta) & 2) umma_commit_elect(&bb.o_full);
+                // PV(j) is in the tensor core's queue: S buffer sb may be written again
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bb.pv_issued[sb]);
+                if (meta & kFinal) break;
             }
-            o_init = o_init || kmask != 0;
-            umma_commit_elect(&bb.v_empty[sb]);
-            umma_commit_elect(&bb.pv_done[j_pv & 1]);
-            if (sw_flags(meta) & 2) umma_commit_elect(&bb.o_full);
-            ++j_pv;
         }
         if (aborted) {
-            umma_commit_elect(&bb.drain);
-            if (lane == 0) drain_wait(&bb.drain, 0);
+            umma_commit_elect(&bb.drain[warp == kWarpQk ? 1 : 0]);
+            if (lane == 0) drain_wait(&bb.drain[warp == kWarpQk ? 1 : 0], 0);
             __syncwarp();
         }
     } else if (warp >= kWarpCorr0) {
