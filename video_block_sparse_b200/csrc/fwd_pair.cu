@@ -109,6 +109,7 @@ struct Misc {
     uint32_t s_meta[kSBuf];  // step word of each S buffer
     uint32_t tmem_base;
     int abort;
+    int end_g;  // the CTA's last step, once its softmax is done (the other softmax warps stop there)
     alignas(16) float alpha[kSBuf][128];  // per S buffer, row: O rescale factor of that step
     int rflag[kSBuf][4];                  // per S buffer, lane quarter: some row rescales
     float m_state[2][128];                // [step parity][row]: offset after the step's decision
@@ -131,14 +132,6 @@ struct Layout {
     static constexpr uint32_t SMEM_BYTES = MISC_BYTES + TILE_BYTES + 1024;  // + alignment slack
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
-
-// Non-blocking check of a phase by lane 0, made warp-uniform.
-__device__ __forceinline__ bool probe_warp(uint64_t* bar, uint32_t parity)
-{
-    uint32_t ok = 0;
-    if ((threadIdx.x & 31) == 0) ok = mbar_test_wait(bar, parity) ? 1u : 0u;
-    return __shfl_sync(0xffffffffu, ok, 0) != 0;
-}
 
 template <bool NEG>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -194,6 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bb.drain[0], 1);
         mbar_init(&bb.drain[1], 1);
         m.abort = 0;
+        m.end_g = 0x7fffffff;
         fence_mbar_init();
     }
     if (warp == kWarpMma) {
@@ -514,23 +508,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t spar = (g / kSBuf) & 1;
             int n_before = 0;
             float m_prev = -INFINITY;
-            bool got_dec = false;
             if (my_tiles == 0) break;
-            if (g > 0 && !probe_warp(&bb.s_full[b], spar)) {
-                // step g may not exist: the previous step's hand-off says
-                if (!wait_warp_inl(&bb.dec[(g - 1) % kSBuf][wq], ((g - 1) / kSBuf) & 1, &m.abort, err))
-                    goto softmax_exit;
-                n_before = m.n_state[(g - 1) & 1][wq];
-                if (n_before >= my_tiles) {
-                    // no step g: pass the end on to the warp of step g + 1
-                    if (lane == 0) m.n_state[g & 1][wq] = n_before;
-                    mbar_arrive(&bb.dec[b][wq]);
-                    break;
-                }
-                m_prev = m.m_state[(g - 1) & 1][r];
-                got_dec = true;
-            }
             if (!wait_warp_inl(&bb.s_full[b], spar, &m.abort, err)) goto softmax_exit;
+            if (g > *reinterpret_cast<volatile int*>(&m.end_g)) break;  // past the CTA's last step
             const uint32_t meta = m.s_meta[b];
             tc_fence_after();
             const int na = sw_na(meta), nb = sw_nb(meta), flags = sw_flags(meta);
@@ -563,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float ext = NEG ? min3(fminf(e4[0], e4[1]), e4[2], e4[3]) : max3(fmaxf(e4[0], e4[1]), e4[2], e4[3]);
 
             // decision: the row's offset after this step (lazy: raised by more than kTau only)
-            if (g > 0 && !got_dec) {
+            if (g > 0) {
                 if (!wait_warp_inl(&bb.dec[(g - 1) % kSBuf][wq], ((g - 1) / kSBuf) & 1, &m.abort, err))
                     goto softmax_exit;
                 n_before = m.n_state[(g - 1) & 1][wq];
@@ -647,7 +627,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m.mfin[n & 1][r] = m_run;
                 mbar_arrive(&bb.l_full[n & 1]);
             }
-            if (meta & kFinal) break;
+            if (meta & kFinal) {
+                // no step g + 1 or g + 2 will come: complete their s_full phases (two
+                // arrivals each) so that the warps waiting for them wake up, see
+                // end_g and stop.  Those warps have consumed their previous phase of
+                // those barriers: they decided steps g - 2 and g - 1 before this one.
+                if (wq == 0 && lane == 0) {
+                    m.end_g = g;
+                    for (int e = 1; e <= 2; ++e) {
+                        mbar_arrive(&bb.s_full[(g + e) % kSBuf]);
+                        mbar_arrive(&bb.s_full[(g + e) % kSBuf]);
+                    }
+                }
+                break;
+            }
         }
     softmax_exit:;
     }
