@@ -61,8 +61,7 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kSoftWarps = 12;  // warps 0-11: softmax, three per SMSP
-constexpr int kWarpCorr0 = 12;  // warps 12-15: correction and epilogue
+constexpr int kWarpCorr0 = 12;  // warps 0-11: softmax, three per SMSP; 12-15: correction and epilogue
 constexpr int kWarpProd = 16;
 constexpr int kWarpMma = 17;
 constexpr int kWarpVProd = 18;

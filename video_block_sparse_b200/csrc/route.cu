@@ -239,23 +239,47 @@ __global__ void __launch_bounds__(256) score_topk_kernel(const uint16_t* __restr
     }
     __syncthreads();
 
+    // Each thread scores kJT consecutive key cubes against the CTA's QB query
+    // cubes, so that every q element read from shared memory feeds kJT FMAs
+    // (two at QB = 8: four would cost occupancy).  Every (query, key) sum still
+    // runs over d = 0..127 in order.
+    constexpr int kJT = QB >= 8 ? 2 : 4;
     const uint4* krow = reinterpret_cast<const uint4*>(kc + head * nq * kD);
-    for (int j = threadIdx.x; j < nq; j += blockDim.x) {
-        double acc[QB];
+    for (int j0 = threadIdx.x * kJT; j0 < nq; j0 += blockDim.x * kJT) {
+        double acc[QB][kJT];
 #pragma unroll
-        for (int r = 0; r < QB; ++r) acc[r] = 0.0;
+        for (int r = 0; r < QB; ++r)
+#pragma unroll
+            for (int t = 0; t < kJT; ++t) acc[r][t] = 0.0;
         for (int ch = 0; ch < kD / 8; ++ch) {
-            const uint4 w = __ldg(krow + (int64_t)j * (kD / 8) + ch);
-            const uint32_t p[4] = {w.x, w.y, w.z, w.w};
+            uint32_t p[kJT][4];
+#pragma unroll
+            for (int t = 0; t < kJT; ++t) {
+                const uint4 w = j0 + t < nq ? __ldg(krow + (int64_t)(j0 + t) * (kD / 8) + ch) : make_uint4(0, 0, 0, 0);
+                p[t][0] = w.x;
+                p[t][1] = w.y;
+                p[t][2] = w.z;
+                p[t][3] = w.w;
+            }
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const double kv = bf16_to_f64((e & 1) ? (p[e >> 1] >> 16) : (p[e >> 1] & 0xFFFFu));
+                double kv[kJT];
 #pragma unroll
-                for (int r = 0; r < QB; ++r) acc[r] = __fma_rn(qd[r * kD + ch * 8 + e], kv, acc[r]);
+                for (int t = 0; t < kJT; ++t)
+                    kv[t] = bf16_to_f64((e & 1) ? (p[t][e >> 1] >> 16) : (p[t][e >> 1] & 0xFFFFu));
+#pragma unroll
+                for (int r = 0; r < QB; ++r) {
+                    const double qv = qd[r * kD + ch * 8 + e];
+#pragma unroll
+                    for (int t = 0; t < kJT; ++t) acc[r][t] = __fma_rn(qv, kv[t], acc[r][t]);
+                }
             }
         }
 #pragma unroll
-        for (int r = 0; r < QB; ++r) keys[r * nq + j] = score_key(acc[r]);
+        for (int t = 0; t < kJT; ++t)
+            if (j0 + t < nq)
+#pragma unroll
+                for (int r = 0; r < QB; ++r) keys[r * nq + j0 + t] = score_key(acc[r][t]);
     }
     __syncthreads();
 
