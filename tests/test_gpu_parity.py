@@ -189,6 +189,23 @@ def test_fwd_edge_lists(vsa, seed, topk, dup):
         _check_items(p, out, lse, oracle.all_items(1, 2, 5), f"edge{seed}/{flags}", precise=flags != 0)
 
 
+@pytest.mark.parametrize("seed,topk,plan", [(20, 1, False), (21, 2, False), (22, 3, True)])
+def test_fwd_many_short_tiles(vsa, seed, topk, plan):
+    """More tiles than SMs, each of one to three steps (two to six KV cubes), some
+    cubes empty: every CTA walks several tiles, so the step rings, the two-tile
+    hand-off of row sums to the epilogue and the end-of-stream signalling run with
+    very short tiles.  Every row is checked."""
+    p = _small(seed, nq=9, H=80, topk=topk)
+    q, k, v = common.dev(p.qt), common.dev(p.kt), common.dev(p.vt)
+    idx = torch.from_numpy(p.idx).cuda()
+    vbs = torch.from_numpy(p.vbs).cuda()
+    pl = vsa.plan(idx) if plan else None
+    out, lse = vsa.fwd(q, k, v, idx, vbs, p.cfg.sm_scale, want_lse=True, plan=pl)
+    torch.cuda.synchronize()
+    _no_device_error(vsa)
+    _check_items(p, out, lse, oracle.all_items(1, 80, 9), f"short{seed}")
+
+
 def test_fwd_all_masked_rows(vsa):
     p = _small(10, nq=3, H=1, topk=2, vbs=[0, 0, 64])
     p.idx[:] = np.array([[[[0, 1], [2, 0], [1, 1]]]], np.int32)
