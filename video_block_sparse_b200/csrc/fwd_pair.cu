@@ -508,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int n_before = 0;
             float m_prev = -INFINITY;
             if (my_tiles == 0) break;
-            if (!wait_warp_inl(&bb.s_full[b], spar, &m.abort, err)) goto softmax_exit;
+            if (!wait_warp(&bb.s_full[b], spar, &m.abort, err)) goto softmax_exit;
             if (g > *reinterpret_cast<volatile int*>(&m.end_g)) break;  // past the CTA's last step
             const uint32_t meta = m.s_meta[b];
             tc_fence_after();
@@ -543,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
             // decision: the row's offset after this step (lazy: raised by more than kTau only)
             if (g > 0) {
-                if (!wait_warp_inl(&bb.dec[(g - 1) % kSBuf][wq], ((g - 1) / kSBuf) & 1, &m.abort, err))
+                if (!wait_warp(&bb.dec[(g - 1) % kSBuf][wq], ((g - 1) / kSBuf) & 1, &m.abort, err))
                     goto softmax_exit;
                 n_before = m.n_state[(g - 1) & 1][wq];
                 m_prev = m.m_state[(g - 1) & 1][r];
@@ -611,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // running row sum: l(g) = l(g - 1) * alpha(g) + sum of P(g)
             float l_prev = 0.f;
             if (g > 0) {
-                if (!wait_warp_inl(&bb.lsum[(g - 1) % kSBuf][wq], ((g - 1) / kSBuf) & 1, &m.abort, err))
+                if (!wait_warp(&bb.lsum[(g - 1) % kSBuf][wq], ((g - 1) / kSBuf) & 1, &m.abort, err))
                     goto softmax_exit;
                 if (!(flags & 1)) l_prev = m.l_state[(g - 1) & 1][r];
             }
@@ -621,7 +621,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (flags & 2) {
                 // the tile's row sum and offset for the epilogue (ring of two tiles)
                 const int n = n_before;
-                if (!wait_warp_inl(&bb.l_empty[n & 1], ((n >> 1) & 1) ^ 1, &m.abort, err)) goto softmax_exit;
+                if (!wait_warp(&bb.l_empty[n & 1], ((n >> 1) & 1) ^ 1, &m.abort, err)) goto softmax_exit;
                 m.lfin[n & 1][r] = l_run;
                 m.mfin[n & 1][r] = m_run;
                 mbar_arrive(&bb.l_full[n & 1]);
