@@ -66,21 +66,25 @@ __device__ __forceinline__ void cand_insert(int (&co)[kCand], int (&cj)[kCand], 
 }
 
 // CTA = (bh, 32 consecutive rows); warp w handles row i0 + w.  Column
-// bitmaps are staged through shared memory in chunks.
+// bitmaps are staged through shared memory in chunks, each row padded with
+// zero words to ws words (a multiple of 4 with ws / 4 odd), so that the
+// 16-byte loads of 32 lanes reading 32 different rows hit distinct banks in
+// every quarter warp.
 __global__ void __launch_bounds__(1024) plan_cand_kernel(const uint32_t* __restrict__ bits, int32_t* __restrict__ cand,
-                                                         int32_t* __restrict__ cand_ov, int nq, int words,
+                                                         int32_t* __restrict__ cand_ov, int nq, int words, int ws,
                                                          int chunk_rows)
 {
-    extern __shared__ uint32_t sh[];
+    extern __shared__ uint4 sh4[];
+    uint32_t* sh = reinterpret_cast<uint32_t*>(sh4);
     const int rb = (nq + 31) / 32;
     const int bh = blockIdx.x / rb, i0 = (blockIdx.x % rb) * 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t* bbh = bits + (int64_t)bh * nq * words;
-    uint32_t* rows = sh;                        // 32 x words: this CTA's rows
-    uint32_t* cols = sh + 32 * words;           // chunk_rows x words: current column chunk
-    for (int e = threadIdx.x; e < 32 * words; e += blockDim.x) {
-        const int r = e / words, w = e - r * words;
-        rows[e] = i0 + r < nq ? bbh[(int64_t)(i0 + r) * words + w] : 0u;
+    uint32_t* rows = sh;                     // 32 x ws: this CTA's rows
+    uint32_t* cols = sh + 32 * ws;           // chunk_rows x ws: current column chunk
+    for (int e = threadIdx.x; e < 32 * ws; e += blockDim.x) {
+        const int r = e / ws, w = e - r * ws;
+        rows[e] = i0 + r < nq && w < words ? bbh[(int64_t)(i0 + r) * words + w] : 0u;
     }
     const int i = i0 + warp;
     int co[kCand], cj[kCand];
@@ -92,16 +96,22 @@ __global__ void __launch_bounds__(1024) plan_cand_kernel(const uint32_t* __restr
     for (int c0 = 0; c0 < nq; c0 += chunk_rows) {
         const int cn = min(chunk_rows, nq - c0);
         __syncthreads();
-        for (int e = threadIdx.x; e < cn * words; e += blockDim.x) cols[e] = bbh[(int64_t)c0 * words + e];
+        for (int e = threadIdx.x; e < cn * ws; e += blockDim.x) {
+            const int r = e / ws, w = e - r * ws;
+            cols[e] = w < words ? bbh[(int64_t)(c0 + r) * words + w] : 0u;
+        }
         __syncthreads();
         if (i < nq) {
-            const uint32_t* ri = rows + warp * words;
+            const uint4* ri = reinterpret_cast<const uint4*>(rows + warp * ws);
             for (int jj = lane; jj < cn; jj += 32) {
                 const int j = c0 + jj;
                 if (j == i) continue;
-                const uint32_t* rj = cols + jj * words;
+                const uint4* rj = reinterpret_cast<const uint4*>(cols + jj * ws);
                 int ov = 0;
-                for (int w = 0; w < words; ++w) ov += __popc(ri[w] & rj[w]);
+                for (int w = 0; w < ws / 4; ++w) {
+                    const uint4 a = ri[w], b = rj[w];
+                    ov += __popc(a.x & b.x) + __popc(a.y & b.y) + __popc(a.z & b.z) + __popc(a.w & b.w);
+                }
                 cand_insert(co, cj, ov, j);
             }
         }
@@ -252,15 +262,18 @@ cudaError_t launch_plan(const int32_t* topk_idx, int32_t* plan, int B, int H, in
     plan_bits_kernel<<<(unsigned)((lists + warps_per_block - 1) / warps_per_block), 32 * warps_per_block, 0, s>>>(
         topk_idx, bits, (int)lists, nq, topk, words, err);
 
-    // column chunk: up to 32 KiB of bitmaps; plus this CTA's 32 rows
-    int chunk_rows = (32 * 1024) / (words * 4);
+    // padded row stride (a multiple of 4 words, stride / 4 odd); column chunk: up to
+    // 32 KiB of bitmaps, plus this CTA's 32 rows
+    int stride = (words + 3) / 4 * 4;
+    if (((stride / 4) & 1) == 0) stride += 4;
+    int chunk_rows = (32 * 1024) / (stride * 4);
     if (chunk_rows > 512) chunk_rows = 512;
     if (chunk_rows < 1) chunk_rows = 1;
-    const size_t smem_c = (size_t)(32 + chunk_rows) * words * 4;
+    const size_t smem_c = (size_t)(32 + chunk_rows) * stride * 4;
     cudaError_t e = cudaFuncSetAttribute(plan_cand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_c);
     if (e != cudaSuccess) return e;
     const int rb = (nq + 31) / 32;
-    plan_cand_kernel<<<(unsigned)(B * H * rb), 1024, smem_c, s>>>(bits, cand, cand_ov, nq, words, chunk_rows);
+    plan_cand_kernel<<<(unsigned)(B * H * rb), 1024, smem_c, s>>>(bits, cand, cand_ov, nq, words, stride, chunk_rows);
 
     const size_t smem_m = (size_t)2 * nq * 4;
     e = cudaFuncSetAttribute(plan_match_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_m);
