@@ -25,21 +25,21 @@
 // tensor core sees one PV and one QK per softmax step.  Steps run on across
 // tile boundaries; the tile's offsets and sums restart at its first step.
 //
-// Roles (448 threads, one persistent CTA per SM):
-//   warps 0-7   softmax: warp w owns TMEM lanes 32 (w % 4) .. +31 (query rows)
-//               and key half w / 4 (columns 0-63: the step's first KV cube,
-//               64-127: the second).  The two warps of a lane quarter share
-//               each row's step maximum through shared memory, so both halves
-//               use the same offset; each keeps the sum of its own half.
-//   warps 8-11  O correction and epilogue (thread = row): rescale the rows
+// Roles (640 threads, one persistent CTA per SM):
+//   warps 0-11  softmax: warp w owns TMEM lanes 32 (w % 4) .. +31 (query rows,
+//               all 128 columns) and the steps g with g % 3 == w / 4, so each
+//               SMSP runs three softmax warps on three consecutive steps
+//   warps 12-15 O correction and epilogue (thread = row): rescale the rows
 //               whose running offset rose, once the previous PV has finished;
 //               at a tile's end, O / l -> out and the log-sum-exp -> lse
-//   warp 12     TMA producer: builds each tile's step list (shared cubes
-//               first) and streams Q (one buffer), K pairs (ring of 2) and
-//               V pairs (ring of 3)
-//   warp 13     MMA issuer (the whole warp runs the schedule, one elected lane
-//               issues); zeroes V pad rows inside a partial k-step before the
-//               product; owns the TMEM allocation.
+//   warp 16     TMA producer of Q and K: builds each tile's step list (shared
+//               cubes first), streams Q (one buffer) and K pairs (ring of 2)
+//               and posts each step's V pair to warp 18
+//   warp 17     PV MMA issuer (the whole warp runs the schedule, one elected
+//               lane issues); zeroes V pad rows inside a partial k-step before
+//               the product; owns the TMEM allocation
+//   warp 18     TMA producer of V pairs (ring of 3)
+//   warp 19     QK MMA issuer
 //
 // Softmax.  Logits in base 2 (x = s * sm_scale * log2 e).  Keys at or beyond
 // vbs of their cube and cubes the row's query cube did not select are
