@@ -22,8 +22,8 @@
 // for the other cube's rows.  Cubes both lists name are walked first, so a
 // tile whose query cubes select similar cubes (the pairing that vsa_plan
 // chooses) loads each shared K/V cube once for both: the L2->SM traffic of
-// the gather, the binding resource of this operator on B200, drops with the
-// overlap of the paired lists.
+// the gather and the tensor work both drop with the overlap of the paired
+// lists.
 //
 // Each thread of a softmax warp owns one query row (one TMEM lane), so the
 // row maximum and the row sum are thread-local: no cross-lane reduction.
