@@ -387,11 +387,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t acc = o_init ? 1u : 0u;
 #pragma unroll
                 for (int kstep = 0; kstep < 8; ++kstep) {
-                    if (kmask & (1u << kstep)) {
-                        const uint32_t a_col = kstep < 4 ? 8u * kstep : 64u + 8u * (kstep - 4);
-                        umma_ts_elect(o_tmem, p_tmem + a_col, d_hi | (vl + ((kstep * 2048) >> 4)), idesc_pv, acc);
-                        acc = 1u;
-                    }
+                    const uint32_t on = (kmask >> kstep) & 1u;  // warp-uniform, no branch
+                    const uint32_t a_col = kstep < 4 ? 8u * kstep : 64u + 8u * (kstep - 4);
+                    umma_ts_elect_if(o_tmem, p_tmem + a_col, d_hi | (vl + ((kstep * 2048) >> 4)), idesc_pv, acc, on);
+                    acc |= on;
                 }
                 o_init = o_init || kmask != 0;
                 umma_commit_elect(&bb.v_empty[sb]);

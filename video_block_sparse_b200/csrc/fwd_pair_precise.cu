@@ -369,12 +369,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t acc = o_init[x] ? 1u : 0u;
 #pragma unroll
                     for (int kstep = 0; kstep < 8; ++kstep) {
-                        if (kmask & (1u << kstep)) {
-                            const uint64_t bd = d_hi | (vl + ((kstep * 2048) >> 4));
-                            umma_ts_elect(o_tmem, p_tmem + kstep * 8, bd, idesc_pv, acc);
-                            acc = 1u;
-                            if (PRECISE) umma_ts_elect(o_tmem, p_tmem + 64 + kstep * 8, bd, idesc_pv, 1u);
-                        }
+                        const uint32_t on = (kmask >> kstep) & 1u;  // warp-uniform, no branch
+                        const uint64_t bd = d_hi | (vl + ((kstep * 2048) >> 4));
+                        umma_ts_elect_if(o_tmem, p_tmem + kstep * 8, bd, idesc_pv, acc, on);
+                        acc |= on;
+                        if (PRECISE) umma_ts_elect_if(o_tmem, p_tmem + 64 + kstep * 8, bd, idesc_pv, 1u, on);
                     }
                     o_init[x] = o_init[x] || kmask != 0;
                     umma_commit_elect(&m.v_empty[sw_vslot(c)]);
