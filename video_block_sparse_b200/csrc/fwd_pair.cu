@@ -103,7 +103,8 @@ struct Bars {
 
 struct Misc {
     Bars bar;
-    int4 vreq[kVReq];        // V load request: first token of cube a (-1: none), of cube b, head, last
+    int4 vreq[kVReq];        // V load request: first token of cube a (-1: none), of cube b, head, step word
+    uint32_t v_meta[kSBuf];  // step word of the V pair in each V buffer
     uint32_t k_meta[kKBuf];  // step word of the K pair in each K buffer
     uint32_t s_meta[kSBuf];  // step word of each S buffer
     uint32_t tmem_base;
@@ -266,8 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // the step's V pair, for the V producer
                     if (!aborted && wait_bar(&bb.vr_empty[vr], ((kc / kVReq) & 1) ^ 1, &m.abort, err)) {
                         m.vreq[vr] = make_int4(meta.na > 0 ? tok0 + 64 * meta.ja : -1,
-                                               meta.nb > 0 ? tok0 + 64 * meta.jb : -1, t.h,
-                                               (word & kFinal) ? 1 : 0);
+                                               meta.nb > 0 ? tok0 + 64 * meta.jb : -1, t.h, (int)word);
                         mbar_arrive(&bb.vr_full[vr]);
                     } else {
                         aborted = true;
@@ -293,13 +293,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&bb.vr_empty[vr]);
             // the V buffer is free once the PV three steps back finished
             if (!wait_bar(&bb.v_empty[vb], ((vc / kSBuf) & 1) ^ 1, &m.abort, err)) break;
+            m.v_meta[vb] = (uint32_t)rq.w;  // published by the arrival below
             mbar_expect_tx(&bb.v_full[vb], 2 * kHalfBox * ((rq.x >= 0) + (rq.y >= 0)));
             armed_v = (vc / kSBuf) & 1;
             armed_vb = vb;
             uint8_t* vdst = tiles_ptr + L::V_OFF + vb * kTileBytes;
             if (rq.x >= 0) load_cube(&tmv, &bb.v_full[vb], vdst, 0, rq.z, rq.x);
             if (rq.y >= 0) load_cube(&tmv, &bb.v_full[vb], vdst, 1, rq.z, rq.y);
-            if (rq.w) break;  // the CTA's last step
+            if ((uint32_t)rq.w & kFinal) break;  // the CTA's last step
         }
         if (lane == 0 && armed_v >= 0 && aborted_flag(&m.abort)) drain_wait(&bb.v_full[armed_vb], armed_v);
         __syncwarp();
@@ -335,12 +336,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     aborted = true;
                     break;
                 }
-                __syncwarp();
-                if (lane == 0) {
-                    m.s_meta[sb] = meta;
-                    mbar_arrive(&bb.s_full[sb]);  // publishes the step word (release)
-                }
-                __syncwarp();
+                m.s_meta[sb] = meta;                // every lane stores the same word
+                mbar_arrive_elect(&bb.s_full[sb]);  // publishes it (release)
                 tc_fence_after();
                 const uint32_t kl = kl0 + ((uint32_t)kb * kTileBytes >> 4);
 #pragma unroll
@@ -350,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 umma_commit_elect(&bb.s_full[sb]);
                 umma_commit_elect(&bb.k_empty[kb]);
-                if (sw_flags(meta) & 2) umma_commit_elect(&bb.q_empty);
+                umma_commit_elect_if(&bb.q_empty, sw_flags(meta) & 2);
                 if (meta & kFinal) break;
             }
         } else {
@@ -361,8 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int sb = j % kSBuf;
                 const uint32_t par = (j / kSBuf) & 1;
                 if (!wait_warp(&bb.v_full[sb], par, &m.abort, err)) { aborted = true; break; }
-                if (!wait_warp(&bb.p_full[sb], par, &m.abort, err)) { aborted = true; break; }
-                const uint32_t meta = m.s_meta[sb];
+                // everything that needs only the V pair is done before waiting for P
+                const uint32_t meta = m.v_meta[sb];
                 const int na = sw_na(meta), nb = sw_nb(meta);
                 const uint32_t vl = vl0 + ((uint32_t)sb * kTileBytes >> 4);
                 const int za = (na & 15) ? 16 - (na & 15) : 0, zb = (nb & 15) ? 16 - (nb & 15) : 0;
@@ -378,6 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     fence_proxy_async_smem();
                     __syncwarp();
                 }
+                if (!wait_warp(&bb.p_full[sb], par, &m.abort, err)) { aborted = true; break; }
                 tc_fence_after();
                 // k-steps (16 keys) 0..ceil16(na)-1 of half 0 and 4..4+ceil16(nb)-1 of half 1; the
                 // bf16 P of key half h sits in the first 32 columns of that half's 64
@@ -393,13 +391,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     acc |= on;
                 }
                 o_init = o_init || kmask != 0;
+                // PV(j) is in the tensor core's queue: S buffer sb may be written again (the
+                // QK issuer's products go after it; the commits below track this warp's only)
+                tc_fence_before();
+                mbar_arrive_elect(&bb.pv_issued[sb]);
                 umma_commit_elect(&bb.v_empty[sb]);
                 umma_commit_elect(&bb.pv_done[j & 1]);
-                if (sw_flags(meta) & 2) umma_commit_elect(&bb.o_full);
-                // PV(j) is in the tensor core's queue: S buffer sb may be written again
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bb.pv_issued[sb]);
+                umma_commit_elect_if(&bb.o_full, sw_flags(meta) & 2);
                 if (meta & kFinal) break;
             }
         }

@@ -164,6 +164,29 @@ __device__ __forceinline__ void umma_commit_elect(uint64_t* bar)
         : "memory");
 }
 
+// Commit issued by one elected lane only when `issue` is nonzero (no branch).
+__device__ __forceinline__ void umma_commit_elect_if(uint64_t* bar, uint32_t issue)
+{
+    asm volatile(
+        "{\n\t.reg .pred e, q;\n\t"
+        "setp.ne.b32 q, %1, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "and.pred e, e, q;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar)),
+        "r"(issue)
+        : "memory");
+}
+
+// mbarrier arrival by one elected lane of a converged warp (no branch).
+__device__ __forceinline__ void mbar_arrive_elect(uint64_t* bar)
+{
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}" ::"r"(smem_u32(bar))
+        : "memory");
+}
+
 // Packed pair arithmetic (one instruction for two fp32 lanes on sm_100).
 __device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0, float c1)
 {
