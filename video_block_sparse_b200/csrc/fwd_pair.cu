@@ -149,7 +149,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tiles = (raw_addr + L::MISC_BYTES + 1023u) & ~1023u;  // 1 KiB aligned for 128B swizzle
     uint8_t* tiles_ptr = smem_raw + (tiles - raw_addr);
 
-    const int warp = threadIdx.x >> 5;
+    // Values that are the same in every lane (the warp index, a step word read from
+    // shared memory) go through a shuffle from lane 0: the compiler then knows them
+    // to be warp-uniform, and branches on them need no divergence handling around
+    // the warp-collective tcgen05 loads and stores they contain (Wan 832x480 forward
+    // 4.75 -> 4.67 ms).
+    const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0);
     const uint32_t lane = threadIdx.x & 31;
     const int my_tiles = n_tiles > (int)blockIdx.x ? (n_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
@@ -418,7 +423,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int b = g % kSBuf;
                 if (!wait_warp(&bb.a_full[b], (g / kSBuf) & 1, &m.abort, err)) goto corr_exit;
                 const uint32_t meta = m.s_meta[b];
-                if (!(sw_flags(meta) & 1) && m.rflag[b][wq] != 0) {
+                const int rescale = __shfl_sync(0xffffffffu, !(sw_flags(meta) & 1) && m.rflag[b][wq] != 0, 0);
+                if (rescale) {
                     // O row r *= alpha (1 for rows whose offset stayed), once the
                     // previous step's PV has finished
                     const int jp = g - 1;
@@ -496,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // so a barrier is never two phases behind its waiter.
         const int wq = warp & 3, par = warp >> 2;
         const int r = 32 * wq + (int)lane;  // query row of the tile == TMEM lane
-        const int qbit = r >> 6;            // 0: query cube i1, 1: i2
+        const int qbit = wq >> 1;           // 0: query cube i1, 1: i2 (rows r >> 6)
         const uint32_t lane_base = tbase + ((uint32_t)(32 * wq) << 16);
         constexpr float kNeutral = NEG ? INFINITY : -INFINITY;  // a masked logit
         for (int g = par;; g += kSBuf) {
@@ -507,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (my_tiles == 0) break;
             if (!wait_warp(&bb.s_full[b], spar, &m.abort, err)) goto softmax_exit;
             if (g > *reinterpret_cast<volatile int*>(&m.end_g)) break;  // past the CTA's last step
-            const uint32_t meta = m.s_meta[b];
+            const uint32_t meta = __shfl_sync(0xffffffffu, m.s_meta[b], 0);  // warp-uniform
             tc_fence_after();
             const int na = sw_na(meta), nb = sw_nb(meta), flags = sw_flags(meta);
             const int nv0 = ((sw_ma(meta) >> qbit) & 1) ? na : 0;  // valid keys of each half
