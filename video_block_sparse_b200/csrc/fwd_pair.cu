@@ -18,8 +18,8 @@
 // both; vsa_plan pairs query cubes whose lists overlap most.
 //
 // Pipeline.  TMEM holds three S/P buffers (columns 0, 128, 256) and O
-// (columns 384-511).  Step g uses buffer g % 3, and the MMA issuer runs the
-// products in the order  ..., PV(g), QK(g + 3), PV(g + 1), QK(g + 4), ...
+// (columns 384-511).  Step g uses buffer g % 3, and the two MMA issuers run
+// the products in the order  ..., PV(g), QK(g + 3), PV(g + 1), QK(g + 4), ...
 // so the logits of the next two steps are ready while the softmax of step g
 // runs; the softmax, not the QK -> softmax -> PV chain, sets the pace, and the
 // tensor core sees one PV and one QK per softmax step.  Steps run on across
@@ -317,8 +317,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // its next group, so the groups reach the tensor core back to back.  The
         // order QK(j) after PV(j - 3) (they share S buffer j % 3) is kept by
         // barrier pv_issued: the PV warp arrives after issuing PV(j) (after a
-        // tcgen05 before-fence), the QK warp waits for it before QK(j + 3).
-        // In each warp the whole warp runs the schedule and one elected lane issues.
+        // tcgen05 before-fence), the QK warp waits for it before QK(j + 3).  In each
+        // warp the whole warp runs the schedule and one elected lane issues, with no
+        // branch around an elect: conditions go into the issue predicate.
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);
         // operand descriptors built once; a k-step adds its byte offset / 16
