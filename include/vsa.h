@@ -262,6 +262,17 @@ VSA_API int vsa_untile(const vsa_bf16 *x_tiled, vsa_bf16 *x_grid, int B, int T, 
                cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Diagnostic of the pipeline's failure handling.  Launches one warp that
+ * runs the forward kernels' bounded mbarrier wait on a barrier nothing ever
+ * completes: the wait gives up after ~2 s of GPU clock, latches code 3 in
+ * the device error word (read it with vsa_device_status) and returns, and
+ * the kernel exits normally.  `result` is a device int: bit 0 = the wait
+ * reported success (never expected), bit 1 = the abort flag was raised.
+ * Returns VSA_ERR_NULL or VSA_ERR_LAUNCH on failure to launch, else VSA_OK.
+ * ---------------------------------------------------------------------- */
+VSA_API int vsa_stall_check(int *result, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * Device error word.  Synchronises `stream`, returns VSA_OK or
  * VSA_ERR_DEVICE (and clears the word), or VSA_ERR_LAUNCH if the stream
  * reports a CUDA error.  `detail` (may be NULL) receives the latched code:

@@ -97,6 +97,10 @@ def test_fwd_rejects_null_and_misaligned_without_a_device(vsa):
     assert vsa.get_lib().vsa_fwd_ex(p, p, p, p, p, p, None, 1, 512, 2, 128, 8, 2, 0.1, 8, None) == -1  # unknown flag
 
 
+def test_stall_check_rejects_null_without_a_device(vsa):
+    assert vsa.get_lib().vsa_stall_check(None, None) == -2
+
+
 def test_route_rejects_bad_arguments_without_a_device(vsa):
     p = _fake(1 << 20)
     ws = vsa.route_workspace_size(1, 2, 8, 128)

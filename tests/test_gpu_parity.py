@@ -258,6 +258,24 @@ def test_fwd_bad_index_latches_device_error(vsa):
     assert rc == -7 and detail == 2
 
 
+def test_stalled_pipeline_wait_ends_with_error_status(vsa):
+    """A bounded pipeline wait that nothing completes gives up (~2 s of clock),
+    latches code 3, raises the abort flag and returns; the context stays usable."""
+    import time
+
+    assert vsa.device_status() == (0, 0)
+    t0 = time.perf_counter()
+    bits = vsa.stall_check()
+    elapsed = time.perf_counter() - t0
+    assert bits == 2  # the wait reported failure and raised the abort flag
+    assert vsa.device_status() == (-7, 3)
+    assert 0.2 < elapsed < 60.0
+    p = _small(16, nq=4, H=1, topk=2, vbs=[64, 40, 64, 9])
+    out, lse = _run_fwd(vsa, p)
+    _check_items(p, out, lse, oracle.all_items(1, 1, 4), "after-stall", precise=False)
+    assert vsa.device_status() == (0, 0)
+
+
 def test_fwd_rejects_bad_calls(vsa):
     p = _small(15, nq=4, H=1, topk=2)
     q, k, v = common.dev(p.qt), common.dev(p.kt), common.dev(p.vt)

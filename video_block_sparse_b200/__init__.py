@@ -63,9 +63,10 @@ def _load():
     lib.vsa_tile.argtypes = [P, P, I, I, I, I, I, I, P]
     lib.vsa_untile.argtypes = [P, P, I, I, I, I, I, I, P]
     lib.vsa_device_status.argtypes = [P, P]
+    lib.vsa_stall_check.argtypes = [P, P]
     for name in ("vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_fwd_planned", "vsa_plan", "vsa_route", "vsa_route_noalloc", "vsa_cube_counts",
                  "vsa_tile",
-                 "vsa_untile", "vsa_device_status"):
+                 "vsa_untile", "vsa_device_status", "vsa_stall_check"):
         getattr(lib, name).restype = I
     return lib
 
@@ -232,6 +233,17 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk_idx: torch.Tenso
                                          _ptr(lse), B, S, H, D, nq, topk, float(sm_scale), int(flags),
                                          _stream(stream)), "vsa_fwd_planned")
     return (out, lse) if (want_lse or lse is not None) else out
+
+
+def stall_check(stream=None) -> int:
+    """Run the bounded-wait diagnostic (a wait that nothing completes must run out,
+    latch error 3 and return); returns its result bits (bit 0: the wait succeeded,
+    bit 1: the abort flag was raised) after the stream has finished."""
+    result = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rc = get_lib().vsa_stall_check(_ptr(result), _stream(stream))
+    if rc != 0:
+        raise RuntimeError(f"vsa_stall_check: {status_string(rc)}")
+    return int(result.item())
 
 
 def device_status(stream=None) -> tuple[int, int]:

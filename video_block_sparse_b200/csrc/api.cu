@@ -246,6 +246,15 @@ int vsa_untile(const vsa_bf16* x_tiled, vsa_bf16* x_grid, int B, int T, int Hh, 
     return launch_status(vsa::launch_untile(x_tiled, x_grid, B, vsa::make_geom(T, Hh, W), H * D, stream));
 }
 
+int vsa_stall_check(int* result, cudaStream_t stream)
+{
+    if (result == nullptr) return VSA_ERR_NULL;
+    int* err;
+    const int rc = device_error_word(&err);
+    if (rc != VSA_OK) return rc;
+    return launch_status(vsa::launch_stall_check(err, result, stream));
+}
+
 int vsa_device_status(cudaStream_t stream, int* detail)
 {
     if (detail) *detail = 0;

@@ -59,6 +59,7 @@ cudaError_t launch_fwd_pair(const uint16_t* q, const uint16_t* k, const uint16_t
 
 // ---- plan.cu (pairing of query cubes by selection overlap)
 size_t plan_workspace_bytes(int B, int H, int nq);
+cudaError_t launch_stall_check(int* err, int* result, cudaStream_t s);
 cudaError_t launch_plan(const int32_t* topk_idx, int32_t* plan, int B, int H, int nq, int topk, void* workspace,
                         int* err, cudaStream_t s);
 
