@@ -23,6 +23,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -65,7 +66,9 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        # the raw samples (the JSON line carries their summary); VSA_CLOCK_DIR picks the folder
+        folder = os.environ.get("VSA_CLOCK_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(folder, f"vsa_clocks_rank{index}.csv")
 
     def __enter__(self):
         os.makedirs(os.path.dirname(self.path), exist_ok=True)
