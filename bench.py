@@ -114,6 +114,29 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# --------------------------------------------------------------------------- ranks
+
+def problem_config(rank: int, heads: int = 0):
+    """The workload of one rank: an independent seeded problem per rank (weak scaling);
+    `heads` overrides the head count (a reduced case for profiler captures only)."""
+    import dataclasses
+
+    cfg = dataclasses.replace(synth.CONFIGS[WORKLOAD], seed=rank)
+    if heads:
+        cfg = dataclasses.replace(cfg, H=heads)
+    return cfg
+
+
+def max_over_ranks(values, device) -> list[float]:
+    """Every rank's timings -> their maximum over ranks, on every rank (one all-reduce
+    when a process group of more than one rank is up; the values unchanged otherwise)."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist = torch.distributed
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
 # --------------------------------------------------------------------------- GPU arm
 
 def run_gpu(args, rank, world, local_rank):
@@ -121,12 +144,7 @@ def run_gpu(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    cfg = synth.CONFIGS[WORKLOAD]
-    import dataclasses
-
-    cfg = dataclasses.replace(cfg, seed=rank)  # an independent problem per rank
-    if args.heads:
-        cfg = dataclasses.replace(cfg, H=args.heads)  # a reduced case for profiler captures only
+    cfg = problem_config(rank, args.heads)
     T, Hh, W = cfg.grid
     vbs_h = vsa.cube_counts(T, Hh, W)
     nq = len(vbs_h)
@@ -263,10 +281,8 @@ def run_gpu(args, rank, world, local_rank):
         raise RuntimeError("pipelined end-to-end result differs from the device-timed step's result")
 
     ms_step = ms_total / args.steps
-    t = torch.tensor([ms_step, e2e_ms, statistics.mean(fwd_ms), e2e_serial_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms_step, e2e_ms, fwd_avg, e2e_serial_ms = (float(x) for x in t.tolist())
+    ms_step, e2e_ms, fwd_avg, e2e_serial_ms = max_over_ranks(
+        [ms_step, e2e_ms, statistics.mean(fwd_ms), e2e_serial_ms], dev)
     return dict(cfg=cfg, S=S, ms_step=ms_step, e2e_ms=e2e_ms, e2e_serial_ms=e2e_serial_ms, fwd_ms=fwd_avg,
                 fwd_list=fwd_ms,
                 clocks=clk.summary(), launches=launches_per_step * args.steps,
