@@ -365,9 +365,13 @@ int oracle_fwd_items(const uint16_t *q, const uint16_t *k, const uint16_t *v,
  * bit.  For each (b, h): overlap(i, j) = number of distinct cubes that both
  * lists name; each cube's candidates are the 8 cubes j != i with the largest
  * overlap (ties: smaller j); rounds: each unpaired cube proposes to its first
- * unpaired candidate, mutual proposals pair, until a round pairs none;
- * leftovers pair in index order; tiles are listed by smaller index as
- * (smaller, larger) or (i, -1).  plan is [B*H][ceil(Nq/2)][2]. */
+ * unpaired candidate, mutual proposals pair, until a round pairs none (at
+ * most 64 rounds).  Refills: while two or more cubes are unpaired, each
+ * unpaired cube's candidates become the 8 unpaired cubes j != i with the
+ * largest overlap (same ties) and the rounds run again; stop when a refill
+ * pairs none (at most 64 refills).  Leftovers pair in index order; tiles
+ * are listed by smaller index as (smaller, larger) or (i, -1).
+ * plan is [B*H][ceil(Nq/2)][2]. */
 int oracle_plan(const int32_t *topk_idx, int B, int H, int Nq, int topk, int32_t *plan)
 {
     if (B <= 0 || H <= 0 || Nq <= 0 || topk < 1) return ORACLE_ERR_ARG;
@@ -398,40 +402,51 @@ int oracle_plan(const int32_t *topk_idx, int B, int H, int Nq, int topk, int32_t
                 if (member[(size_t)j * Nq + c]) dist[(size_t)j * ndist_max + n++] = c;
             ndist[j] = n;
         }
-        for (int i = 0; i < Nq; ++i) {
-            int best_ov[8], best_j[8];
-            for (int c = 0; c < NC; ++c) { best_ov[c] = -1; best_j[c] = -1; }
-            for (int j = 0; j < Nq; ++j) {
-                if (j == i) continue;
-                int ov = 0;
-                for (int e = 0; e < ndist[j]; ++e) ov += member[(size_t)i * Nq + dist[(size_t)j * ndist_max + e]];
-                /* j ascends, so a later j with an equal overlap never displaces an earlier one */
-                int pos = NC;
-                while (pos > 0 && ov > best_ov[pos - 1]) --pos;
-                if (pos < NC) {
-                    for (int c = NC - 1; c > pos; --c) { best_ov[c] = best_ov[c - 1]; best_j[c] = best_j[c - 1]; }
-                    best_ov[pos] = ov;
-                    best_j[pos] = j;
-                }
-            }
-            for (int c = 0; c < NC; ++c) cand[i * NC + c] = best_j[c];
-        }
         for (int i = 0; i < Nq; ++i) partner[i] = -1;
-        for (int round = 0; round < 64; ++round) {
+        /* refill 0 computes every cube's candidates among all cubes; refill r > 0
+           recomputes those of the unpaired cubes among the unpaired cubes */
+        for (int refill = 0; refill <= 64; ++refill) {
+            int unpaired = 0;
+            for (int i = 0; i < Nq; ++i) unpaired += partner[i] < 0;
+            if (refill > 0 && unpaired < 2) break;
             for (int i = 0; i < Nq; ++i) {
-                prop[i] = -1;
                 if (partner[i] >= 0) continue;
-                for (int c = 0; c < NC; ++c) {
-                    int j = cand[i * NC + c];
-                    if (j >= 0 && partner[j] < 0) { prop[i] = j; break; }
+                int best_ov[8], best_j[8];
+                for (int c = 0; c < NC; ++c) { best_ov[c] = -1; best_j[c] = -1; }
+                for (int j = 0; j < Nq; ++j) {
+                    if (j == i || partner[j] >= 0) continue;
+                    int ov = 0;
+                    for (int e = 0; e < ndist[j]; ++e) ov += member[(size_t)i * Nq + dist[(size_t)j * ndist_max + e]];
+                    /* j ascends, so a later j with an equal overlap never displaces an earlier one */
+                    int pos = NC;
+                    while (pos > 0 && ov > best_ov[pos - 1]) --pos;
+                    if (pos < NC) {
+                        for (int c = NC - 1; c > pos; --c) { best_ov[c] = best_ov[c - 1]; best_j[c] = best_j[c - 1]; }
+                        best_ov[pos] = ov;
+                        best_j[pos] = j;
+                    }
                 }
+                for (int c = 0; c < NC; ++c) cand[i * NC + c] = best_j[c];
             }
-            int changed = 0;
-            for (int i = 0; i < Nq; ++i) {
-                int j = prop[i];
-                if (j >= 0 && prop[j] == i) { partner[i] = j; changed = 1; }
+            int paired_any = 0;
+            for (int round = 0; round < 64; ++round) {
+                for (int i = 0; i < Nq; ++i) {
+                    prop[i] = -1;
+                    if (partner[i] >= 0) continue;
+                    for (int c = 0; c < NC; ++c) {
+                        int j = cand[i * NC + c];
+                        if (j >= 0 && partner[j] < 0) { prop[i] = j; break; }
+                    }
+                }
+                int changed = 0;
+                for (int i = 0; i < Nq; ++i) {
+                    int j = prop[i];
+                    if (j >= 0 && prop[j] == i) { partner[i] = j; changed = 1; }
+                }
+                if (!changed) break;
+                paired_any = 1;
             }
-            if (!changed) break;
+            if (!paired_any) break;
         }
         int pending = -1, odd = -1;
         for (int i = 0; i < Nq; ++i) {

@@ -434,6 +434,27 @@ def test_plan_hand_example(oracle_lib):
     assert oracle_lib.plan(idx).tolist() == [[[0, 2], [1, 3], [4, -1]]]
 
 
+def test_plan_refills_candidates_of_leftovers(oracle_lib):
+    """Sixteen hubs in eight twin pairs (lists: the core cubes 0-7 plus one cube
+    of their own) and four cubes 16-19 that each hold two core cubes and one
+    shared cube: 16 and 18 share cube 16, 17 and 19 share cube 17.  Every hub
+    overlaps a leftover cube by 2 and its twin by 9, so round 1 pairs the twins
+    and the four others, whose 8 candidates are all hubs, are left unpaired.
+    The refill recomputes their candidates among themselves and pairs them by
+    overlap, (16, 18) and (17, 19), not in index order (16, 17), (18, 19)."""
+    nq, topk = 20, 10
+    idx = np.empty((1, 1, nq, topk), np.int32)
+    core = list(range(8))
+    for h in range(16):
+        lst = core + [8 + h // 2]
+        idx[0, 0, h] = lst + lst[:topk - len(lst)]  # duplicates are ignored
+    for c, own in ((16, [0, 1, 16]), (17, [4, 5, 17]), (18, [2, 3, 16]), (19, [6, 7, 17])):
+        idx[0, 0, c] = (own * topk)[:topk]
+    plan = oracle_lib.plan(idx)
+    _check_pairing(plan, nq)
+    assert plan[0].tolist() == [[2 * p, 2 * p + 1] for p in range(8)] + [[16, 18], [17, 19]]
+
+
 def test_plan_pairs_planted_twins(oracle_lib):
     """Cubes planted in pairs with identical lists (and lists that share
     nothing across pairs) are paired with their twin, whatever their order."""

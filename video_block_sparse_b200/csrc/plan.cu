@@ -13,6 +13,12 @@
 //   3. match  : rounds of mutual proposals: every unpaired cube proposes to
 //               its first still-unpaired candidate; two cubes that propose
 //               to each other are paired.  Rounds repeat until none pairs.
+//               Refills: while two or more cubes are unpaired, their
+//               candidates are recomputed among the unpaired cubes (same
+//               rule) and the rounds run again, until a refill pairs none.
+//               Without the refills ~55 of 624 cubes per head at Wan 832x480
+//               ended up paired in index order, whatever their overlap, and
+//               the CTAs that drew those tiles set the forward's end.
 //               Cubes left over are paired in index order (the last one
 //               alone if their number is odd).  Tiles are emitted in order
 //               of their smaller cube index, as (smaller, larger) or (i, -1).
@@ -29,6 +35,7 @@ namespace {
 
 constexpr int kCand = 8;
 constexpr int kMaxRounds = 64;
+constexpr int kMaxRefills = 64;
 
 // One warp per (bh, i) list: clear the bitmap row, then set the listed bits.
 __global__ void plan_bits_kernel(const int32_t* __restrict__ topk_idx, uint32_t* __restrict__ bits, int n_lists,
@@ -151,45 +158,85 @@ __global__ void __launch_bounds__(1024) plan_cand_kernel(const uint32_t* __restr
     }
 }
 
-// One CTA per (bh): proposal rounds over the candidate lists, leftovers in
-// index order, then the tiles in order of their smaller cube.
-__global__ void __launch_bounds__(1024) plan_match_kernel(const int32_t* __restrict__ cand, int32_t* __restrict__ plan,
-                                                          int nq)
+// One CTA per (bh): proposal rounds over the candidate lists; refills while
+// two or more cubes are unpaired (their candidates recomputed among the
+// unpaired cubes, then the rounds again); leftovers in index order; then the
+// tiles in order of their smaller cube.
+__global__ void __launch_bounds__(1024) plan_match_kernel(int32_t* cand, const uint32_t* __restrict__ bits,
+                                                          int32_t* __restrict__ plan, int nq, int words)
 {
     extern __shared__ int32_t smi[];
     int32_t* partner = smi;       // nq: paired cube, -1 unpaired
     int32_t* prop = smi + nq;     // nq: this round's proposal
-    __shared__ int changed;
+    __shared__ int n_unpaired;
     __shared__ int nleft;
     const int bh = blockIdx.x;
-    const int32_t* cb = cand + (int64_t)bh * nq * kCand;
+    // candidate lists: written by plan_cand_kernel, rewritten here by the refills
+    // (plain loads: the read-only path must not serve them)
+    int32_t* cb = cand + (int64_t)bh * nq * kCand;
+    const uint32_t* bbh = bits + (int64_t)bh * nq * words;
     for (int i = threadIdx.x; i < nq; i += blockDim.x) partner[i] = -1;
     __syncthreads();
-    for (int round = 0; round < kMaxRounds; ++round) {
-        for (int i = threadIdx.x; i < nq; i += blockDim.x) {
-            int p = -1;
-            if (partner[i] < 0) {
+    for (int refill = 0; refill <= kMaxRefills; ++refill) {
+        if (refill > 0) {
+            int mine = 0;
+            for (int i = threadIdx.x; i < nq; i += blockDim.x) mine += partner[i] < 0 ? 1 : 0;
+            if (threadIdx.x == 0) n_unpaired = 0;
+            __syncthreads();
+            if (mine > 0) atomicAdd(&n_unpaired, mine);
+            __syncthreads();
+            if (n_unpaired < 2) break;  // the same value in every thread
+            // each unpaired cube's kCand candidates among the unpaired cubes
+            // (largest overlap first, ties by the smaller index, as plan_cand_kernel)
+            for (int i = threadIdx.x; i < nq; i += blockDim.x) {
+                if (partner[i] >= 0) continue;
+                int co[kCand], cj[kCand];
+#pragma unroll
                 for (int c = 0; c < kCand; ++c) {
-                    const int j = cb[(int64_t)i * kCand + c];
-                    if (j >= 0 && partner[j] < 0) {
-                        p = j;
-                        break;
+                    co[c] = -1;
+                    cj[c] = 0x7fffffff;
+                }
+                const uint32_t* bi = bbh + (int64_t)i * words;
+                for (int j = 0; j < nq; ++j) {
+                    if (j == i || partner[j] >= 0) continue;
+                    const uint32_t* bj = bbh + (int64_t)j * words;
+                    int ov = 0;
+                    for (int w = 0; w < words; ++w) ov += __popc(__ldg(bi + w) & __ldg(bj + w));
+                    cand_insert(co, cj, ov, j);
+                }
+#pragma unroll
+                for (int c = 0; c < kCand; ++c) cb[(int64_t)i * kCand + c] = co[c] >= 0 ? cj[c] : -1;
+            }
+            __syncthreads();
+        }
+        bool paired_any = false;
+        for (int round = 0; round < kMaxRounds; ++round) {
+            for (int i = threadIdx.x; i < nq; i += blockDim.x) {
+                int p = -1;
+                if (partner[i] < 0) {
+                    for (int c = 0; c < kCand; ++c) {
+                        const int j = cb[(int64_t)i * kCand + c];
+                        if (j >= 0 && partner[j] < 0) {
+                            p = j;
+                            break;
+                        }
                     }
                 }
+                prop[i] = p;
             }
-            prop[i] = p;
-        }
-        if (threadIdx.x == 0) changed = 0;
-        __syncthreads();
-        for (int i = threadIdx.x; i < nq; i += blockDim.x) {
-            const int j = prop[i];
-            if (j >= 0 && prop[j] == i) {
-                partner[i] = j;  // the mirror thread sets partner[j]
-                changed = 1;
+            __syncthreads();
+            int mine = 0;
+            for (int i = threadIdx.x; i < nq; i += blockDim.x) {
+                const int j = prop[i];
+                if (j >= 0 && prop[j] == i) {
+                    partner[i] = j;  // the mirror thread sets partner[j]
+                    mine = 1;
+                }
             }
+            if (!__syncthreads_or(mine)) break;  // a barrier too: the next round reads partner
+            paired_any = true;
         }
-        __syncthreads();
-        if (!changed) break;
+        if (!paired_any) break;  // the same in every thread
     }
     // leftovers: pair in index order (one warp, ballot-based)
     if (threadIdx.x < 32) {
@@ -278,7 +325,7 @@ cudaError_t launch_plan(const int32_t* topk_idx, int32_t* plan, int B, int H, in
     const size_t smem_m = (size_t)2 * nq * 4;
     e = cudaFuncSetAttribute(plan_match_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_m);
     if (e != cudaSuccess) return e;
-    plan_match_kernel<<<(unsigned)(B * H), 1024, smem_m, s>>>(cand, plan, nq);
+    plan_match_kernel<<<(unsigned)(B * H), 1024, smem_m, s>>>(cand, bits, plan, nq, words);
     return cudaGetLastError();
 }
 
