@@ -239,10 +239,13 @@ def stall_check(stream=None) -> int:
     """Run the bounded-wait diagnostic (a wait that nothing completes must run out,
     latch error 3 and return); returns its result bits (bit 0: the wait succeeded,
     bit 1: the abort flag was raised) after the stream has finished."""
+    s = stream if stream is not None else torch.cuda.current_stream()
     result = torch.zeros(1, dtype=torch.int32, device="cuda")
-    rc = get_lib().vsa_stall_check(_ptr(result), _stream(stream))
+    s.wait_stream(torch.cuda.current_stream())  # the zeroed result is ready on s
+    rc = get_lib().vsa_stall_check(_ptr(result), _stream(s))
     if rc != 0:
         raise RuntimeError(f"vsa_stall_check: {status_string(rc)}")
+    s.synchronize()
     return int(result.item())
 
 
