@@ -241,7 +241,8 @@ def stall_check(stream=None) -> int:
     bit 1: the abort flag was raised) after the stream has finished."""
     s = stream if stream is not None else torch.cuda.current_stream()
     result = torch.zeros(1, dtype=torch.int32, device="cuda")
-    s.wait_stream(torch.cuda.current_stream())  # the zeroed result is ready on s
+    if stream is not None:
+        s.wait_stream(torch.cuda.current_stream())  # the zeroed result is ready on s
     rc = get_lib().vsa_stall_check(_ptr(result), _stream(s))
     if rc != 0:
         raise RuntimeError(f"vsa_stall_check: {status_string(rc)}")
