@@ -487,6 +487,54 @@ def test_plan_is_a_pairing_and_beats_index_order(oracle_lib, nq, topk, seed):
         assert planned >= ordered
 
 
+def _plan_restated(lists, nq, ncand=8, rounds=64, refills=64):
+    """The pairing rule as stated (proposal rounds over the ncand best candidates,
+    refills among the unpaired cubes, leftovers in index order), written from the
+    statement with sets and an overlap matrix."""
+    sets = [set(int(x) for x in row if 0 <= x < nq) for row in lists]
+    ov = np.array([[len(a & b) for b in sets] for a in sets])
+    partner = [-1] * nq
+    for refill in range(refills + 1):
+        free = [i for i in range(nq) if partner[i] < 0]
+        if refill > 0 and len(free) < 2:
+            break
+        cand = {}
+        for i in free:
+            others = [j for j in free if j != i]
+            cand[i] = sorted(others, key=lambda j: (-ov[i, j], j))[:ncand]
+        formed = False
+        for _ in range(rounds):
+            prop = {i: next((j for j in cand[i] if partner[j] < 0), -1) for i in range(nq) if partner[i] < 0}
+            pairs = [(i, j) for i, j in prop.items() if j >= 0 and prop.get(j) == i and i < j]
+            if not pairs:
+                break
+            for i, j in pairs:
+                partner[i], partner[j] = j, i
+            formed = True
+        if not formed:
+            break
+    left = [i for i in range(nq) if partner[i] < 0]
+    for a in range(0, len(left) - 1, 2):
+        partner[left[a]], partner[left[a + 1]] = left[a + 1], left[a]
+    odd = left[-1] if len(left) % 2 else -1
+    return [[i, -1 if i == odd else partner[i]] for i in range(nq) if partner[i] > i or i == odd]
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_plan_matches_the_restated_rule(oracle_lib, seed):
+    """Random lists (with duplicates and out-of-range ids half the time): the
+    oracle's plan equals the rule restated with sets."""
+    g = np.random.default_rng(500 + seed)
+    nq = int(g.integers(2, 48))
+    topk = int(g.integers(1, min(9, nq) + 1))
+    idx = synth.random_topk(500 + seed, 1, 2, nq, topk, distinct=bool(seed % 2))
+    if seed % 3 == 0:
+        idx[0, 0, 0, 0] = nq + 3  # ignored by the rule
+    plan = oracle_lib.plan(idx).tolist()
+    for bh in range(2):
+        assert plan[bh] == _plan_restated(idx[0, bh], nq)
+
+
 def test_plan_ignores_duplicates_and_bad_ids(oracle_lib):
     """Overlaps count distinct cubes; ids outside [0, Nq) are ignored."""
     idx = np.array([[[[1, 1, 2], [1, 2, 9], [3, 3, 3], [-1, 3, 0]]]], np.int32)
