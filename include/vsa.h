@@ -77,6 +77,21 @@ VSA_API int vsa_can_implement(int D, int sm_version);
  * gets out = 0 and lse = -inf.  K/V slots at or beyond vbs[c] are never
  * read into the result, even if they hold NaN or Inf.
  *
+ * Numerics (default mode): logits and the P.V product accumulate in fp32;
+ * each softmax weight enters the P.V product rounded to bf16 and the row
+ * sum adds the same rounded weights, so out is a softmax-weighted mean of
+ * the selected v rows with each weight off by at most 2^-9 of itself, then
+ * rounded to bf16; lse is the log of that same row sum (within 2e-3 of
+ * exact, plus the fp32 logit error).  VSA_FWD_PRECISE_P tightens both.
+ *
+ * Real (non-pad) V rows must be finite: two query cubes share a tile, and a
+ * KV cube that only one of them selects enters the other's P.V product with
+ * weight exactly 0, so an Inf or NaN in one of its real V rows turns into
+ * NaN in that column of the other cube's rows (0 * Inf).  A non-finite
+ * value in a real K row reaches only the rows whose query cube selected its
+ * cube (the other rows' logits there are replaced by -inf); values in pad
+ * slots never reach a product.
+ *
  *   q, k, v  [B, S, H, D] bf16      in
  *   topk_idx [B, H, Nq, topk] int32 in
  *   vbs      [Nq] int32             in
@@ -86,7 +101,9 @@ VSA_API int vsa_can_implement(int D, int sm_version);
  *   sm_scale  logit scale (1/sqrt(D) in the contract).
  *
  * Errors: VSA_ERR_ARG if S != 64*Nq, D != 128, topk < 1, B, H or Nq < 1,
- * or B*H*Nq, S*H*D overflow the kernel's index range; VSA_ERR_NULL for a
+ * Nq > 8192 or topk > 1024 (the kernel's shared-memory staging of the two
+ * lists of a tile), or B*H*Nq, S*H*D overflow the kernel's index range;
+ * VSA_ERR_NULL for a
  * NULL required pointer; VSA_ERR_ALIGN for a pointer not 16-byte aligned;
  * VSA_ERR_ARCH off sm_100; VSA_ERR_LAUNCH if a launch fails.  Out-of-range
  * topk_idx or vbs values found by the kernel set VSA_ERR_DEVICE; the
@@ -100,18 +117,13 @@ VSA_API int vsa_fwd(const vsa_bf16 *q, const vsa_bf16 *k, const vsa_bf16 *v, con
 enum vsa_fwd_flags {
     VSA_FWD_DEFAULT = 0,
     /* Carry the softmax weights P into the P.V product as a bf16 pair
-     * (P = hi + lo) instead of one bf16 value: about 2^-16 relative weight
-     * error instead of 2^-9, for workloads whose softmax is spread over many
-     * keys.  Costs one extra P.V product per tile. */
-    VSA_FWD_PRECISE_P = 1,
-    /* Run the warp-level mma.sync kernel instead of the tcgen05/TMEM/TMA
-     * kernel: the legacy tensor-core path, kept as the measured baseline the
-     * tcgen05 kernel is compared against.  Same results contract. */
-    VSA_FWD_LEGACY_MMA = 2,
-    /* Run the tcgen05 kernel that puts keys on the TMEM lanes (one query
-     * cube per CTA step, S^T = K Q^T) instead of the default paired-tile
-     * kernel; kept as the measured alternative.  Same results contract. */
-    VSA_FWD_KEYS_ON_LANES = 4
+     * (P = hi + lo, within 2^-17 of P) instead of one bf16 value (within
+     * 2^-9): the output is then within a small fraction of a bf16 ulp of the
+     * exact result, where the default's weight rounding can move an output
+     * element by up to 2^-8 * sum_u w_u |v_u - out| before its own rounding
+     * (one ulp at large outputs of spread-out softmax rows).  Costs a second
+     * P.V product per step (about +27 % time at Wan 832x480). */
+    VSA_FWD_PRECISE_P = 1
 };
 
 /* vsa_fwd with option flags (vsa_fwd == vsa_fwd_ex with VSA_FWD_DEFAULT). */
@@ -135,10 +147,7 @@ VSA_API int vsa_fwd_ex(const vsa_bf16 *q, const vsa_bf16 *k, const vsa_bf16 *v, 
  *        skipped.  The plan changes only which cubes share a tile: results
  *        are those of vsa_fwd_ex up to the order of floating-point sums.
  *
- * Errors: as vsa_fwd_ex, plus VSA_ERR_NULL for a NULL plan and VSA_ERR_ARG
- * if flags select another kernel or Nq > 8192 or topk > 1024 (the limits
- * of the paired kernel; without a plan, larger problems run the
- * keys-on-lanes kernel).
+ * Errors: as vsa_fwd_ex, plus VSA_ERR_NULL for a NULL plan.
  * ---------------------------------------------------------------------- */
 VSA_API int vsa_fwd_planned(const vsa_bf16 *q, const vsa_bf16 *k, const vsa_bf16 *v, const int32_t *topk_idx,
                             const int32_t *vbs, const int32_t *plan, vsa_bf16 *out, float *lse, int B, int S,
@@ -260,6 +269,47 @@ VSA_API int vsa_tile(const vsa_bf16 *x_grid, vsa_bf16 *x_tiled, int B, int T, in
 /* Inverse of vsa_tile: x_tiled [B, 64*Nq, H, D] -> x_grid [B, T*Hh*W, H, D]. */
 VSA_API int vsa_untile(const vsa_bf16 *x_tiled, vsa_bf16 *x_grid, int B, int T, int Hh, int W, int H, int D,
                cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * vsa_tile_qkv -- vsa_tile of q, k and v in one launch and, in the same
+ * pass over q and k, the cube means that vsa_route scores.
+ *
+ * The routing's cube means (vsa_route above; TensorRT-LLM PR #7, review
+ * excerpts) are sums over the first vbs[c] tokens of each cube.  Forming
+ * them while the tokens pass through the tiling reads q and k from device
+ * memory once instead of twice; vsa_route_means then finishes the routing.
+ *
+ *   q_grid, k_grid, v_grid    [B, T*Hh*W, H, D] bf16 in (raster order)
+ *   q_tiled, k_tiled, v_tiled [B, 64*Nq, H, D] bf16 out, exactly as vsa_tile
+ *   vbs     [Nq] int32 in: the counts the means divide by (normally those of
+ *           vsa_cube_counts); may be NULL when qc and kc are NULL
+ *   qc, kc  [B, H, Nq, D] bf16 out: the cube means of q and k with
+ *           vsa_route's arithmetic (slots past a cube's real tokens count as
+ *           zeros), bit-identical to the means vsa_route forms from the
+ *           tiled tensors; both NULL to tile only
+ *
+ * Errors: as vsa_tile for each of the three tensors; VSA_ERR_ARG if exactly
+ * one of qc, kc is NULL, or if means are asked for and D != 128;
+ * VSA_ERR_NULL for vbs NULL while means are asked for; VSA_ERR_ALIGN for
+ * qc, kc or vbs not 16-byte aligned.  A vbs value outside [0, 64] latches
+ * device error 2 and gives a zero mean.
+ * ---------------------------------------------------------------------- */
+VSA_API int vsa_tile_qkv(const vsa_bf16 *q_grid, const vsa_bf16 *k_grid, const vsa_bf16 *v_grid, vsa_bf16 *q_tiled,
+                         vsa_bf16 *k_tiled, vsa_bf16 *v_tiled, const int32_t *vbs, vsa_bf16 *qc, vsa_bf16 *kc, int B,
+                         int T, int Hh, int W, int H, int D, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * vsa_route_means -- the scoring and top-k steps of vsa_route, on cube means
+ * already formed (by vsa_tile_qkv):
+ *   qc, kc    [B, H, Nq, D] bf16 in
+ *   topk_idx  [B, H, Nq, topk] int32 out
+ * Same arithmetic and results as vsa_route given the tensors the means came
+ * from; no workspace.  Errors: VSA_ERR_ARG unless B, H >= 1, D = 128 and
+ * 1 <= topk <= Nq <= 4096; VSA_ERR_NULL, VSA_ERR_ALIGN, VSA_ERR_ARCH,
+ * VSA_ERR_LAUNCH as for the other calls.
+ * ---------------------------------------------------------------------- */
+VSA_API int vsa_route_means(const vsa_bf16 *qc, const vsa_bf16 *kc, int32_t *topk_idx, int B, int H, int D, int Nq,
+                            int topk, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
  * Diagnostic of the pipeline's failure handling.  Launches one warp that

@@ -76,11 +76,26 @@ def sample_items(B: int, H: int, nq: int, n: int, seed: int = 0, must=()) -> np.
 
 
 def gather_items(x: torch.Tensor, items: np.ndarray) -> np.ndarray:
-    """x [B, S, H, D] (device) -> float32 [n, 64, D] rows of the listed items."""
-    out = []
-    for b, h, i in items:
-        out.append(x[b, 64 * i: 64 * i + 64, h].float().cpu().numpy())
-    return np.stack(out)
+    """x [B, S, H, D] (device) -> float32 [n, 64, D] rows of the listed items
+    (one device-to-host copy per (b, h) run of the list)."""
+    out = np.empty((len(items), 64, x.shape[-1]), np.float32)
+    key, head = None, None
+    for n, (b, h, i) in enumerate(items):
+        if key != (b, h):
+            key, head = (b, h), x[b, :, h].float().cpu().numpy()
+        out[n] = head[64 * i: 64 * i + 64]
+    return out
+
+
+def gather_lse(lse: torch.Tensor, items: np.ndarray) -> np.ndarray:
+    """lse [B, H, S] (device) -> float64 [n, 64] rows of the listed items."""
+    out = np.empty((len(items), 64), np.float64)
+    key, head = None, None
+    for n, (b, h, i) in enumerate(items):
+        if key != (b, h):
+            key, head = (b, h), lse[b, h].cpu().numpy().astype(np.float64)
+        out[n] = head[64 * i: 64 * i + 64]
+    return out
 
 
 def near_tie_reference(gpu: np.ndarray, o64: np.ndarray, frac: float = 1.0 / 32, bound=None):
@@ -116,26 +131,51 @@ def near_tie_reference(gpu: np.ndarray, o64: np.ndarray, frac: float = 1.0 / 32,
     return ref.astype(np.float32), n_adj
 
 
-# Default forward mode rounds each softmax weight to bf16 before the P.V
-# product (relative error <= 2^-9 per weight); the sum of weights is kept
-# in fp32.  The output before its own rounding is then within
-# 2^-9 * sum_u w_u |v_u| (+ fp32 accumulation, covered by a factor 2) of exact.
-BF16_WEIGHT_BOUND = 2.0 ** -8
-
-
-def compare(gpu_rows: np.ndarray, o64: np.ndarray, heads: np.ndarray, wabs=None) -> dict:
+def compare(gpu_rows: np.ndarray, o64: np.ndarray, heads: np.ndarray) -> dict:
     """The dataset card's pass rule, per head, against bf16_rne(oracle) with the
-    near-midpoint reading (gate), and against the unrounded FP64 oracle
-    (reported).  wabs (oracle's sum_u w_u |v_u|) widens the near-midpoint
-    window by the default mode's weight-rounding bound."""
-    bound = None if wabs is None else BF16_WEIGHT_BOUND * wabs
-    ref, n_adj = near_tie_reference(gpu_rows, o64, bound=bound)
+    1/32-ulp near-midpoint reading (gate; many such ties would flag a bias, so
+    at most 1e-3 of the elements may be taken that way), and against the
+    unrounded FP64 oracle (reported)."""
+    ref, n_adj = near_tie_reference(gpu_rows, o64)
     res = {"gate": _rule(gpu_rows, ref, heads), "fp64": _rule(gpu_rows, o64.astype(np.float32), heads)}
     res["gate"]["near_tie_adjusted"] = n_adj
-    if wabs is None:
-        # plain near-midpoint reading: such ties are rare, so many of them flag a bias
-        res["gate"]["ok"] = bool(res["gate"]["ok"] and n_adj <= max(4, 1e-3 * gpu_rows.size))
+    res["gate"]["ok"] = bool(res["gate"]["ok"] and n_adj <= max(4, 1e-3 * gpu_rows.size))
     return res
+
+
+# The default forward mode rounds each softmax weight to bf16 (relative error
+# <= 2^-9) before the P.V product and sums the same rounded weights, so its
+# output before the final rounding is a weighted mean with perturbed weights:
+# within 2^-8 * sum_u w_u |v_u - out| <= 2^-8 * 2 * sum_u w_u |v_u| of exact.
+DEFAULT_WEIGHT_BOUND = 2.0 ** -7
+
+
+def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
+    a = np.maximum(np.abs(x), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 8)
+
+
+def within_default_bound(gpu_rows: np.ndarray, o64: np.ndarray, wabs: np.ndarray) -> dict:
+    """The default mode's stated per-element error bound (not the card's rule):
+    |gpu - exact| <= half a bf16 ulp + 2^-7 * sum_u w_u |v_u| (+ 2^-20 |exact|
+    for the fp32 accumulation)."""
+    g = gpu_rows.astype(np.float64)
+    err = np.abs(g - o64)
+    lim = bf16_half_ulp(np.maximum(np.abs(g), np.abs(o64))) + DEFAULT_WEIGHT_BOUND * wabs + 2.0 ** -20 * np.abs(o64)
+    worst = float(np.max(err - lim))
+    return {"ok": bool(np.isfinite(g).all() and worst <= 0), "worst_excess": worst,
+            "max_err": float(err.max())}
+
+
+def head_cosine(x: np.ndarray, y: np.ndarray) -> float:
+    """Cosine of two FP32 vectors with the sums taken in FP64.  A head holds
+    64 * 128 * Nq values (5.1 M at Wan 832x480); torch's fp32 cosine on the
+    CPU is off by ~1e-3 at that length (cos(a, a) = 1.0018 on such a vector),
+    larger than the 1e-4 the rule tests for."""
+    x = x.reshape(-1).astype(np.float32).astype(np.float64)
+    y = y.reshape(-1).astype(np.float32).astype(np.float64)
+    den = np.sqrt(float(x @ x) * float(y @ y))
+    return float(x @ y) / max(den, 1e-300)
 
 
 def _rule(a: np.ndarray, b: np.ndarray, heads: np.ndarray) -> dict:
@@ -143,9 +183,7 @@ def _rule(a: np.ndarray, b: np.ndarray, heads: np.ndarray) -> dict:
     cos = []
     for h in np.unique(heads):
         sel = heads == h
-        x = torch.from_numpy(a[sel].reshape(-1).astype(np.float32))
-        y = torch.from_numpy(b[sel].reshape(-1).astype(np.float32))
-        cos.append(float(torch.nn.functional.cosine_similarity(x, y, dim=0)))
+        cos.append(head_cosine(a[sel], b[sel]))
     diff = np.abs(a.astype(np.float32) - b.astype(np.float32))
     r = {"finite": finite, "min_head_cos": min(cos), "max_abs": float(diff.max()), "mean_abs": float(diff.mean())}
     r["ok"] = bool(finite and r["min_head_cos"] >= scoring.MIN_COS and r["max_abs"] <= scoring.MAX_ABS
@@ -153,10 +191,14 @@ def _rule(a: np.ndarray, b: np.ndarray, heads: np.ndarray) -> dict:
     return r
 
 
-def lse_bound(qt, kt, items, sm_scale):
+def lse_bound(qt, kt, items, sm_scale, default_mode=True):
     """Per-row bound on the fp32 error of the log-sum-exp: the logits' dot
     products accumulate in fp32 over 128 terms (error <= ~1e-5 of the sum of
-    |products|) plus a small absolute term for the fp32 sum of weights."""
+    |products|) plus a small absolute term for the fp32 sum of weights.  The
+    default mode's row sum adds the bf16-rounded weights (each within 2^-9 of
+    its value), the sum that also normalises its output: that adds up to
+    -ln(1 - 2^-9) < 2e-3."""
+    extra = 2e-3 if default_mode else 0.0
     sigma = float(np.float32(sm_scale))
     out = []
     kmax = None
@@ -165,5 +207,5 @@ def lse_bound(qt, kt, items, sm_scale):
         if kmax is None or kmax[0] != (b, h):
             kabs = np.abs(oracle.bf16_to_f64(kt[b, :, h]))  # [S, D]
             kmax = ((b, h), kabs.max(axis=0))
-        out.append(1e-4 + 2e-5 * sigma * (np.abs(q) @ kmax[1]))
+        out.append(1e-4 + extra + 2e-5 * sigma * (np.abs(q) @ kmax[1]))
     return np.stack(out)

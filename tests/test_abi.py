@@ -118,6 +118,35 @@ def test_tile_rejects_bad_arguments_without_a_device(vsa):
     assert vsa.get_lib().vsa_untile(p, _fake((1 << 20) + 8), 1, 5, 6, 7, 2, 128, None) == -3
 
 
+def test_tile_qkv_and_route_means_reject_bad_arguments_without_a_device(vsa):
+    p = _fake(1 << 20)
+    lib = vsa.get_lib()
+    # grid 5x6x7, B=1, H=2, D=128
+    assert lib.vsa_tile_qkv(p, p, p, p, p, p, p, p, None, 1, 5, 6, 7, 2, 128, None) == -1  # kc missing
+    assert lib.vsa_tile_qkv(p, p, p, p, p, p, p, p, p, 1, 5, 6, 7, 2, 64, None) == -1  # means need D = 128
+    assert lib.vsa_tile_qkv(p, p, p, p, p, p, None, p, p, 1, 5, 6, 7, 2, 128, None) == -2  # means need vbs
+    assert lib.vsa_tile_qkv(p, p, None, p, p, p, None, None, None, 1, 5, 6, 7, 2, 128, None) == -2
+    assert lib.vsa_tile_qkv(p, p, p, p, p, p, None, None, None, 1, 0, 6, 7, 2, 128, None) == -1
+    assert lib.vsa_tile_qkv(p, p, p, p, p, _fake((1 << 20) + 4), None, None, None, 1, 5, 6, 7, 2, 128, None) == -3
+    assert lib.vsa_route_means(p, p, p, 1, 2, 128, 8, 9, None) == -1  # topk > Nq
+    assert lib.vsa_route_means(p, p, p, 1, 2, 64, 8, 2, None) == -1  # D != 128
+    assert lib.vsa_route_means(p, p, p, 1, 2, 128, 5000, 2, None) == -1  # Nq > 4096
+    assert lib.vsa_route_means(p, None, p, 1, 2, 128, 8, 2, None) == -2
+    assert lib.vsa_route_means(p, p, _fake((1 << 20) + 4), 1, 2, 128, 8, 2, None) == -3
+
+
+def test_route_noalloc_checks_arguments_before_its_array_limit(vsa):
+    """Bad arguments are reported as by vsa_route, even for a problem larger than
+    the fixed array, and before any device is touched."""
+    p = _fake(1 << 20)
+    lib = vsa.get_lib()
+    # B=2, H=40, Nq=1440 needs more than the array; D = 64 is invalid
+    assert lib.vsa_route_noalloc(p, p, p, p, 2, 64 * 1440, 40, 64, 1440, 180, None) == -1
+    assert lib.vsa_route_noalloc(p, p, p, p, 2, 64 * 1440, 40, 128, 1440, 2000, None) == -1  # topk > Nq
+    assert lib.vsa_route_noalloc(None, p, p, p, 2, 64 * 1440, 40, 128, 1440, 180, None) == -2
+    assert lib.vsa_route_noalloc(p, p, _fake((1 << 20) + 4), p, 2, 64 * 1440, 40, 128, 1440, 180, None) == -3
+
+
 def test_product_package_does_not_reach_the_oracle():
     """The product path never imports or loads the oracle."""
     pkg = os.path.join(ROOT, "video_block_sparse_b200")

@@ -50,6 +50,39 @@ def test_tile_untile_bit_exact(vsa, grid, B, H):
     _no_device_error(vsa)
 
 
+@pytest.mark.parametrize("grid,B,H", [((5, 6, 7), 1, 2), ((9, 3, 5), 2, 3), ((21, 30, 52), 1, 40)])
+def test_tile_qkv_and_means_bit_exact(vsa, grid, B, H):
+    """One launch tiles q, k, v exactly as vsa_tile does and forms the cube
+    means of q and k exactly as the routing does from the tiled tensors
+    (including counts below a cube's real extent, above it, and zero); the
+    routing finished from those means equals the oracle's."""
+    g = np.random.default_rng(7)
+    L = int(np.prod(grid))
+    xs = [synth.f32_to_bf16_bits((g.standard_normal((B, L, H, 128)) * 3).astype(np.float32)) for _ in range(3)]
+    vbs = oracle.cube_counts(*grid).copy()
+    nq = len(vbs)
+    vbs[0] = 0
+    vbs[nq - 1] = 64  # a partial cube averaged over its pads as well
+    if nq > 2:
+        vbs[1] = max(1, vbs[1] // 3)
+    dvbs = torch.from_numpy(vbs).cuda()
+    qt, kt, vt, qc, kc = vsa.tile_qkv(*(common.dev(x) for x in xs), grid, dvbs)
+    torch.cuda.synchronize()
+    _no_device_error(vsa)
+    tiled = [oracle.tile(x, *grid) for x in xs]
+    for got, want in zip((qt, kt, vt), tiled):
+        np.testing.assert_array_equal(common.host_bits(got), want)
+    np.testing.assert_array_equal(common.host_bits(qc), oracle.cube_means(tiled[0], vbs))
+    np.testing.assert_array_equal(common.host_bits(kc), oracle.cube_means(tiled[1], vbs))
+    topk = min(nq, 78)
+    got_idx = vsa.route_means(qc, kc, topk)
+    np.testing.assert_array_equal(got_idx.cpu().numpy(), oracle.route(tiled[0], tiled[1], vbs, topk))
+    only = vsa.tile_qkv(*(common.dev(x) for x in xs), grid, means=False)
+    for got, want in zip(only[:3], tiled):
+        np.testing.assert_array_equal(common.host_bits(got), want)
+    _no_device_error(vsa)
+
+
 # ------------------------------------------------------------------ routing
 
 @pytest.mark.parametrize("name", ["tiny", "wan480", "adversarial", "wan720"])
@@ -98,28 +131,55 @@ def _run_fwd(vsa, p: common.Prepared, flags=0):
     return out, lse
 
 
-def _check_items(p: common.Prepared, out, lse, items, tag, precise=False):
-    """The pass rule on the listed items.  The default mode rounds each weight
-    to bf16 before P.V, so its near-midpoint window includes that rounding's
-    error bound (oracle's sum_u w_u |v_u| times 2^-8); the precise mode keeps
-    the weights to ~2^-17 and is gated with the plain 1/32-ulp window."""
-    o64, l64, wabs = oracle.fwd_items(p.qt, p.kt, p.vt, p.idx, p.vbs, p.cfg.sm_scale, items, want_wabs=True)
+def _check_items(p: common.Prepared, out, lse, items, tag, rule=True, precise=False):
+    """rule=True: the card's pass rule against bf16_rne(oracle) with only the
+    1/32-ulp near-midpoint reading (the gate of every Wan-shaped case, in both
+    precision modes).  rule=False: the default mode's stated per-element error
+    bound instead (small cases whose softmax rows are spread out and whose
+    outputs reach |out| >= 4, where the default's weight rounding can move an
+    element by one bf16 ulp; the precise mode meets the rule there).
+    precise: the output came from the precise mode (tighter lse bound)."""
+    got = oracle.fwd_items(p.qt, p.kt, p.vt, p.idx, p.vbs, p.cfg.sm_scale, items, want_wabs=not rule)
+    o64, l64, wabs = got if not rule else (*got, None)
     rows = common.gather_items(out, items)
-    res = common.compare(rows, o64, items[:, 1] + 1000 * items[:, 0], wabs=None if precise else wabs)
+    hid = items[:, 1] + 1000 * items[:, 0]
+    res = common.compare(rows, o64, hid)
     print(f"\n[{tag}] gate {res['gate']}\n[{tag}] vs fp64 {res['fp64']}")
-    assert res["gate"]["ok"], res
-    got_lse = np.stack([lse[b, h, 64 * i: 64 * i + 64].cpu().numpy() for b, h, i in items]).astype(np.float64)
+    if rule:
+        assert res["gate"]["ok"], res
+    else:
+        bnd = common.within_default_bound(rows, o64, wabs)
+        print(f"[{tag}] default-mode bound {bnd}")
+        assert bnd["ok"], bnd
+    assert res["fp64"]["finite"] and res["fp64"]["min_head_cos"] >= 0.9999, res["fp64"]
+    got_lse = common.gather_lse(lse, items)
     fin = np.isfinite(l64)
     assert np.array_equal(fin, np.isfinite(got_lse))
-    bound = common.lse_bound(p.qt, p.kt, items, p.cfg.sm_scale)
+    bound = common.lse_bound(p.qt, p.kt, items, p.cfg.sm_scale, default_mode=not precise)
     assert np.all(np.abs(got_lse[fin] - l64[fin]) <= bound[fin]), float(np.max(np.abs(got_lse[fin] - l64[fin])))
+
+
+def _head_items(p: common.Prepared, heads, batches=None):
+    it = oracle.all_items(p.cfg.B, p.cfg.H, p.nq)
+    keep = np.isin(it[:, 1], heads)
+    if batches is not None:
+        keep &= np.isin(it[:, 0], batches)
+    return it[keep]
 
 
 def test_fwd_tiny_precise_all_rows(vsa):
     p = common.prepare("tiny")
     out, lse = _run_fwd(vsa, p, flags=vsa.FWD_PRECISE_P)
-    items = oracle.all_items(p.cfg.B, p.cfg.H, p.nq)
-    _check_items(p, out, lse, items, "tiny/precise", precise=True)
+    _check_items(p, out, lse, oracle.all_items(p.cfg.B, p.cfg.H, p.nq), "tiny/precise", precise=True)
+
+
+def test_fwd_tiny_default_within_its_bound(vsa):
+    """The tiny configuration (U[0.5, 4] value scales, softmax spread over up to
+    128 keys) is the one case the default mode does not meet the rule on: one
+    bf16 ulp at |out| >= 4 is 0.031.  It stays within its stated bound."""
+    p = common.prepare("tiny")
+    out, lse = _run_fwd(vsa, p)
+    _check_items(p, out, lse, oracle.all_items(p.cfg.B, p.cfg.H, p.nq), "tiny/default", rule=False)
 
 
 def test_fwd_mid_ragged_all_rows(vsa):
@@ -131,27 +191,58 @@ def test_fwd_mid_ragged_all_rows(vsa):
         _check_items(p, out, lse, items, f"mid/flags{flags}", precise=flags != 0)
 
 
-@pytest.mark.parametrize("name,n", [("wan480", 120), ("adversarial", 160), ("sweep32", 60), ("sweep156", 40)])
-def test_fwd_full_size_sampled(vsa, name, n):
+def _run_fwd_both_pairings(vsa, p):
+    """The default mode with the consecutive pairing and with vsa_plan's."""
+    q, k, v = common.dev(p.qt), common.dev(p.kt), common.dev(p.vt)
+    idx = torch.from_numpy(p.idx).cuda()
+    vbs = torch.from_numpy(p.vbs).cuda()
+    res = {}
+    for planned in (False, True):
+        pl = vsa.plan(idx) if planned else None
+        out, lse = vsa.fwd(q, k, v, idx, vbs, p.cfg.sm_scale, want_lse=True, plan=pl)
+        torch.cuda.synchronize()
+        _no_device_error(vsa)
+        assert bool(torch.isfinite(out).all())
+        res[planned] = (out, lse)
+    return res
+
+
+@pytest.mark.parametrize("name,heads", [
+    ("wan480", [0, 17]),
+    ("adversarial", list(synth.ADV_T_HEADS) + [synth.ADV_FORCED_HEAD, 1]),
+    ("sweep32", [3]),
+    ("sweep156", [3]),
+])
+def test_fwd_full_size_whole_heads(vsa, name, heads):
+    """Every row of whole heads at full size (the adversarial config: its three
+    Student-t heads, the head with the forced low-count cubes and a clean head),
+    with the consecutive and the planned pairing."""
     p = common.prepare(name)
-    out, lse = _run_fwd(vsa, p)
-    assert bool(torch.isfinite(out).all())
-    must = []
-    if p.cfg.adversarial:
-        must = [(0, h, i) for h in synth.ADV_T_HEADS for i in (0, 311, 623)]
-        must += [(0, synth.ADV_FORCED_HEAD, i) for i in range(0, 624, 40)]
-    items = common.sample_items(p.cfg.B, p.cfg.H, p.nq, n, seed=3, must=must)
-    _check_items(p, out, lse, items, name)
+    items = _head_items(p, heads)
+    for planned, (out, lse) in _run_fwd_both_pairings(vsa, p).items():
+        _check_items(p, out, lse, items, f"{name}/planned{int(planned)}")
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name,n", [("wan720", 60), ("sweep312", 24), ("dense624", 16)])
-def test_fwd_large_sampled(vsa, name, n):
+@pytest.mark.parametrize("name,heads", [("wan720", [0]), ("sweep312", [5]), ("dense624", [2])])
+def test_fwd_large_whole_heads(vsa, name, heads):
     p = common.prepare(name)
-    out, lse = _run_fwd(vsa, p)
-    assert bool(torch.isfinite(out).all())
-    items = common.sample_items(p.cfg.B, p.cfg.H, p.nq, n, seed=4)
-    _check_items(p, out, lse, items, name)
+    items = _head_items(p, heads)
+    for planned, (out, lse) in _run_fwd_both_pairings(vsa, p).items():
+        _check_items(p, out, lse, items, f"{name}/planned{int(planned)}")
+
+
+@pytest.mark.slow
+def test_fwd_wan480_every_row(vsa):
+    """Every row of the whole Wan 832x480 output, as the bench computes it
+    (planned pairing), element by element against the oracle."""
+    p = common.prepare("wan480")
+    q, k, v = common.dev(p.qt), common.dev(p.kt), common.dev(p.vt)
+    idx, vbs = torch.from_numpy(p.idx).cuda(), torch.from_numpy(p.vbs).cuda()
+    out, lse = vsa.fwd(q, k, v, idx, vbs, p.cfg.sm_scale, want_lse=True, plan=vsa.plan(idx))
+    torch.cuda.synchronize()
+    _no_device_error(vsa)
+    _check_items(p, out, lse, oracle.all_items(p.cfg.B, p.cfg.H, p.nq), "wan480/all")
 
 
 def test_fwd_dense_matches_library_attention(vsa):
@@ -186,7 +277,8 @@ def test_fwd_edge_lists(vsa, seed, topk, dup):
     p = _small(seed, topk=topk, dup=dup, vbs=[64, 1, 17, 33, 48][:5])
     for flags in (0, vsa.FWD_PRECISE_P):
         out, lse = _run_fwd(vsa, p, flags)
-        _check_items(p, out, lse, oracle.all_items(1, 2, 5), f"edge{seed}/{flags}", precise=flags != 0)
+        _check_items(p, out, lse, oracle.all_items(1, 2, 5), f"edge{seed}/{flags}", rule=flags != 0,
+                     precise=flags != 0)
 
 
 @pytest.mark.parametrize("seed,topk,plan", [(20, 1, False), (21, 2, False), (22, 3, True)])
@@ -203,7 +295,7 @@ def test_fwd_many_short_tiles(vsa, seed, topk, plan):
     out, lse = vsa.fwd(q, k, v, idx, vbs, p.cfg.sm_scale, want_lse=True, plan=pl)
     torch.cuda.synchronize()
     _no_device_error(vsa)
-    _check_items(p, out, lse, oracle.all_items(1, 80, 9), f"short{seed}")
+    _check_items(p, out, lse, oracle.all_items(1, 80, 9), f"short{seed}", rule=False)
 
 
 def test_fwd_all_masked_rows(vsa):
@@ -226,6 +318,35 @@ def test_fwd_nan_pads_do_not_leak(vsa):
     out1, lse1 = _run_fwd(vsa, p)
     assert torch.equal(out0.view(torch.int16), out1.view(torch.int16))
     assert torch.equal(lse0, lse1)
+
+
+def test_fwd_nonfinite_real_v_row(vsa):
+    """An Inf in a real V row (the contract asks for finite real rows): every
+    query cube that selected that KV cube gets a non-finite value in that
+    column, as the definition does; its tile partner, which did not select
+    the cube, gets NaN there (weight 0 times Inf: the documented deviation of
+    paired tiles); every other element still matches the oracle."""
+    p = _small(19, nq=4, H=1, topk=2, vbs=[64, 64, 64, 64])
+    p.idx[0, 0] = np.array([[0, 2], [1, 3], [0, 1], [3, 1]], np.int32)
+    j, r, d = 2, 5, 7
+    p.vt[0, 64 * j + r, 0, d] = 0x7F80  # +inf in a real row of cube 2 (selected by query cube 0 only)
+    plan = torch.tensor([[[0, 1], [2, 3]]], dtype=torch.int32).cuda()
+    q, k, v = common.dev(p.qt), common.dev(p.kt), common.dev(p.vt)
+    out = vsa.fwd(q, k, v, torch.from_numpy(p.idx).cuda(), torch.from_numpy(p.vbs).cuda(), p.cfg.sm_scale, plan=plan)
+    torch.cuda.synchronize()
+    _no_device_error(vsa)
+    items = oracle.all_items(1, 1, 4)
+    o64, _, wabs = oracle.fwd_items(p.qt, p.kt, p.vt, p.idx, p.vbs, p.cfg.sm_scale, items, want_wabs=True)
+    rows = common.gather_items(out, items)
+    col = np.zeros(rows.shape, bool)
+    col[..., d] = True
+    assert not np.isfinite(rows[0][col[0]]).any() and not np.isfinite(o64[0][col[0]]).any()  # selected it
+    assert np.isnan(rows[1][col[1]]).all() and np.isfinite(o64[1]).all()  # partner: the deviation
+    finite = np.isfinite(o64)
+    finite[1] &= ~col[1]
+    bnd = common.within_default_bound(np.where(finite, rows, 0), np.where(finite, o64, 0), np.where(finite, wabs, 0))
+    assert bnd["ok"], bnd
+    assert np.isfinite(rows[2:]).all()  # the other tile never saw cube 2
 
 
 def test_fwd_deterministic(vsa):
@@ -272,7 +393,7 @@ def test_stalled_pipeline_wait_ends_with_error_status(vsa):
     assert 0.2 < elapsed < 60.0
     p = _small(16, nq=4, H=1, topk=2, vbs=[64, 40, 64, 9])
     out, lse = _run_fwd(vsa, p)
-    _check_items(p, out, lse, oracle.all_items(1, 1, 4), "after-stall", precise=False)
+    _check_items(p, out, lse, oracle.all_items(1, 1, 4), "after-stall", rule=False)
     assert vsa.device_status() == (0, 0)
 
 
@@ -298,10 +419,15 @@ def test_fwd_negative_scale(vsa):
         out, lse = vsa.fwd(q, k, v, idx, vbs, -0.3, want_lse=True, flags=flags)
         torch.cuda.synchronize()
         _no_device_error(vsa)
-        res = common.compare(common.gather_items(out, items), o64, items[:, 1], wabs=None if flags else wabs)
-        assert res["gate"]["ok"], res
-        got_lse = np.stack([lse[b, h, 64 * i: 64 * i + 64].cpu().numpy() for b, h, i in items])
-        assert np.allclose(got_lse, l64, rtol=1e-5, atol=1e-3)
+        rows = common.gather_items(out, items)
+        if flags:
+            res = common.compare(rows, o64, items[:, 1])
+            assert res["gate"]["ok"], res
+        else:
+            bnd = common.within_default_bound(rows, o64, wabs)
+            assert bnd["ok"], bnd
+        got_lse = common.gather_lse(lse, items)
+        assert np.allclose(got_lse, l64, rtol=1e-5, atol=1e-3 if flags else 3e-3)
 
 
 # ------------------------------------------------------------------ tile plan
@@ -348,7 +474,7 @@ def test_fwd_with_arbitrary_pairing(vsa):
     out, lse = vsa.fwd(q, k, v, idx, vbs, p.cfg.sm_scale, want_lse=True, plan=torch.from_numpy(plan).cuda())
     torch.cuda.synchronize()
     _no_device_error(vsa)
-    _check_items(p, out, lse, oracle.all_items(1, 2, 9), "arbitrary-pairing")
+    _check_items(p, out, lse, oracle.all_items(1, 2, 9), "arbitrary-pairing", rule=False)
 
 
 def test_fwd_plan_bad_entry_latches_error(vsa):
@@ -359,16 +485,3 @@ def test_fwd_plan_bad_entry_latches_error(vsa):
             plan=torch.from_numpy(plan).cuda())
     rc, detail = vsa.device_status()
     assert rc == -7 and detail == 4
-
-
-def test_fwd_planned_full_size_sampled(vsa):
-    """Wan 832x480 shape, planner's pairing from the GPU planner, sampled rows."""
-    p = common.prepare("wan480")
-    q, k, v = common.dev(p.qt), common.dev(p.kt), common.dev(p.vt)
-    idx, vbs = torch.from_numpy(p.idx).cuda(), torch.from_numpy(p.vbs).cuda()
-    plan = vsa.plan(idx)
-    out, lse = vsa.fwd(q, k, v, idx, vbs, p.cfg.sm_scale, want_lse=True, plan=plan)
-    torch.cuda.synchronize()
-    _no_device_error(vsa)
-    items = common.sample_items(p.cfg.B, p.cfg.H, p.nq, 120, seed=5)
-    _check_items(p, out, lse, items, "wan480/planned")

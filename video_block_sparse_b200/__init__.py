@@ -8,8 +8,10 @@ and the current stream to the library and raises ``VSAError`` on a non-zero
 status.  There is no CPU or fallback path: if ``libvsa.so`` is missing or
 cannot be loaded, the first call raises ImportError.
 
-Names follow the C ABI: ``fwd`` (vsa_fwd / vsa_fwd_ex), ``route``,
-``tile``, ``untile``, ``cube_counts``, ``device_status``.
+Names follow the C ABI: ``fwd`` (vsa_fwd / vsa_fwd_ex / vsa_fwd_planned),
+``route``, ``route_means``, ``route_noalloc``, ``plan``, ``tile``,
+``tile_qkv``, ``untile``, ``cube_counts``, ``device_status``,
+``stall_check``.
 """
 from __future__ import annotations
 
@@ -23,16 +25,15 @@ LIB_PATH = os.path.join(_HERE, "libvsa.so")
 
 FWD_DEFAULT = 0
 FWD_PRECISE_P = 1
-FWD_LEGACY_MMA = 2
-FWD_KEYS_ON_LANES = 4
 
 _STATUS = {0: "VSA_OK", -1: "VSA_ERR_ARG", -2: "VSA_ERR_NULL", -3: "VSA_ERR_ALIGN", -4: "VSA_ERR_WORKSPACE",
            -5: "VSA_ERR_ARCH", -6: "VSA_ERR_LAUNCH", -7: "VSA_ERR_DEVICE"}
 
 # every symbol include/vsa.h declares
 EXPORTS = ("vsa_status_string", "vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_fwd_planned",
-           "vsa_plan_workspace_size", "vsa_plan", "vsa_route_workspace_size",
-           "vsa_route", "vsa_route_noalloc", "vsa_cube_counts", "vsa_tile", "vsa_untile", "vsa_device_status")
+           "vsa_plan_workspace_size", "vsa_plan", "vsa_route_workspace_size", "vsa_route", "vsa_route_means",
+           "vsa_route_noalloc", "vsa_cube_counts", "vsa_tile", "vsa_tile_qkv", "vsa_untile", "vsa_stall_check",
+           "vsa_device_status")
 
 
 class VSAError(RuntimeError):
@@ -62,11 +63,13 @@ def _load():
     lib.vsa_cube_counts.argtypes = [I, I, I, P, P]
     lib.vsa_tile.argtypes = [P, P, I, I, I, I, I, I, P]
     lib.vsa_untile.argtypes = [P, P, I, I, I, I, I, I, P]
+    lib.vsa_tile_qkv.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, P]
+    lib.vsa_route_means.argtypes = [P, P, P, I, I, I, I, I, P]
     lib.vsa_device_status.argtypes = [P, P]
     lib.vsa_stall_check.argtypes = [P, P]
-    for name in ("vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_fwd_planned", "vsa_plan", "vsa_route", "vsa_route_noalloc", "vsa_cube_counts",
-                 "vsa_tile",
-                 "vsa_untile", "vsa_device_status", "vsa_stall_check"):
+    for name in ("vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_fwd_planned", "vsa_plan", "vsa_route",
+                 "vsa_route_means", "vsa_route_noalloc", "vsa_cube_counts", "vsa_tile", "vsa_tile_qkv", "vsa_untile",
+                 "vsa_device_status", "vsa_stall_check"):
         getattr(lib, name).restype = I
     return lib
 
@@ -149,6 +152,51 @@ def untile(x_tiled: torch.Tensor, grid, out: torch.Tensor | None = None, stream=
     if out.shape != (B, T * Hh * W, H, D):
         raise ValueError("untile: shape mismatch")
     _check(get_lib().vsa_untile(_ptr(x_tiled), _ptr(out), B, T, Hh, W, H, D, _stream(stream)), "vsa_untile")
+    return out
+
+
+def tile_qkv(q_grid: torch.Tensor, k_grid: torch.Tensor, v_grid: torch.Tensor, grid, vbs: torch.Tensor | None = None,
+             means: bool = True, out=None, stream=None):
+    """vsa_tile_qkv: tile q, k, v ([B, T*Hh*W, H, D] raster) in one launch and,
+    if `means`, form the cube means of q and k ([B, H, Nq, D]) in the same pass.
+    Returns (q_tiled, k_tiled, v_tiled, qc, kc) (qc, kc None without means).
+    `out` may hold preallocated tensors in that order."""
+    T, Hh, W = grid
+    B, L, H, D = q_grid.shape
+    for t, n in ((q_grid, "q_grid"), (k_grid, "k_grid"), (v_grid, "v_grid")):
+        _bf16(t, n)
+        if t.shape != q_grid.shape:
+            raise ValueError("tile_qkv: q, k, v shapes differ")
+    nq = ctypes.c_int(0)
+    _check(get_lib().vsa_cube_counts(T, Hh, W, None, ctypes.byref(nq)), "vsa_cube_counts")
+    nq = nq.value
+    if out is None:
+        dev = q_grid.device
+        out = [torch.empty(B, 64 * nq, H, D, dtype=q_grid.dtype, device=dev) for _ in range(3)]
+        out += [torch.empty(B, H, nq, D, dtype=q_grid.dtype, device=dev) for _ in range(2)] if means else [None, None]
+    qt, kt, vt, qc, kc = out
+    if L != T * Hh * W or any(x.shape != (B, 64 * nq, H, D) for x in (qt, kt, vt)):
+        raise ValueError("tile_qkv: shape mismatch")
+    if means and (vbs is None or qc is None or kc is None or qc.shape != (B, H, nq, D) or kc.shape != qc.shape):
+        raise ValueError("tile_qkv: means need vbs and [B, H, Nq, D] outputs")
+    _check(get_lib().vsa_tile_qkv(_ptr(q_grid), _ptr(k_grid), _ptr(v_grid), _ptr(qt), _ptr(kt), _ptr(vt),
+                                  _ptr(vbs) if means else None, _ptr(qc) if means else None,
+                                  _ptr(kc) if means else None, B, T, Hh, W, H, D, _stream(stream)), "vsa_tile_qkv")
+    return (qt, kt, vt, qc, kc) if means else (qt, kt, vt, None, None)
+
+
+def route_means(qc: torch.Tensor, kc: torch.Tensor, topk: int, out: torch.Tensor | None = None,
+                stream=None) -> torch.Tensor:
+    """vsa_route_means: topk_idx [B, H, Nq, topk] int32 from cube means qc, kc [B, H, Nq, D]."""
+    B, H, nq, D = qc.shape
+    _bf16(qc, "qc")
+    _bf16(kc, "kc")
+    if kc.shape != qc.shape:
+        raise ValueError("route_means: qc and kc shapes differ")
+    if out is None:
+        out = torch.empty(B, H, nq, topk, dtype=torch.int32, device=qc.device)
+    _check(get_lib().vsa_route_means(_ptr(qc), _ptr(kc), _ptr(out), B, H, D, nq, topk, _stream(stream)),
+           "vsa_route_means")
     return out
 
 

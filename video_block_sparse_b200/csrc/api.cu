@@ -5,6 +5,7 @@
 
 #include "internal.h"
 
+#include <atomic>
 #include <climits>
 #include <cstdint>
 
@@ -13,9 +14,12 @@ namespace {
 // One error word per device; kernels latch the first error with atomicCAS.
 __device__ int g_device_error;
 
+// Per-device values looked up on first use.  Host threads may make their first
+// calls at the same time: each slot is an atomic, and racing threads store the
+// same value.
 constexpr int kMaxDevices = 64;
-int* g_err_ptr[kMaxDevices];
-int g_sm_version[kMaxDevices];
+std::atomic<int*> g_err_ptr[kMaxDevices];
+std::atomic<int> g_sm_version[kMaxDevices];
 
 int current_device(int* dev)
 {
@@ -25,14 +29,16 @@ int current_device(int* dev)
 
 int device_sm(int dev)
 {
-    if (g_sm_version[dev] == 0) {
+    int sm = g_sm_version[dev].load(std::memory_order_relaxed);
+    if (sm == 0) {
         int major = 0, minor = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
             return -1;
-        g_sm_version[dev] = major * 10 + minor;
+        sm = major * 10 + minor;
+        g_sm_version[dev].store(sm, std::memory_order_relaxed);
     }
-    return g_sm_version[dev];
+    return sm;
 }
 
 // Address of this device's error word (looked up once per device).
@@ -40,12 +46,14 @@ int device_error_word(int** out)
 {
     int dev;
     if (current_device(&dev) != VSA_OK) return VSA_ERR_LAUNCH;
-    if (g_err_ptr[dev] == nullptr) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return VSA_ERR_LAUNCH;
-        g_err_ptr[dev] = static_cast<int*>(p);
+    int* p = g_err_ptr[dev].load(std::memory_order_relaxed);
+    if (p == nullptr) {
+        void* a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_device_error) != cudaSuccess || a == nullptr) return VSA_ERR_LAUNCH;
+        p = static_cast<int*>(a);
+        g_err_ptr[dev].store(p, std::memory_order_relaxed);
     }
-    *out = g_err_ptr[dev];
+    *out = p;
     return VSA_OK;
 }
 
@@ -106,12 +114,9 @@ int fwd_dispatch(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const 
 {
     int rc = check_bshd(B, S, H, D, Nq);
     if (rc != VSA_OK) return rc;
-    if (topk < 1 || (flags & ~(VSA_FWD_PRECISE_P | VSA_FWD_LEGACY_MMA | VSA_FWD_KEYS_ON_LANES)) != 0)
-        return VSA_ERR_ARG;
-    if ((flags & VSA_FWD_LEGACY_MMA) && (flags & VSA_FWD_KEYS_ON_LANES)) return VSA_ERR_ARG;
+    if (topk < 1 || (flags & ~VSA_FWD_PRECISE_P) != 0) return VSA_ERR_ARG;
+    if (!vsa::fwd_pair_supported(Nq, topk)) return VSA_ERR_ARG;
     if ((int64_t)B * H * Nq * topk > INT32_MAX) return VSA_ERR_ARG;
-    const bool pair_kernel = (flags & (VSA_FWD_LEGACY_MMA | VSA_FWD_KEYS_ON_LANES)) == 0;
-    if (plan != nullptr && (!pair_kernel || !vsa::fwd_pair_supported(Nq, topk))) return VSA_ERR_ARG;
     if (!q || !k || !v || !topk_idx || !vbs || !out) return VSA_ERR_NULL;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(topk_idx) ||
         !aligned16(vbs) || (lse && !aligned16(lse)) || (plan && !aligned16(plan)))
@@ -120,17 +125,27 @@ int fwd_dispatch(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const 
     int* err;
     if ((rc = device_error_word(&err)) != VSA_OK) return rc;
     const bool precise = (flags & VSA_FWD_PRECISE_P) != 0;
-    if (flags & VSA_FWD_LEGACY_MMA)
-        return launch_status(
-            vsa::launch_fwd_mma(q, k, v, topk_idx, vbs, out, lse, B, S, H, Nq, topk, sm_scale, precise, err, stream));
-    if (pair_kernel && vsa::fwd_pair_supported(Nq, topk))
-        return launch_status(vsa::launch_fwd_pair(q, k, v, topk_idx, vbs, plan, out, lse, B, S, H, Nq, topk, sm_scale,
-                                                  precise, err, stream));
-    return launch_status(
-        vsa::launch_fwd_tc(q, k, v, topk_idx, vbs, out, lse, B, S, H, Nq, topk, sm_scale, precise, err, stream));
+    return launch_status(vsa::launch_fwd_pair(q, k, v, topk_idx, vbs, plan, out, lse, B, S, H, Nq, topk, sm_scale,
+                                              precise, err, stream));
 }
 
 }  // namespace
+
+namespace vsa {
+
+// The checks of vsa_route other than its workspace, in the same order.
+int route_check_args(const uint16_t* q, const uint16_t* k, const int32_t* vbs, const int32_t* topk_idx, int B, int S,
+                     int H, int D, int Nq, int topk)
+{
+    int rc = check_bshd(B, S, H, D, Nq);
+    if (rc != VSA_OK) return rc;
+    if (topk < 1 || topk > Nq || Nq > 4096) return VSA_ERR_ARG;
+    if (!q || !k || !vbs || !topk_idx) return VSA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(vbs) || !aligned16(topk_idx)) return VSA_ERR_ALIGN;
+    return check_arch();
+}
+
+}  // namespace vsa
 
 extern "C" {
 
@@ -218,7 +233,8 @@ int vsa_cube_counts(int T, int Hh, int W, int32_t* vbs_host, int* Nq_out)
     return VSA_OK;
 }
 
-static int check_tile_args(const void* a, const void* b, int B, int T, int Hh, int W, int H, int D)
+// Sizes and the two pointers of a layout transform (no device query).
+static int check_tile_pair(const void* a, const void* b, int B, int T, int Hh, int W, int H, int D)
 {
     if (B < 1 || T < 1 || Hh < 1 || W < 1 || H < 1 || D < 1) return VSA_ERR_ARG;
     if (((int64_t)H * D) % 8 != 0 || (int64_t)H * D > INT32_MAX) return VSA_ERR_ARG;
@@ -227,7 +243,13 @@ static int check_tile_args(const void* a, const void* b, int B, int T, int Hh, i
     if ((int64_t)B * 64 * nq * H * D > ((int64_t)1 << 40)) return VSA_ERR_ARG;
     if (!a || !b) return VSA_ERR_NULL;
     if (!aligned16(a) || !aligned16(b)) return VSA_ERR_ALIGN;
-    return check_arch();
+    return VSA_OK;
+}
+
+static int check_tile_args(const void* a, const void* b, int B, int T, int Hh, int W, int H, int D)
+{
+    const int rc = check_tile_pair(a, b, B, T, Hh, W, H, D);
+    return rc != VSA_OK ? rc : check_arch();
 }
 
 int vsa_tile(const vsa_bf16* x_grid, vsa_bf16* x_tiled, int B, int T, int Hh, int W, int H, int D,
@@ -246,12 +268,57 @@ int vsa_untile(const vsa_bf16* x_tiled, vsa_bf16* x_grid, int B, int T, int Hh, 
     return launch_status(vsa::launch_untile(x_tiled, x_grid, B, vsa::make_geom(T, Hh, W), H * D, stream));
 }
 
+int vsa_tile_qkv(const vsa_bf16* q_grid, const vsa_bf16* k_grid, const vsa_bf16* v_grid, vsa_bf16* q_tiled,
+                 vsa_bf16* k_tiled, vsa_bf16* v_tiled, const int32_t* vbs, vsa_bf16* qc, vsa_bf16* kc, int B, int T,
+                 int Hh, int W, int H, int D, cudaStream_t stream)
+{
+    const bool means = qc != nullptr || kc != nullptr;
+    if (means && (qc == nullptr || kc == nullptr)) return VSA_ERR_ARG;
+    if (means && D != 128) return VSA_ERR_ARG;
+    int rc;
+    if ((rc = check_tile_pair(q_grid, q_tiled, B, T, Hh, W, H, D)) != VSA_OK) return rc;
+    if ((rc = check_tile_pair(k_grid, k_tiled, B, T, Hh, W, H, D)) != VSA_OK) return rc;
+    if ((rc = check_tile_pair(v_grid, v_tiled, B, T, Hh, W, H, D)) != VSA_OK) return rc;
+    if (means) {
+        if (!vbs) return VSA_ERR_NULL;
+        if (!aligned16(vbs) || !aligned16(qc) || !aligned16(kc)) return VSA_ERR_ALIGN;
+    }
+    if ((rc = check_arch()) != VSA_OK) return rc;
+    int* err;
+    if ((rc = device_error_word(&err)) != VSA_OK) return rc;
+    vsa::TileJob job;
+    const vsa_bf16* src[3] = {q_grid, k_grid, v_grid};
+    vsa_bf16* dst[3] = {q_tiled, k_tiled, v_tiled};
+    for (int t = 0; t < 3; ++t) {
+        job.src[t] = reinterpret_cast<const uint4*>(src[t]);
+        job.dst[t] = reinterpret_cast<uint4*>(dst[t]);
+    }
+    job.means[0] = qc;
+    job.means[1] = kc;
+    job.means[2] = nullptr;
+    return launch_status(vsa::launch_tile_cubes(job, 3, vbs, B, vsa::make_geom(T, Hh, W), H, D, err, stream));
+}
+
+int vsa_route_means(const vsa_bf16* qc, const vsa_bf16* kc, int32_t* topk_idx, int B, int H, int D, int Nq, int topk,
+                    cudaStream_t stream)
+{
+    if (B < 1 || H < 1 || Nq < 1 || D != 128) return VSA_ERR_ARG;
+    if (topk < 1 || topk > Nq || Nq > 4096) return VSA_ERR_ARG;
+    if ((int64_t)B * H * Nq * topk > INT32_MAX) return VSA_ERR_ARG;
+    if (!qc || !kc || !topk_idx) return VSA_ERR_NULL;
+    if (!aligned16(qc) || !aligned16(kc) || !aligned16(topk_idx)) return VSA_ERR_ALIGN;
+    const int rc = check_arch();
+    if (rc != VSA_OK) return rc;
+    return launch_status(vsa::launch_score_topk(qc, kc, topk_idx, B, H, Nq, topk, stream));
+}
+
 int vsa_stall_check(int* result, cudaStream_t stream)
 {
     if (result == nullptr) return VSA_ERR_NULL;
-    int* err;
-    const int rc = device_error_word(&err);
+    int rc = check_arch();
     if (rc != VSA_OK) return rc;
+    int* err;
+    if ((rc = device_error_word(&err)) != VSA_OK) return rc;
     return launch_status(vsa::launch_stall_check(err, result, stream));
 }
 

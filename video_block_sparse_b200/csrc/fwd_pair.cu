@@ -133,7 +133,7 @@ struct Layout {
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-template <bool NEG>
+template <bool NEG, bool PRECISE>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv, const int32_t* __restrict__ topk_idx,
@@ -384,7 +384,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait_warp(&bb.p_full[sb], par, &m.abort, err)) { aborted = true; break; }
                 tc_fence_after();
                 // k-steps (16 keys) 0..ceil16(na)-1 of half 0 and 4..4+ceil16(nb)-1 of half 1; the
-                // bf16 P of key half h sits in the first 32 columns of that half's 64
+                // bf16 P of key half h sits in the first 32 columns of that half's 64 (precise
+                // mode: the high and low parts of 32-key chunk c in columns 32 c .. +15, +16 .. +31)
                 const uint32_t kmask = ((1u << ((na + 15) >> 4)) - 1u) | (((1u << ((nb + 15) >> 4)) - 1u) << 4);
                 const uint32_t p_tmem = tbase + 128u * sb;
                 if (sw_flags(meta) & 1) o_init = false;
@@ -392,8 +393,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int kstep = 0; kstep < 8; ++kstep) {
                     const uint32_t on = (kmask >> kstep) & 1u;  // warp-uniform, no branch
-                    const uint32_t a_col = kstep < 4 ? 8u * kstep : 64u + 8u * (kstep - 4);
-                    umma_ts_elect_if(o_tmem, p_tmem + a_col, d_hi | (vl + ((kstep * 2048) >> 4)), idesc_pv, acc, on);
+                    const uint64_t vdesc = d_hi | (vl + ((kstep * 2048) >> 4));
+                    if (PRECISE) {
+                        // the weights of keys 16 kstep .. +15: high bf16 part, then the low part
+                        const uint32_t a_col = 32u * (kstep >> 1) + 8u * (kstep & 1);
+                        umma_ts_elect_if(o_tmem, p_tmem + a_col, vdesc, idesc_pv, acc, on);
+                        acc |= on;
+                        umma_ts_elect_if(o_tmem, p_tmem + a_col + 16u, vdesc, idesc_pv, acc, on);
+                    } else {
+                        const uint32_t a_col = kstep < 4 ? 8u * kstep : 64u + 8u * (kstep - 4);
+                        umma_ts_elect_if(o_tmem, p_tmem + a_col, vdesc, idesc_pv, acc, on);
+                    }
                     acc |= on;
                 }
                 o_init = o_init || kmask != 0;
@@ -571,13 +581,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
             // pass 2: P = exp2(x - m) as bf16 pairs; chunk ch's P goes to columns
             // 64 (ch / 2) + 16 (ch % 2): each half's P fills the half's first 32
-            // columns, over logits already consumed
+            // columns, over logits already consumed.  Precise mode: P = hi + lo, two
+            // bf16 parts (lo = bf16(P - hi), so hi + lo is within 2^-17 of P) in the
+            // chunk's own columns 32 ch .. +15 and +16 .. +31
             const float mu = m_run == -INFINITY ? 0.f : m_run;
             float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll 1
             for (int ch = 0; ch < 4; ++ch) {
                 const int nv = (ch < 2 ? nv0 : nv1) - 32 * (ch & 1);
-                uint32_t pk[16];
+                uint32_t pk[16], pl[16];
                 if (nv > 0) {
                     float sc[32];
                     tmem_ld32(s_addr + 32 * ch, reinterpret_cast<uint32_t*>(sc));
@@ -599,14 +611,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                             p0 = ex2(x0);
                             p1 = ex2(x1);
                         }
-                        fadd2(ls0, ls1, p0, p1);
                         pk[c] = pack_bf16(p0, p1);
+                        const float h0 = __uint_as_float(pk[c] << 16), h1 = __uint_as_float(pk[c] & 0xffff0000u);
+                        if (PRECISE) {
+                            pl[c] = pack_bf16(p0 - h0, p1 - h1);  // the differences are exact in fp32
+                            fadd2(ls0, ls1, p0, p1);
+                        } else {
+                            // the row sum adds the bf16 weights the P.V product sees, so that
+                            // numerator and denominator carry the same rounding
+                            fadd2(ls0, ls1, h0, h1);
+                        }
                     }
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) pk[c] = 0u;
+                    for (int c = 0; c < 16; ++c) pk[c] = pl[c] = 0u;
                 }
-                tmem_st16(s_addr + 64 * (ch >> 1) + 16 * (ch & 1), pk);
+                if (PRECISE) {
+                    tmem_st16(s_addr + 32 * ch, pk);
+                    tmem_st16(s_addr + 32 * ch + 16, pl);
+                } else {
+                    tmem_st16(s_addr + 64 * (ch >> 1) + 16 * (ch & 1), pk);
+                }
             }
             tmem_st_wait();
             tc_fence_before();
@@ -655,12 +680,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kWarpMma) tmem_dealloc(tbase, 512);
 }
 
-template <bool NEG>
+template <bool NEG, bool PRECISE>
 cudaError_t launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const int32_t* topk_idx,
                    const int32_t* vbs, const int32_t* plan, uint16_t* out, float* lse, int B, int S, int H, int nq,
                    int topk, float scale_log2, int* err, cudaStream_t s)
 {
-    auto kern = fwd_pair_kernel<NEG>;
+    auto kern = fwd_pair_kernel<NEG, PRECISE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Layout::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
@@ -682,16 +707,18 @@ cudaError_t launch_fwd_pair(const uint16_t* q, const uint16_t* k, const uint16_t
                             const int32_t* vbs, const int32_t* plan, uint16_t* out, float* lse, int B, int S, int H,
                             int nq, int topk, float sm_scale, bool precise_p, int* err, cudaStream_t s)
 {
-    if (precise_p)
-        return launch_fwd_pair_shared(q, k, v, topk_idx, vbs, plan, out, lse, B, S, H, nq, topk, sm_scale, true, err, s);
     CUtensorMap mq, mk, mv;
     const int64_t tokens = (int64_t)B * S;
     if (!make_map(&mq, q, tokens, H) || !make_map(&mk, k, tokens, H) || !make_map(&mv, v, tokens, H))
         return cudaErrorInvalidValue;
     const float scale_log2 = sm_scale * 1.4426950408889634f;
+    if (precise_p)
+        return scale_log2 < 0.f
+                   ? launch<true, true>(mq, mk, mv, topk_idx, vbs, plan, out, lse, B, S, H, nq, topk, scale_log2, err, s)
+                   : launch<false, true>(mq, mk, mv, topk_idx, vbs, plan, out, lse, B, S, H, nq, topk, scale_log2, err, s);
     return scale_log2 < 0.f
-               ? launch<true>(mq, mk, mv, topk_idx, vbs, plan, out, lse, B, S, H, nq, topk, scale_log2, err, s)
-               : launch<false>(mq, mk, mv, topk_idx, vbs, plan, out, lse, B, S, H, nq, topk, scale_log2, err, s);
+               ? launch<true, false>(mq, mk, mv, topk_idx, vbs, plan, out, lse, B, S, H, nq, topk, scale_log2, err, s)
+               : launch<false, false>(mq, mk, mv, topk_idx, vbs, plan, out, lse, B, S, H, nq, topk, scale_log2, err, s);
 }
 
 }  // namespace vsa

@@ -1,5 +1,4 @@
-// Device helpers shared by the paired-tile forward kernels (fwd_pair.cu and
-// fwd_pair_precise.cu): step descriptors, bounded mbarrier waits, tcgen05 /
+// Device helpers of the paired-tile forward kernel (fwd_pair.cu): step descriptors, bounded mbarrier waits, tcgen05 /
 // TMEM wrappers, packed fp32 pair arithmetic, the tile list generator (the
 // union of two selection lists, shared cubes first) and the TMA tensor maps.
 // Everything lives in an anonymous namespace: each kernel file gets its own

@@ -219,8 +219,22 @@ __device__ void select_row(const uint64_t* __restrict__ keys, int n, int topk, i
     __syncwarp();
 }
 
+// Scoring threads: kQH groups of query cubes x kKG groups of key cubes.  A
+// thread keeps a kQT x kJT block of (query, key) sums in registers: every q
+// element read from shared memory feeds kJT FMAs and every k element loaded
+// feeds kQT, so shared-memory reads stay below the FP64 pipe's rate.  Every
+// (query, key) sum still runs over d = 0..127 in order.
+constexpr int kJT = 4;
+constexpr int kKG = 160;  // key groups of kJT cubes (624 cubes: one pass)
 template <int QB>
-__global__ void __launch_bounds__(256) score_topk_kernel(const uint16_t* __restrict__ qc,
+struct ScoreShape {
+    static constexpr int kQT = QB < 4 ? QB : 4;  // query cubes per thread
+    static constexpr int kQH = QB / kQT;         // query groups
+    static constexpr int kThreads = kQH * kKG;
+};
+
+template <int QB>
+__global__ void __launch_bounds__(ScoreShape<QB>::kThreads) score_topk_kernel(const uint16_t* __restrict__ qc,
                                                          const uint16_t* __restrict__ kc, int32_t* __restrict__ topk_idx,
                                                          int H, int nq, int ns, int topk, int sel_warps)
 {
@@ -239,16 +253,14 @@ __global__ void __launch_bounds__(256) score_topk_kernel(const uint16_t* __restr
     }
     __syncthreads();
 
-    // Each thread scores kJT consecutive key cubes against the CTA's QB query
-    // cubes, so that every q element read from shared memory feeds kJT FMAs
-    // (two at QB = 8: four would cost occupancy).  Every (query, key) sum still
-    // runs over d = 0..127 in order.
-    constexpr int kJT = QB >= 8 ? 2 : 4;
+    constexpr int kQT = ScoreShape<QB>::kQT;
+    const int qg = threadIdx.x / kKG, kg = threadIdx.x % kKG;
+    const double* qrow = qd + qg * kQT * kD;
     const uint4* krow = reinterpret_cast<const uint4*>(kc + head * nq * kD);
-    for (int j0 = threadIdx.x * kJT; j0 < nq; j0 += blockDim.x * kJT) {
-        double acc[QB][kJT];
+    for (int j0 = kg * kJT; j0 < nq; j0 += kKG * kJT) {
+        double acc[kQT][kJT];
 #pragma unroll
-        for (int r = 0; r < QB; ++r)
+        for (int r = 0; r < kQT; ++r)
 #pragma unroll
             for (int t = 0; t < kJT; ++t) acc[r][t] = 0.0;
         for (int ch = 0; ch < kD / 8; ++ch) {
@@ -268,8 +280,8 @@ __global__ void __launch_bounds__(256) score_topk_kernel(const uint16_t* __restr
                 for (int t = 0; t < kJT; ++t)
                     kv[t] = bf16_to_f64((e & 1) ? (p[t][e >> 1] >> 16) : (p[t][e >> 1] & 0xFFFFu));
 #pragma unroll
-                for (int r = 0; r < QB; ++r) {
-                    const double qv = qd[r * kD + ch * 8 + e];
+                for (int r = 0; r < kQT; ++r) {
+                    const double qv = qrow[r * kD + ch * 8 + e];
 #pragma unroll
                     for (int t = 0; t < kJT; ++t) acc[r][t] = __fma_rn(qv, kv[t], acc[r][t]);
                 }
@@ -279,7 +291,7 @@ __global__ void __launch_bounds__(256) score_topk_kernel(const uint16_t* __restr
         for (int t = 0; t < kJT; ++t)
             if (j0 + t < nq)
 #pragma unroll
-                for (int r = 0; r < QB; ++r) keys[r * nq + j0 + t] = score_key(acc[r][t]);
+                for (int r = 0; r < kQT; ++r) keys[(qg * kQT + r) * nq + j0 + t] = score_key(acc[r][t]);
     }
     __syncthreads();
 
@@ -300,14 +312,9 @@ size_t route_workspace_bytes(int B, int H, int nq, int D)
     return 2 * (size_t)B * H * nq * D * sizeof(uint16_t);
 }
 
-cudaError_t launch_route(const uint16_t* q, const uint16_t* k, const int32_t* vbs, int32_t* topk_idx, int B, int S,
-                         int H, int nq, int topk, void* workspace, int* err, cudaStream_t s)
+cudaError_t launch_score_topk(const uint16_t* qc, const uint16_t* kc, int32_t* topk_idx, int B, int H, int nq,
+                              int topk, cudaStream_t s)
 {
-    uint16_t* qc = static_cast<uint16_t*>(workspace);
-    uint16_t* kc = qc + (size_t)B * H * nq * kD;
-    cube_mean_kernel<<<dim3(nq, B, 2), 128, 0, s>>>(q, k, vbs, qc, kc, S, H, nq, err);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
     int ns = 32;  // selection buffer: topk rounded up to a power of two
     while (ns < topk) ns <<= 1;
     // rows per CTA and selecting warps sized to the shared-memory budget
@@ -319,23 +326,35 @@ cudaError_t launch_route(const uint16_t* q, const uint16_t* k, const int32_t* vb
     int w = qb;
     while (w > 1 && smem_for(qb, w) > budget) w >>= 1;
     const size_t smem = smem_for(qb, w);
+    cudaError_t e;
     if (qb == 8) {
         auto kern = score_topk_kernel<8>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kern<<<dim3((nq + 7) / 8, H, B), 256, smem, s>>>(qc, kc, topk_idx, H, nq, ns, topk, w);
+        kern<<<dim3((nq + 7) / 8, H, B), ScoreShape<8>::kThreads, smem, s>>>(qc, kc, topk_idx, H, nq, ns, topk, w);
     } else if (qb == 4) {
         auto kern = score_topk_kernel<4>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kern<<<dim3((nq + 3) / 4, H, B), 256, smem, s>>>(qc, kc, topk_idx, H, nq, ns, topk, w);
+        kern<<<dim3((nq + 3) / 4, H, B), ScoreShape<4>::kThreads, smem, s>>>(qc, kc, topk_idx, H, nq, ns, topk, w);
     } else {
         auto kern = score_topk_kernel<2>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kern<<<dim3((nq + 1) / 2, H, B), 256, smem, s>>>(qc, kc, topk_idx, H, nq, ns, topk, w);
+        kern<<<dim3((nq + 1) / 2, H, B), ScoreShape<2>::kThreads, smem, s>>>(qc, kc, topk_idx, H, nq, ns, topk, w);
     }
     return cudaGetLastError();
+}
+
+cudaError_t launch_route(const uint16_t* q, const uint16_t* k, const int32_t* vbs, int32_t* topk_idx, int B, int S,
+                         int H, int nq, int topk, void* workspace, int* err, cudaStream_t s)
+{
+    uint16_t* qc = static_cast<uint16_t*>(workspace);
+    uint16_t* kc = qc + (size_t)B * H * nq * kD;
+    cube_mean_kernel<<<dim3(nq, B, 2), 128, 0, s>>>(q, k, vbs, qc, kc, S, H, nq, err);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_score_topk(qc, kc, topk_idx, B, H, nq, topk, s);
 }
 
 }  // namespace vsa

@@ -13,10 +13,13 @@
 // this library's module holds kScratchBytes of it until the process exits.
 // Host code cannot use the variable's name as a device address, so the first
 // call on each device looks the address up with cudaGetSymbolAddress (with
-// that device current) and caches it.
+// that device current) and caches it.  The cache slots are atomics: host
+// threads making their first calls at the same time store the same address.
 #include "vsa.h"
 
 #include "internal.h"
+
+#include <atomic>
 
 namespace {
 
@@ -28,7 +31,7 @@ constexpr size_t kScratchBytes = size_t(16) << 20;
 static __device__ __align__(256) unsigned char g_route_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
-void* g_scratch_addr[kMaxDevices];
+std::atomic<void*> g_scratch_addr[kMaxDevices];
 
 }  // namespace
 
@@ -37,19 +40,21 @@ extern "C" {
 VSA_API int vsa_route_noalloc(const vsa_bf16* q, const vsa_bf16* k, const int32_t* vbs, int32_t* topk_idx, int B,
                               int S, int H, int D, int Nq, int topk, cudaStream_t stream)
 {
-    const size_t need = vsa_route_workspace_size(B, H, Nq, D);
-    if (need == 0) return VSA_ERR_ARG;
-    if (need > kScratchBytes) return VSA_ERR_WORKSPACE;  // the fixed array is too small for this problem
+    // vsa_route's own checks first (arguments, then the device's architecture),
+    // so that a bad call gets the same error as from vsa_route
+    const int rc = vsa::route_check_args(q, k, vbs, topk_idx, B, S, H, D, Nq, topk);
+    if (rc != VSA_OK) return rc;
+    if (vsa_route_workspace_size(B, H, Nq, D) > kScratchBytes) return VSA_ERR_WORKSPACE;  // the array is too small
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return VSA_ERR_LAUNCH;
-    if (g_scratch_addr[dev] == nullptr) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || p == nullptr) return VSA_ERR_LAUNCH;
-        g_scratch_addr[dev] = p;
+    void* scratch = g_scratch_addr[dev].load(std::memory_order_relaxed);
+    if (scratch == nullptr) {
+        if (cudaGetSymbolAddress(&scratch, g_route_scratch) != cudaSuccess || scratch == nullptr) return VSA_ERR_LAUNCH;
+        g_scratch_addr[dev].store(scratch, std::memory_order_relaxed);
     }
-    // vsa_route validates every argument and overwrites the whole scratch
-    // region it uses before reading it, so no clearing is needed here.
-    return vsa_route(q, k, vbs, topk_idx, B, S, H, D, Nq, topk, g_scratch_addr[dev], kScratchBytes, stream);
+    // vsa_route overwrites the whole scratch region it uses before reading it,
+    // so no clearing is needed here.
+    return vsa_route(q, k, vbs, topk_idx, B, S, H, D, Nq, topk, scratch, kScratchBytes, stream);
 }
 
 }  // extern "C"
