@@ -33,12 +33,14 @@
 //               whose running offset rose, once the previous PV has finished;
 //               at a tile's end, O / l -> out and the log-sum-exp -> lse
 //   warp 16     TMA producer of Q and K: builds each tile's step list (shared
-//               cubes first), streams Q (one buffer) and K pairs (ring of 2)
-//               and posts each step's V pair to warp 18
+//               cubes first) from lists copied in one tile ahead, streams Q
+//               (one buffer; loaded after the tile's first K pair) and K pairs
+//               (ring of 3) and posts each step's V pair to warp 18
 //   warp 17     PV MMA issuer (the whole warp runs the schedule, one elected
 //               lane issues); zeroes V pad rows inside a partial k-step before
 //               the product; owns the TMEM allocation
-//   warp 18     TMA producer of V pairs (ring of 3)
+//   warp 18     TMA producer of V pairs (ring of 2: a V pair is needed only
+//               after its step's softmax, so it has two steps to land)
 //   warp 19     QK MMA issuer
 //
 // Softmax.  Logits in base 2 (x = s * sm_scale * log2 e).  Keys at or beyond
@@ -68,8 +70,9 @@ constexpr int kWarpVProd = 18;
 constexpr int kWarpQk = 19;  // kWarpMma issues the PV products, kWarpQk the QK products
 constexpr int kThreads = 20 * 32;
 constexpr int kVReq = 4;  // ring of V load requests from the K producer to the V producer
-constexpr int kSBuf = 3;  // S/P buffers in TMEM (also the V ring depth)
-constexpr int kKBuf = 2;  // K ring depth
+constexpr int kSBuf = 3;  // S/P buffers in TMEM
+constexpr int kKBuf = 3;  // K ring depth
+constexpr int kVBuf = 2;  // V ring depth
 constexpr uint32_t kOCol = 384;
 constexpr uint32_t kFinal = 1u << 22;  // step word: last step of the CTA's last tile
 
@@ -86,7 +89,7 @@ constexpr uint32_t kPolyPairs = VSA_POLY_PAIRS;
 struct Bars {
     uint64_t q_full, q_empty;                // Q tile landed / last QK of the tile done
     uint64_t k_full[kKBuf], k_empty[kKBuf];  // K pair landed / its QK done
-    uint64_t v_full[kSBuf], v_empty[kSBuf];  // V pair landed / its PV done
+    uint64_t v_full[kVBuf], v_empty[kVBuf];  // V pair landed / its PV done
     uint64_t s_full[kSBuf];  // step word published + QK done (2 arrivals)
     uint64_t a_full[kSBuf];  // offsets decided (the 128 threads of the step's softmax warps)
     uint64_t p_full[kSBuf];  // P written (128 softmax threads) and O corrected (128)
@@ -104,7 +107,7 @@ struct Bars {
 struct Misc {
     Bars bar;
     int4 vreq[kVReq];        // V load request: first token of cube a (-1: none), of cube b, head, step word
-    uint32_t v_meta[kSBuf];  // step word of the V pair in each V buffer
+    uint32_t v_meta[kVBuf];  // step word of the V pair in each V buffer
     uint32_t k_meta[kKBuf];  // step word of the K pair in each K buffer
     uint32_t s_meta[kSBuf];  // step word of each S buffer
     uint32_t tmem_base;
@@ -119,15 +122,16 @@ struct Misc {
     float mfin[2][128];                   // [tile parity][row]: running offset at the tile's end
     uint32_t bits1[kMaxNq / 32];          // membership bitmaps of the tile's two lists
     uint32_t bits2[kMaxNq / 32];
-    int32_t list1[kMaxTopk];              // the tile's two selection lists
-    int32_t list2[kMaxTopk];
+    int32_t list1[2][kMaxTopk];           // [tile parity]: the tile's two selection lists
+    int32_t list2[2][kMaxTopk];           // (the next tile's are copied in while this one runs)
+    uint8_t vbs8[kMaxNq];                 // the valid counts (255: out of range)
 };
 
 struct Layout {
     static constexpr uint32_t Q_OFF = 0;                           // Q tile
     static constexpr uint32_t K_OFF = Q_OFF + kTileBytes;          // K ring
     static constexpr uint32_t V_OFF = K_OFF + kKBuf * kTileBytes;  // V ring
-    static constexpr uint32_t TILE_BYTES = V_OFF + kSBuf * kTileBytes;
+    static constexpr uint32_t TILE_BYTES = V_OFF + kVBuf * kTileBytes;
     static constexpr uint32_t MISC_BYTES = (sizeof(Misc) + 1023) / 1024 * 1024;
     static constexpr uint32_t SMEM_BYTES = MISC_BYTES + TILE_BYTES + 1024;  // + alignment slack
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -166,9 +170,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bb.k_full[i], 1);
             mbar_init(&bb.k_empty[i], 1);
         }
-        for (int i = 0; i < kSBuf; ++i) {
+        for (int i = 0; i < kVBuf; ++i) {
             mbar_init(&bb.v_full[i], 1);
             mbar_init(&bb.v_empty[i], 1);
+        }
+        for (int i = 0; i < kSBuf; ++i) {
             mbar_init(&bb.s_full[i], 2);    // MMA warp (step word) + QK completion
             mbar_init(&bb.a_full[i], 128);  // the four softmax warps of the step
             mbar_init(&bb.p_full[i], 256);  // those and every correction thread
@@ -195,6 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         m.end_g = 0x7fffffff;
         fence_mbar_init();
     }
+    vbs_stage(vbs, nq, m.vbs8);
     if (warp == kWarpMma) {
         tmem_alloc(&m.tmem_base, 512);
         tmem_relinquish();
@@ -218,30 +225,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         int armed_q = -1, armed_k = -1, armed_kb = 0;
         bool aborted = false;
         uint8_t* qdst = tiles_ptr + L::Q_OFF;
+        TileRef t_next;
+        if (my_tiles > 0) {
+            t_next = checked_tile(blockIdx.x, H, nq, tiles_per_bh, plan, lane == 0 ? err : nullptr);
+            lists_fetch(t_next, topk_idx, H, nq, topk, m.list1[0], m.list2[0], lane);
+        }
         for (int n = 0; n < my_tiles && !aborted; ++n) {
-            const TileRef t =
-                checked_tile(blockIdx.x + n * gridDim.x, H, nq, tiles_per_bh, plan, lane == 0 ? err : nullptr);
-            gen_start(gen, t, topk_idx, vbs, H, nq, topk, m.list1, m.list2, m.bits1, m.bits2, err, lane);
+            const TileRef t = t_next;
+            int32_t* l1 = m.list1[n & 1];
+            int32_t* l2 = m.list2[n & 1];
+            gen_start(gen, t, m.vbs8, nq, topk, l1, l2, m.bits1, m.bits2, err, lane);
             const int tok0 = t.b * S;
-            if (lane == 0) {
-                if (wait_bar(&bb.q_empty, (n & 1) ^ 1, &m.abort, err)) {
-                    mbar_expect_tx(&bb.q_full, 2 * kHalfBox * ((t.i1 >= 0) + (t.i2 >= 0)));
-                    armed_q = n & 1;
-                    if (t.i1 >= 0) load_cube(&tmq, &bb.q_full, qdst, 0, t.h, tok0 + 64 * t.i1);
-                    if (t.i2 >= 0) load_cube(&tmq, &bb.q_full, qdst, 1, t.h, tok0 + 64 * t.i2);
-                } else {
-                    aborted = true;
-                }
-            }
-            aborted = __shfl_sync(0xffffffffu, aborted, 0);
+            bool q_pending = true;  // Q is loaded after the tile's first K pair (which needs no Q buffer)
             bool first = true;
             while (!aborted) {
                 const Entry ea = gen.next;
                 Entry eb{0, 0, 0};
                 if (ea.mem != 0) {
-                    gen.next = gen_pull(gen, m.list1, m.list2, m.bits1, m.bits2, vbs, lane);
+                    gen.next = gen_pull(gen, l1, l2, m.bits1, m.bits2, m.vbs8, lane);
                     eb = gen.next;
-                    if (eb.mem != 0) gen.next = gen_pull(gen, m.list1, m.list2, m.bits1, m.bits2, vbs, lane);
+                    if (eb.mem != 0) gen.next = gen_pull(gen, l1, l2, m.bits1, m.bits2, m.vbs8, lane);
                 }
                 const bool last = gen.next.mem == 0;
                 StepMeta meta;
@@ -277,12 +280,40 @@ __global__ void __launch_bounds__(kThreads, 1)
                     } else {
                         aborted = true;
                     }
+                    // the tile's Q, once the previous tile's last QK has released the buffer
+                    if (!aborted && q_pending) {
+                        if (wait_bar(&bb.q_empty, (n & 1) ^ 1, &m.abort, err)) {
+                            mbar_expect_tx(&bb.q_full, 2 * kHalfBox * ((t.i1 >= 0) + (t.i2 >= 0)));
+                            armed_q = n & 1;
+                            if (t.i1 >= 0) load_cube(&tmq, &bb.q_full, qdst, 0, t.h, tok0 + 64 * t.i1);
+                            if (t.i2 >= 0) load_cube(&tmq, &bb.q_full, qdst, 1, t.h, tok0 + 64 * t.i2);
+                        } else {
+                            aborted = true;
+                        }
+                    }
                 }
+                if (q_pending && n + 1 < my_tiles) {
+                    // the next tile, once this one's first loads are out: its lists copied
+                    // into the other list buffer and its Q cubes prefetched into L2
+                    t_next = checked_tile(blockIdx.x + (n + 1) * gridDim.x, H, nq, tiles_per_bh, plan,
+                                          lane == 0 ? err : nullptr);
+                    lists_fetch(t_next, topk_idx, H, nq, topk, m.list1[(n + 1) & 1], m.list2[(n + 1) & 1], lane);
+                    if (lane == 0) {
+                        for (int s = 0; s < 2; ++s) {
+                            const int i = s == 0 ? t_next.i1 : t_next.i2;
+                            if (i < 0) continue;
+                            tma_prefetch_3d(&tmq, 0, t_next.h, t_next.b * S + 64 * i);
+                            tma_prefetch_3d(&tmq, 64, t_next.h, t_next.b * S + 64 * i);
+                        }
+                    }
+                }
+                q_pending = false;
                 aborted = __shfl_sync(0xffffffffu, aborted, 0);
                 ++kc;
                 if (last) break;
             }
         }
+        cp_async_wait_all();  // a list copy still in flight after an abort
         if (aborted && lane == 0) {
             // copies issued by this thread must land before the CTA's shared memory goes away
             if (armed_q >= 0) drain_wait(&bb.q_full, armed_q);
@@ -292,15 +323,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ TMA producer of V
         int armed_v = -1, armed_vb = 0;
         for (int vc = 0; my_tiles > 0 && lane == 0; ++vc) {
-            const int vr = vc % kVReq, vb = vc % kSBuf;
+            const int vr = vc % kVReq, vb = vc % kVBuf;
             if (!wait_bar(&bb.vr_full[vr], (vc / kVReq) & 1, &m.abort, err)) break;
             const int4 rq = m.vreq[vr];
             mbar_arrive(&bb.vr_empty[vr]);
-            // the V buffer is free once the PV three steps back finished
-            if (!wait_bar(&bb.v_empty[vb], ((vc / kSBuf) & 1) ^ 1, &m.abort, err)) break;
+            // the V buffer is free once the PV two steps back finished
+            if (!wait_bar(&bb.v_empty[vb], ((vc / kVBuf) & 1) ^ 1, &m.abort, err)) break;
             m.v_meta[vb] = (uint32_t)rq.w;  // published by the arrival below
             mbar_expect_tx(&bb.v_full[vb], 2 * kHalfBox * ((rq.x >= 0) + (rq.y >= 0)));
-            armed_v = (vc / kSBuf) & 1;
+            armed_v = (vc / kVBuf) & 1;
             armed_vb = vb;
             uint8_t* vdst = tiles_ptr + L::V_OFF + vb * kTileBytes;
             if (rq.x >= 0) load_cube(&tmv, &bb.v_full[vb], vdst, 0, rq.z, rq.x);
@@ -361,18 +392,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t o_tmem = tbase + kOCol;
             bool o_init = false;
             for (int j = 0; my_tiles > 0; ++j) {
-                const int sb = j % kSBuf;
+                const int sb = j % kSBuf, vb = j % kVBuf;
                 const uint32_t par = (j / kSBuf) & 1;
-                if (!wait_warp(&bb.v_full[sb], par, &m.abort, err)) { aborted = true; break; }
+                if (!wait_warp(&bb.v_full[vb], (j / kVBuf) & 1, &m.abort, err)) { aborted = true; break; }
                 // everything that needs only the V pair is done before waiting for P
-                const uint32_t meta = m.v_meta[sb];
+                const uint32_t meta = m.v_meta[vb];
                 const int na = sw_na(meta), nb = sw_nb(meta);
-                const uint32_t vl = vl0 + ((uint32_t)sb * kTileBytes >> 4);
+                const uint32_t vl = vl0 + ((uint32_t)vb * kTileBytes >> 4);
                 const int za = (na & 15) ? 16 - (na & 15) : 0, zb = (nb & 15) ? 16 - (nb & 15) : 0;
                 if (za + zb > 0) {
                     // V rows between vbs and the next multiple of 16 are read by the last
                     // k-step of their cube: zero them (both d halves) before the product
-                    const uint32_t vbase = tiles + L::V_OFF + sb * kTileBytes;
+                    const uint32_t vbase = tiles + L::V_OFF + vb * kTileBytes;
                     for (int w = lane; w < (za + zb) * 16; w += 32) {
                         const int zr = w >> 4, chunk = w & 15;
                         const int row = zr < za ? na + zr : 64 + nb + (zr - za);
@@ -411,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // QK issuer's products go after it; the commits below track this warp's only)
                 tc_fence_before();
                 mbar_arrive_elect(&bb.pv_issued[sb]);
-                umma_commit_elect(&bb.v_empty[sb]);
+                umma_commit_elect(&bb.v_empty[vb]);
                 umma_commit_elect(&bb.pv_done[j & 1]);
                 umma_commit_elect_if(&bb.o_full, sw_flags(meta) & 2);
                 if (meta & kFinal) break;
@@ -429,6 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int qbit = r >> 6;
         const uint32_t oa = tbase + ((uint32_t)(32 * wq) << 16) + kOCol;
         int g = 0;
+        bool released = false;  // this tile's first step was released by the previous tile's epilogue
         for (int n = 0; n < my_tiles; ++n) {
             for (;;) {
                 const int b = g % kSBuf;
@@ -453,8 +485,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tmem_st_wait();
                 }
-                tc_fence_before();
-                mbar_arrive(&bb.p_full[b]);
+                if (!released) {
+                    tc_fence_before();
+                    mbar_arrive(&bb.p_full[b]);
+                }
+                released = false;
                 ++g;
                 if (sw_flags(meta) & 2) break;
             }
@@ -473,23 +508,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float inv = has ? __frcp_rn(l) : 0.f;
                 const int64_t token = (int64_t)t.b * S + 64LL * cube + (r & 63);
                 uint16_t* dst = out + (token * H + t.h) * kD;
-#pragma unroll 1
+                // read and round the whole row first ...
+                uint32_t pk[4][16];
+#pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
                     uint32_t o[32];
                     tmem_ld32(oa + 32 * c4, o);
                     tmem_ld_wait();
-                    if (cube >= 0) {
 #pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            uint32_t w[4];
+                    for (int e = 0; e < 16; ++e)
+                        pk[c4][e] = has ? pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv)
+                                        : 0u;
+                }
+                // ... so that the next tile's first product, which overwrites O, need not
+                // wait for the stores.  Every product of this tile has completed (o_full),
+                // so this arrival can only count toward the next step's phase.
+                if (n + 1 < my_tiles) {
+                    tc_fence_before();
+                    mbar_arrive(&bb.p_full[g % kSBuf]);
+                    released = true;
+                }
+                if (cube >= 0) {
 #pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                w[e] = has ? pack_bf16(__uint_as_float(o[8 * v + 2 * e]) * inv,
-                                                       __uint_as_float(o[8 * v + 2 * e + 1]) * inv)
-                                           : 0u;
-                            st_global_v4(dst + 32 * c4 + 8 * v, w[0], w[1], w[2], w[3]);
-                        }
-                    }
+                    for (int c4 = 0; c4 < 4; ++c4)
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            st_global_v4(dst + 32 * c4 + 8 * v, pk[c4][4 * v], pk[c4][4 * v + 1], pk[c4][4 * v + 2],
+                                         pk[c4][4 * v + 3]);
                 }
                 if (lse != nullptr && cube >= 0)
                     lse[((int64_t)t.b * H + t.h) * S + 64LL * cube + (r & 63)] =

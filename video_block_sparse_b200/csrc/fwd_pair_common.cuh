@@ -356,7 +356,7 @@ __device__ __forceinline__ bool test_bit(const uint32_t* bits, int j) { return (
 
 // Scan forward to the next qualifying entry (warp-uniform result).
 __device__ Entry gen_pull(ListGen& g, const int32_t* l1, const int32_t* l2, const uint32_t* b1, const uint32_t* b2,
-                          const int32_t* __restrict__ vbs, uint32_t lane)
+                          const uint8_t* vbs8, uint32_t lane)
 {
     Entry e{0, 0, 0};
     for (;;) {
@@ -373,7 +373,7 @@ __device__ Entry gen_pull(ListGen& g, const int32_t* l1, const int32_t* l2, cons
             bool q = false;
             if (idx < len) {
                 const int j = list[idx];
-                const int n = j >= 0 ? __ldg(vbs + j) : 0;
+                const int n = j >= 0 ? vbs8[j] : 0;
                 if (n > 0 && n <= 64) {
                     if (g.phase == 0)
                         q = g.dedupe && test_bit(b1, j);
@@ -392,18 +392,45 @@ __device__ Entry gen_pull(ListGen& g, const int32_t* l1, const int32_t* l2, cons
         const int idx = g.base - 32 + l;
         const int j = list[idx];
         e.j = j;
-        e.n = __ldg(vbs + j);
+        e.n = vbs8[j];
         e.mem = g.phase == 0 ? 3 : (g.phase == 1 ? 1 : 2);
         return e;
     }
 }
 
-// Stage a tile's lists and membership bitmaps in shared memory and prime the
-// generator.  Invalid cube ids latch an error and are dropped (stored as -1);
-// invalid vbs values latch an error and count as empty cubes.
-__device__ void gen_start(ListGen& g, const TileRef& t, const int32_t* __restrict__ topk_idx,
-                          const int32_t* __restrict__ vbs, int H, int nq, int topk, int32_t* l1, int32_t* l2,
-                          uint32_t* b1, uint32_t* b2, int* err, uint32_t lane)
+// The valid counts as bytes in shared memory (read for every list entry); a
+// count outside [0, 64] is kept as 255, which the list code treats as an
+// empty cube after latching the error.
+__device__ __forceinline__ void vbs_stage(const int32_t* __restrict__ vbs, int nq, uint8_t* vbs8)
+{
+    for (int c = threadIdx.x; c < nq; c += blockDim.x) {
+        const int n = __ldg(vbs + c);
+        vbs8[c] = (uint8_t)(n < 0 || n > 64 ? 255 : n);
+    }
+}
+
+// Copy a tile's two selection lists into shared memory asynchronously
+// (cp.async, one entry per lane and pass); gen_start waits for them.  Run one
+// tile ahead, so that the copies overlap the previous tile's steps.
+__device__ __forceinline__ void lists_fetch(const TileRef& t, const int32_t* __restrict__ topk_idx, int H, int nq,
+                                            int topk, int32_t* l1, int32_t* l2, uint32_t lane)
+{
+    for (int s = 0; s < 2; ++s) {
+        const int i = s == 0 ? t.i1 : t.i2;
+        if (i < 0) continue;
+        const int32_t* src = topk_idx + (((int64_t)t.b * H + t.h) * nq + i) * topk;
+        int32_t* dst = s == 0 ? l1 : l2;
+        for (int e = lane; e < topk; e += 32) cp_async4(dst + e, src + e);
+    }
+    cp_async_commit();
+}
+
+// Build a tile's membership bitmaps from its lists (fetched by lists_fetch)
+// and prime the generator.  Invalid cube ids latch an error and are dropped
+// (stored as -1); invalid vbs values latch an error and count as empty cubes.
+// vbs8: the valid counts staged in shared memory (vbs_stage).
+__device__ void gen_start(ListGen& g, const TileRef& t, const uint8_t* vbs8, int nq, int topk, int32_t* l1,
+                          int32_t* l2, uint32_t* b1, uint32_t* b2, int* err, uint32_t lane)
 {
     const int words = (nq + 31) >> 5;
     for (int w = lane; w < words; w += 32) {
@@ -412,35 +439,48 @@ __device__ void gen_start(ListGen& g, const TileRef& t, const int32_t* __restric
     }
     g.len1 = t.i1 >= 0 ? topk : 0;
     g.len2 = t.i2 >= 0 ? topk : 0;
+    cp_async_wait_all();
     __syncwarp();
-    bool dup = false;
+    // bitmaps by non-returning shared-memory ORs; a list names a cube twice iff
+    // its bitmap holds fewer bits than it has valid entries
+    int valid[2] = {0, 0};
     for (int s = 0; s < 2; ++s) {
         const int len = s == 0 ? g.len1 : g.len2;
         if (len == 0) continue;
-        const int i = s == 0 ? t.i1 : t.i2;
-        const int32_t* src = topk_idx + (((int64_t)t.b * H + t.h) * nq + i) * topk;
-        int32_t* dst = s == 0 ? l1 : l2;
+        int32_t* lst = s == 0 ? l1 : l2;
         uint32_t* bits = s == 0 ? b1 : b2;
         for (int e = lane; e < len; e += 32) {
-            int j = __ldg(src + e);
+            int j = lst[e];
             if (j < 0 || j >= nq) {
                 atomicCAS(err, 0, (int)kErrTopkIdx);
                 j = -1;
             } else {
-                const int n = __ldg(vbs + j);
-                if (n < 0 || n > 64) atomicCAS(err, 0, (int)kErrVbs);
-                const uint32_t old = atomicOr(&bits[j >> 5], 1u << (j & 31));
-                if (old & (1u << (j & 31))) dup = true;
+                if (vbs8[j] > 64) atomicCAS(err, 0, (int)kErrVbs);
+                atomicOr(&bits[j >> 5], 1u << (j & 31));  // result unused: a reduction
+                ++valid[s];
             }
-            dst[e] = j;
+            lst[e] = j;
         }
     }
     __syncwarp();
-    g.dedupe = !__any_sync(0xffffffffu, dup) && g.len1 > 0 && g.len2 > 0;
+    int set[2] = {0, 0};
+    for (int w = lane; w < words; w += 32) {
+        set[0] += __popc(b1[w]);
+        set[1] += __popc(b2[w]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        valid[0] += __shfl_xor_sync(0xffffffffu, valid[0], o);
+        valid[1] += __shfl_xor_sync(0xffffffffu, valid[1], o);
+        set[0] += __shfl_xor_sync(0xffffffffu, set[0], o);
+        set[1] += __shfl_xor_sync(0xffffffffu, set[1], o);
+    }
+    const bool dup = set[0] != valid[0] || set[1] != valid[1];
+    g.dedupe = !dup && g.len1 > 0 && g.len2 > 0;
     g.phase = g.dedupe ? 0 : 1;
     g.base = 0;
     g.mask = 0;
-    g.next = gen_pull(g, l1, l2, b1, b2, vbs, lane);
+    g.next = gen_pull(g, l1, l2, b1, b2, vbs8, lane);
 }
 
 // A tile with an out-of-range plan entry latches an error; the bad cube is dropped.
