@@ -1,7 +1,8 @@
 """Benchmark of the VSA fine stage on B200: one step = the whole hot path on
 one batch of synthetic Wan2.2 832x480/81f activations:
 
-    tile q, k, v (raster -> cube-major)  ->  route (cube-mean q.k top-k)
+    tile q, k, v (raster -> cube-major, one launch that also forms the cube
+    means of q and k)  ->  route (scores and top-k from those means)
     ->  plan (pair query cubes by selection overlap)
     ->  fine block-sparse attention forward  ->  untile the output
 
@@ -14,6 +15,12 @@ resident in HBM when the timed region starts; they are larger than L2
 
 Under torchrun every rank runs its own independent problem (weak scaling, no
 data-path collective); rank 0 prints one JSON line.
+
+Besides the headline, the line carries (rank 0, N=1): the forward with the
+consecutive pairing and on random selection lists of the same shape (how the
+paired kernel's speed depends on list overlap, with the steps per tile of
+each), and the forward alone at the other configurations (Wan 1280x720 CFG
+pair, the top-k sweep and the dense case); skip those with --no-extras.
 """
 from __future__ import annotations
 
@@ -44,7 +51,8 @@ def flops(cfg, S):
 
 def config_block(cfg, S):
     return {
-        "workload": "Wan2.2 T2V-A14B 832x480/81f VSA fine stage (tile q,k,v -> route -> plan -> fwd -> untile)",
+        "workload": "Wan2.2 T2V-A14B 832x480/81f VSA fine stage (tile q,k,v + cube means -> route -> plan -> fwd "
+                    "-> untile)",
         "B": cfg.B, "latent_grid": list(cfg.grid), "S_padded": S, "H": cfg.H, "D": 128, "topk": cfg.topk,
         "sm_scale": cfg.sm_scale, "global_batch": cfg.B, "seq_len": S, "parallelism": "replicas (independent problem per GPU)",
         "l2": "inputs larger than L2 (1.0 GB raster q,k,v read per step); no flush",
@@ -154,8 +162,8 @@ def run_gpu(args, rank, world, local_rank):
     vbs = vbs_h.to(dev)
     B, L, H, D = q_g.shape
     qt, kt, vt = (torch.empty(B, S, H, D, dtype=torch.bfloat16, device=dev) for _ in range(3))
+    qc, kc = (torch.empty(B, H, nq, D, dtype=torch.bfloat16, device=dev) for _ in range(2))
     idx = torch.empty(B, H, nq, cfg.topk, dtype=torch.int32, device=dev)
-    ws = torch.empty(vsa.route_workspace_size(B, H, nq, D), dtype=torch.uint8, device=dev)
     plan = torch.empty(B * H, (nq + 1) // 2, 2, dtype=torch.int32, device=dev)
     plan_ws = torch.empty(vsa.plan_workspace_size(B, H, nq, cfg.topk), dtype=torch.uint8, device=dev)
     out_t = torch.empty_like(qt)
@@ -165,20 +173,18 @@ def run_gpu(args, rank, world, local_rank):
     ev_f0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ev_f1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
 
-    def step(i=None):
-        vsa.tile(q_g, cfg.grid, out=qt)
-        vsa.tile(k_g, cfg.grid, out=kt)
-        vsa.tile(v_g, cfg.grid, out=vt)
-        vsa.route(qt, kt, vbs, cfg.topk, out=idx, workspace=ws)
+    def step(i=None, src=(q_g, k_g, v_g), dst=None):
+        vsa.tile_qkv(*src, cfg.grid, vbs, out=[qt, kt, vt, qc, kc])
+        vsa.route_means(qc, kc, cfg.topk, out=idx)
         vsa.plan(idx, out=plan, workspace=plan_ws)
         if i is not None:
             ev_f0[i].record(stream)
         vsa.fwd(qt, kt, vt, idx, vbs, cfg.sm_scale, out=out_t, lse=lse, plan=plan)
         if i is not None:
             ev_f1[i].record(stream)
-        vsa.untile(out_t, cfg.grid, out=out_g)
+        vsa.untile(out_t, cfg.grid, out=out_g if dst is None else dst)
 
-    launches_per_step = 3 + 2 + 3 + 1 + 1  # tile x3, route, plan, fwd, untile
+    launches_per_step = 1 + 1 + 3 + 1 + 1  # tile_qkv, route_means, plan (3 kernels), fwd, untile
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -253,13 +259,7 @@ def run_gpu(args, rank, world, local_rank):
             stream.wait_event(ev_in[i])
             if i >= 2:
                 stream.wait_event(ev_out[i - 2])  # out buffer read back
-            vsa.tile(qb, cfg.grid, out=qt)
-            vsa.tile(kb, cfg.grid, out=kt)
-            vsa.tile(vb, cfg.grid, out=vt)
-            vsa.route(qt, kt, vbs, cfg.topk, out=idx, workspace=ws)
-            vsa.plan(idx, out=plan, workspace=plan_ws)
-            vsa.fwd(qt, kt, vt, idx, vbs, cfg.sm_scale, out=out_t, lse=lse, plan=plan)
-            vsa.untile(out_t, cfg.grid, out=ob)
+            step(src=(qb, kb, vb), dst=ob)
             ev_done[i].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_done[i])
@@ -283,10 +283,111 @@ def run_gpu(args, rank, world, local_rank):
     ms_step = ms_total / args.steps
     ms_step, e2e_ms, fwd_avg, e2e_serial_ms = max_over_ranks(
         [ms_step, e2e_ms, statistics.mean(fwd_ms), e2e_serial_ms], dev)
+    extras = None
+    if world == 1 and args.extras:
+        extras = run_extras(vsa, dev, cfg, qt, kt, vt, qc, kc, idx, vbs, read_peaks()[0])
     return dict(cfg=cfg, S=S, ms_step=ms_step, e2e_ms=e2e_ms, e2e_serial_ms=e2e_serial_ms, fwd_ms=fwd_avg,
                 fwd_list=fwd_ms,
-                clocks=clk.summary(), launches=launches_per_step * args.steps,
+                clocks=clk.summary(), launches=launches_per_step * args.steps, extras=extras,
                 h2d=3 * q_h.numel() * 2, d2h=out_g.numel() * 2)
+
+
+# --------------------------------------------------------------------------- extras
+
+def steps_per_tile(idx: np.ndarray, plan: np.ndarray | None, vbs: np.ndarray) -> np.ndarray:
+    """Steps each tile of the paired forward walks: the distinct cubes with a valid
+    token that either list names (every entry when a list repeats a cube), two per step.
+    plan None: the consecutive pairing (2p, 2p + 1)."""
+    B, H, nq, topk = idx.shape
+    valid = vbs > 0
+    out = []
+    for bh in range(B * H):
+        lists = idx[bh // H, bh % H]
+        pairs = plan[bh] if plan is not None else [(2 * p, 2 * p + 1 if 2 * p + 1 < nq else -1)
+                                                   for p in range((nq + 1) // 2)]
+        for a, c in pairs:
+            la = lists[a][valid[lists[a]]]
+            if c < 0:
+                n = len(la)
+            else:
+                lc = lists[c][valid[lists[c]]]
+                dup = len(set(la.tolist())) < len(la) or len(set(lc.tolist())) < len(lc)
+                n = len(la) + len(lc) if dup else len(set(la.tolist()) | set(lc.tolist()))
+            out.append((n + 1) // 2)
+    return np.array(out)
+
+
+def time_fwd(vsa, args, n=10, warm=3):
+    """Average forward time (ms) over n calls, CUDA events on the current stream."""
+    for _ in range(warm):
+        vsa.fwd(*args[0], **args[1])
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for a, b in ev:
+        a.record()
+        vsa.fwd(*args[0], **args[1])
+        b.record()
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+
+def run_extras(vsa, dev, cfg, qt, kt, vt, qc, kc, idx, vbs, peak):
+    """The forward alone: the headline workload with the consecutive pairing and on
+    random selection lists, then the other configurations."""
+    out = torch.empty_like(qt)
+    vbs_h = vbs.cpu().numpy()
+    res = {}
+
+    def fwd_case(q, k, v, ix, vb, c, plan):
+        ms = time_fwd(vsa, ((q, k, v, ix, vb, c.sm_scale), {"out": out if out.shape == q.shape else None,
+                                                              "plan": plan}))
+        return ms
+
+    # pairing and overlap
+    ix_h = idx.cpu().numpy()
+    plan = vsa.plan(idx)
+    fl = flops(cfg, qt.shape[1])
+    cases = {}
+    for name, ix_dev, ix_np in (("routed", idx, ix_h),
+                                ("random_lists", None, synth.random_topk(11, cfg.B, cfg.H, len(vbs_h), cfg.topk))):
+        if ix_dev is None:
+            ix_dev = torch.from_numpy(ix_np).to(dev)
+        pl = vsa.plan(ix_dev)
+        row = {}
+        for tag, p in (("planned", pl), ("consecutive", None)):
+            ms = fwd_case(qt, kt, vt, ix_dev, vbs, cfg, p)
+            spt = steps_per_tile(ix_np, p.cpu().numpy() if p is not None else None, vbs_h)
+            row[tag] = {"fwd_ms": ms, "tflops": fl / (ms * 1e-3) / 1e12, "frac": fl / (ms * 1e-3) / 1e12 / peak,
+                        "steps_per_tile_mean": float(spt.mean()), "steps_total": int(spt.sum())}
+        cases[name] = row
+    res["pairing"] = cases
+
+    # other configurations: forward alone (inputs tiled and routed by the library first)
+    cfgs = {}
+    for name in ("sweep32", "sweep156", "sweep312", "dense624", "wan720"):
+        c = synth.CONFIGS[name]
+        if c.grid == cfg.grid and c.B == cfg.B and c.H == cfg.H:
+            q_, k_, v_, qc_, kc_, vb_ = qt, kt, vt, qc, kc, vbs
+        else:
+            T, Hh, W = c.grid
+            g = [synth.bits_to_torch(x).to(dev) for x in synth.grid_qkv(c)]
+            vb_ = vsa.cube_counts(T, Hh, W).to(dev)
+            q_, k_, v_, qc_, kc_ = vsa.tile_qkv(*g, c.grid, vb_)
+            del g
+        ix = vsa.route_means(qc_, kc_, c.topk)
+        pl = vsa.plan(ix)
+        o_ = torch.empty_like(q_)
+        ms = time_fwd(vsa, ((q_, k_, v_, ix, vb_, c.sm_scale), {"out": o_, "plan": pl}), n=5, warm=2)
+        f = flops(c, q_.shape[1])
+        spt = steps_per_tile(ix.cpu().numpy(), pl.cpu().numpy(), vb_.cpu().numpy())
+        cfgs[name] = {"B": c.B, "H": c.H, "latent_grid": list(c.grid), "S_padded": q_.shape[1], "topk": c.topk,
+                      "tflop_per_call": f / 1e12, "fwd_ms": ms, "tflops": f / (ms * 1e-3) / 1e12,
+                      "frac": f / (ms * 1e-3) / 1e12 / peak, "steps_per_tile_mean": float(spt.mean())}
+        del q_, k_, v_, o_
+    res["configs"] = cfgs
+    rc, detail = vsa.device_status()
+    if rc != 0:
+        raise RuntimeError(f"device error {rc}/{detail} in the extra cases")
+    return res
 
 
 # --------------------------------------------------------------------------- oracle timing
@@ -346,6 +447,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--oracle-seconds", type=float, default=15.0,
                     help="CPU time for the oracle baseline sample (0 skips it)")
+    ap.add_argument("--no-extras", dest="extras", action="store_false",
+                    help="skip the extra forward cases (pairing, random lists, other configurations)")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the head count (a smaller case for ncu captures; not a bench line)")
     args = ap.parse_args()
@@ -375,7 +478,9 @@ def main():
         line = {
             "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 0,
             "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": flops(cfg, S) / (value * 1e12) * 1e3, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": flops(cfg, S) / (value * 1e12) * 1e3,
+            "ms_per_step_source": "extrapolated: the workload's FLOPs over the rate of the timed sample",
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config_block(cfg, S),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": f"{items} query-cube work items of the workload (2 heads drawn), {secs:.1f} s"},
@@ -433,6 +538,8 @@ def main():
         "gpu_launches": res["launches"],
         "clocks": res["clocks"],
     }
+    if res["extras"] is not None:
+        line["fwd_extra"] = res["extras"]
     print(json.dumps(line))
 
 

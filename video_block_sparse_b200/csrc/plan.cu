@@ -72,6 +72,44 @@ __device__ __forceinline__ void cand_insert(int (&co)[kCand], int (&cj)[kCand], 
     cj[p] = j;
 }
 
+// Merge the 32 lanes' candidate lists (each sorted, larger overlap first, ties by
+// the smaller cube): kCand rounds of a warp-wide (max ov, min j) pick; lane 0
+// writes the winners (-1 where there are fewer than kCand), and their overlaps
+// if out_o is given.
+__device__ void warp_merge_cand(const int (&co)[kCand], const int (&cj)[kCand], int lane, int32_t* out_j,
+                                int32_t* out_o)
+{
+    int head = 0;
+    for (int c = 0; c < kCand; ++c) {
+        int ov = -1, j = 0x7fffffff;
+#pragma unroll
+        for (int q = 0; q < kCand; ++q)
+            if (q == head) {
+                ov = co[q];
+                j = cj[q];
+            }
+        // key: larger ov first, then smaller j
+        for (int s = 16; s >= 1; s >>= 1) {
+            const int ov2 = __shfl_xor_sync(0xffffffffu, ov, s);
+            const int j2 = __shfl_xor_sync(0xffffffffu, j, s);
+            if (ov2 > ov || (ov2 == ov && j2 < j)) {
+                ov = ov2;
+                j = j2;
+            }
+        }
+        // the owner of the winner advances its head
+        bool mine = false;
+#pragma unroll
+        for (int q = 0; q < kCand; ++q)
+            if (q == head && cj[q] == j && co[q] == ov) mine = true;
+        if (mine) ++head;
+        if (lane == 0) {
+            out_j[c] = ov >= 0 ? j : -1;
+            if (out_o != nullptr) out_o[c] = ov;
+        }
+    }
+}
+
 // CTA = (bh, 32 consecutive rows); warp w handles row i0 + w.  Column
 // bitmaps are staged through shared memory in chunks, each row padded with
 // zero words to ws words (a multiple of 4 with ws / 4 odd), so that the
@@ -124,38 +162,7 @@ __global__ void __launch_bounds__(1024) plan_cand_kernel(const uint32_t* __restr
         }
     }
     if (i >= nq) return;
-    // merge the 32 lanes' lists: kCand rounds of a warp-wide (max ov, min j) pick
-    int head = 0;
-    int32_t* out_j = cand + ((int64_t)bh * nq + i) * kCand;
-    int32_t* out_o = cand_ov + ((int64_t)bh * nq + i) * kCand;
-    for (int c = 0; c < kCand; ++c) {
-        int ov = -1, j = 0x7fffffff;
-#pragma unroll
-        for (int q = 0; q < kCand; ++q)
-            if (q == head) {
-                ov = co[q];
-                j = cj[q];
-            }
-        // key: larger ov first, then smaller j
-        for (int s = 16; s >= 1; s >>= 1) {
-            const int ov2 = __shfl_xor_sync(0xffffffffu, ov, s);
-            const int j2 = __shfl_xor_sync(0xffffffffu, j, s);
-            if (ov2 > ov || (ov2 == ov && j2 < j)) {
-                ov = ov2;
-                j = j2;
-            }
-        }
-        // the owner of the winner advances its head
-        bool mine = false;
-#pragma unroll
-        for (int q = 0; q < kCand; ++q)
-            if (q == head && cj[q] == j && co[q] == ov) mine = true;
-        if (mine) ++head;
-        if (lane == 0) {
-            out_j[c] = ov >= 0 ? j : -1;
-            out_o[c] = ov;
-        }
-    }
+    warp_merge_cand(co, cj, lane, cand + ((int64_t)bh * nq + i) * kCand, cand_ov + ((int64_t)bh * nq + i) * kCand);
 }
 
 // One CTA per (bh): proposal rounds over the candidate lists; refills while
@@ -187,9 +194,11 @@ __global__ void __launch_bounds__(1024) plan_match_kernel(int32_t* cand, const u
             __syncthreads();
             if (n_unpaired < 2) break;  // the same value in every thread
             // each unpaired cube's kCand candidates among the unpaired cubes
-            // (largest overlap first, ties by the smaller index, as plan_cand_kernel)
-            for (int i = threadIdx.x; i < nq; i += blockDim.x) {
-                if (partner[i] >= 0) continue;
+            // (largest overlap first, ties by the smaller index, as plan_cand_kernel):
+            // one warp per unpaired cube, its lanes over the other unpaired cubes
+            const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+            for (int i = warp; i < nq; i += (int)(blockDim.x >> 5)) {
+                if (partner[i] >= 0) continue;  // warp-uniform
                 int co[kCand], cj[kCand];
 #pragma unroll
                 for (int c = 0; c < kCand; ++c) {
@@ -197,15 +206,14 @@ __global__ void __launch_bounds__(1024) plan_match_kernel(int32_t* cand, const u
                     cj[c] = 0x7fffffff;
                 }
                 const uint32_t* bi = bbh + (int64_t)i * words;
-                for (int j = 0; j < nq; ++j) {
+                for (int j = lane; j < nq; j += 32) {
                     if (j == i || partner[j] >= 0) continue;
                     const uint32_t* bj = bbh + (int64_t)j * words;
                     int ov = 0;
                     for (int w = 0; w < words; ++w) ov += __popc(__ldg(bi + w) & __ldg(bj + w));
                     cand_insert(co, cj, ov, j);
                 }
-#pragma unroll
-                for (int c = 0; c < kCand; ++c) cb[(int64_t)i * kCand + c] = co[c] >= 0 ? cj[c] : -1;
+                warp_merge_cand(co, cj, lane, cb + (int64_t)i * kCand, nullptr);
             }
             __syncthreads();
         }
