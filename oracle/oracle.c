@@ -24,7 +24,7 @@
  *    means of K rounded to bf16 before they are used for routing, query
  *    blocks routed by a centroid score.
  *
- * Readings where the pages leave a step open (each is listed in the design doc):
+ * Readings where the pages leave a step open (the design notes list each):
  *  - inside a cube the real tokens come first, in local (t,h,w) row-major
  *    order over the cube's real extent, then zero pads up to 64;
  *  - routing scores are the dot products of bf16 cube means (sequential

@@ -4,9 +4,10 @@ input/output buffers, deployments with every allocation fixed at start-up).
 The library supplies the scratch from a fixed array in its own device code.
 
 This file is collected last on purpose, so that a run stopping at the first
-failure has already run every other test.  It must pass on its own in a fresh
-process as well as after the other tests (the first call on the device does
-the one-time address lookup either way)."""
+failure has already run every other test.  It passes both after the other
+tests and run alone in a fresh process (`pytest -m gpu tests/test_zz_no_alloc.py`),
+where its first call is the first use of the library on the device and does
+the one-time lookup of the array's address."""
 from __future__ import annotations
 
 import ctypes
