@@ -58,9 +58,11 @@ def _load():
         lib.oracle_fwd_items_ex.argtypes = [P, P, P, P, P, I, I, I, I, I, I, ctypes.c_double, P, I64, P, P, P]
         lib.oracle_num_threads.argtypes = []
         lib.oracle_plan.argtypes = [P, I, I, I, I, P]
+        lib.oracle_cube_sums.argtypes = [P, P, P, I, I, I, I, I]
+        lib.oracle_fwd_proxy_items.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, ctypes.c_double, P, I64, P, P]
         for name in ("oracle_f64_to_bf16", "oracle_bf16_to_f64", "oracle_cube_counts", "oracle_tile",
                      "oracle_untile", "oracle_cube_means", "oracle_route", "oracle_fwd_items", "oracle_fwd_items_ex",
-                     "oracle_num_threads", "oracle_plan"):
+                     "oracle_num_threads", "oracle_plan", "oracle_cube_sums", "oracle_fwd_proxy_items"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -132,6 +134,40 @@ def cube_means(x: np.ndarray, vbs: np.ndarray) -> np.ndarray:
     out = np.empty((B, H, nq, D), dtype=np.uint16)
     _check(_load().oracle_cube_means(_ptr(x), _ptr(vbs), _ptr(out), B, S, H, D, nq), "cube_means")
     return out
+
+
+def cube_sums(x: np.ndarray, vbs: np.ndarray) -> np.ndarray:
+    """[B, S, H, D] bf16 -> [B, H, Nq, D] bf16 sums over the valid tokens (the
+    summed-V summaries of proxy compensation)."""
+    B, S, H, D = x.shape
+    nq = S // 64
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    vbs = np.ascontiguousarray(vbs, dtype=np.int32)
+    out = np.empty((B, H, nq, D), dtype=np.uint16)
+    _check(_load().oracle_cube_sums(_ptr(x), _ptr(vbs), _ptr(out), B, S, H, D, nq), "cube_sums")
+    return out
+
+
+def fwd_proxy_items(q, k, v, kc, vc, topk_idx, vbs, sm_scale: float, items: np.ndarray):
+    """Proxy-compensated fine forward for the listed (b, h, query cube) items:
+    selected cubes exact, every omitted cube with valid tokens through its mean
+    key kc and summed value vc, the denominator weighted by the valid counts.
+    Returns out [n, 64, D] and lse [n, 64] (natural log), float64."""
+    B, S, H, D = q.shape
+    nq = S // 64
+    topk = topk_idx.shape[-1]
+    assert topk_idx.shape == (B, H, nq, topk) and kc.shape == (B, H, nq, D) and vc.shape == kc.shape
+    arrs = [np.ascontiguousarray(a, dtype=np.uint16) for a in (q, k, v, kc, vc)]
+    topk_idx = np.ascontiguousarray(topk_idx, dtype=np.int32)
+    vbs = np.ascontiguousarray(vbs, dtype=np.int32)
+    items = np.ascontiguousarray(items, dtype=np.int32).reshape(-1, 3)
+    n = items.shape[0]
+    out = np.empty((n, 64, D), dtype=np.float64)
+    lse = np.empty((n, 64), dtype=np.float64)
+    sigma = float(np.float32(sm_scale))
+    _check(_load().oracle_fwd_proxy_items(*(_ptr(a) for a in arrs), _ptr(topk_idx), _ptr(vbs), B, S, H, D, nq, topk,
+                                          sigma, _ptr(items), n, _ptr(out), _ptr(lse)), "fwd_proxy_items")
+    return out, lse
 
 
 def route(q: np.ndarray, k: np.ndarray, vbs: np.ndarray, topk: int, want_scores: bool = False):

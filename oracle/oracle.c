@@ -350,6 +350,135 @@ int oracle_fwd_items_ex(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
 }
 
+/* ------------------------------------------------------------------ proxy compensation
+ *
+ * TensorRT-LLM PR #7 (the embedded FlashInfer PR "support proxy-compensated
+ * block-sparse attention"): selected blocks stay exact; every omitted KV block
+ * contributes through one arithmetic-mean K summary and one summed-V summary;
+ * a block already covered by an exact route is not counted again by its proxy
+ * (score-keep); the softmax denominator is corrected by the token mass the
+ * proxy represents, the true length of a partial block included.
+ * TensorRT-Edge-LLM "Video Sparse Attention Runner": KC and VC are BF16 block
+ * means of K and block sums of V; every block not attended exactly contributes
+ * through its mean key and summed value.
+ *
+ * For query row s of cube i, with E the selected tokens (multiplicity kept)
+ * and O the cubes j with vbs[j] > 0 that i does not select:
+ *   x_u  = sigma * q_s . k_u                 (u in E)
+ *   y_j  = sigma * q_s . kc_j                (j in O)
+ *   out  = (sum_u e^{x_u} v_u + sum_j e^{y_j} vc_j) / (sum_u e^{x_u} + sum_j vbs[j] e^{y_j})
+ *   lse  = log of that denominator
+ * Rows with E and O both empty: out = 0, lse = -inf. */
+
+/* vc[b, h, c, :] = bf16_rne(sequential FP64 sum of x over the first vbs[c] tokens of cube c) */
+int oracle_cube_sums(const uint16_t *x, const int32_t *vbs, uint16_t *xs, int B, int S, int H, int D, int Nq)
+{
+    if (B <= 0 || H <= 0 || D <= 0 || Nq <= 0 || S != 64 * Nq) return ORACLE_ERR_ARG;
+    for (int c = 0; c < Nq; ++c)
+        if (vbs[c] < 0 || vbs[c] > 64) return ORACLE_ERR_ARG;
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h)
+            for (int c = 0; c < Nq; ++c)
+                for (int d = 0; d < D; ++d) {
+                    double acc = 0.0;
+                    for (int u = 0; u < vbs[c]; ++u)
+                        acc += bf16_bits_to_f64(x[(((int64_t)b * S + 64LL * c + u) * H + h) * D + d]);
+                    xs[(((int64_t)b * H + h) * Nq + c) * D + d] = f64_to_bf16_bits(acc);
+                }
+    return ORACLE_OK;
+}
+
+int oracle_fwd_proxy_items(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *kc,
+                           const uint16_t *vc, const int32_t *topk_idx, const int32_t *vbs, int B, int S, int H,
+                           int D, int Nq, int topk, double sigma, const int32_t *items, int64_t n_items,
+                           double *out, double *lse)
+{
+    if (B <= 0 || H <= 0 || D <= 0 || Nq <= 0 || S != 64 * Nq || topk < 1) return ORACLE_ERR_ARG;
+    for (int c = 0; c < Nq; ++c)
+        if (vbs[c] < 0 || vbs[c] > 64) return ORACLE_ERR_ARG;
+    for (int64_t it = 0; it < n_items; ++it) {
+        int b = items[3 * it], h = items[3 * it + 1], i = items[3 * it + 2];
+        if (b < 0 || b >= B || h < 0 || h >= H || i < 0 || i >= Nq) return ORACLE_ERR_ARG;
+        const int32_t *sel = topk_idx + (((int64_t)b * H + h) * Nq + i) * topk;
+        for (int t = 0; t < topk; ++t)
+            if (sel[t] < 0 || sel[t] >= Nq) return ORACLE_ERR_ARG;
+    }
+    int failed = 0;
+#pragma omp parallel
+    {
+        int64_t *keys = (int64_t *)malloc((size_t)topk * 64 * sizeof(int64_t));
+        int32_t *omitted = (int32_t *)malloc((size_t)Nq * sizeof(int32_t));
+        char *chosen = (char *)malloc((size_t)Nq);
+        double *x = (double *)malloc((size_t)(topk * 64 + Nq) * sizeof(double));
+        if (!keys || !omitted || !chosen || !x) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t it = 0; it < n_items; ++it) {
+            if (!keys || !omitted || !chosen || !x) continue;
+            int b = items[3 * it], h = items[3 * it + 1], i = items[3 * it + 2];
+            const int32_t *sel = topk_idx + (((int64_t)b * H + h) * Nq + i) * topk;
+            /* exact tokens (multiplicity kept) and the omitted cubes (score-keep: a selected cube has no proxy) */
+            int64_t nkeys = 0;
+            for (int c = 0; c < Nq; ++c) chosen[c] = 0;
+            for (int t = 0; t < topk; ++t) {
+                chosen[sel[t]] = 1;
+                for (int u = 0; u < vbs[sel[t]]; ++u) keys[nkeys++] = 64LL * sel[t] + u;
+            }
+            int nom = 0;
+            for (int c = 0; c < Nq; ++c)
+                if (!chosen[c] && vbs[c] > 0) omitted[nom++] = c;
+            for (int r = 0; r < 64; ++r) {
+                int64_t s = 64LL * i + r;
+                const uint16_t *qs = q + (((int64_t)b * S + s) * H + h) * D;
+                double *o = out + (it * 64 + r) * D;
+                if (nkeys == 0 && nom == 0) {
+                    for (int d = 0; d < D; ++d) o[d] = 0.0;
+                    lse[it * 64 + r] = -INFINITY;
+                    continue;
+                }
+                double m = -INFINITY;
+                for (int64_t n = 0; n < nkeys; ++n) {
+                    const uint16_t *ku = k + (((int64_t)b * S + keys[n]) * H + h) * D;
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) dot += bf16_bits_to_f64(qs[d]) * bf16_bits_to_f64(ku[d]);
+                    x[n] = sigma * dot;
+                    if (x[n] > m) m = x[n];
+                }
+                for (int n = 0; n < nom; ++n) {
+                    const uint16_t *kj = kc + (((int64_t)b * H + h) * Nq + omitted[n]) * D;
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) dot += bf16_bits_to_f64(qs[d]) * bf16_bits_to_f64(kj[d]);
+                    x[nkeys + n] = sigma * dot;
+                    if (x[nkeys + n] > m) m = x[nkeys + n];
+                }
+                double l = 0.0;
+                for (int d = 0; d < D; ++d) o[d] = 0.0;
+                for (int64_t n = 0; n < nkeys; ++n) {
+                    double p = exp(x[n] - m);
+                    const uint16_t *vu = v + (((int64_t)b * S + keys[n]) * H + h) * D;
+                    l += p;
+                    for (int d = 0; d < D; ++d) o[d] += p * bf16_bits_to_f64(vu[d]);
+                }
+                for (int n = 0; n < nom; ++n) {
+                    double p = exp(x[nkeys + n] - m);
+                    const uint16_t *vj = vc + (((int64_t)b * H + h) * Nq + omitted[n]) * D;
+                    l += (double)vbs[omitted[n]] * p; /* the token mass the proxy stands for */
+                    for (int d = 0; d < D; ++d) o[d] += p * bf16_bits_to_f64(vj[d]);
+                }
+                for (int d = 0; d < D; ++d) o[d] /= l;
+                lse[it * 64 + r] = m + log(l);
+            }
+        }
+        free(keys);
+        free(omitted);
+        free(chosen);
+        free(x);
+    }
+    return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}
+
 int oracle_fwd_items(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                      const int32_t *topk_idx, const int32_t *vbs,
                      int B, int S, int H, int D, int Nq, int topk, double sigma,

@@ -540,3 +540,105 @@ def test_plan_ignores_duplicates_and_bad_ids(oracle_lib):
     idx = np.array([[[[1, 1, 2], [1, 2, 9], [3, 3, 3], [-1, 3, 0]]]], np.int32)
     # distinct sets: {1,2}, {1,2}, {3}, {3,0}: 0-1 overlap 2, 2-3 overlap 1
     assert oracle_lib.plan(idx).tolist() == [[[0, 1], [2, 3]]]
+
+
+# ------------------------------------------------------------------ proxy compensation
+# TensorRT-LLM PR #7 (FlashInfer PR "support proxy-compensated block-sparse attention") and
+# TensorRT-Edge-LLM "Video Sparse Attention Runner": omitted blocks contribute through their
+# mean key and summed value, the denominator weighted by the tokens each proxy stands for.
+
+def _proxy_case(seed, nq=6, H=2, topk=2, vbs=None, scale=1.5):
+    g = np.random.default_rng(seed)
+    x = [synth.f32_to_bf16_bits((g.standard_normal((1, 64 * nq, H, 128)) * scale).astype(np.float32)) for _ in range(3)]
+    if vbs is None:
+        vbs = g.integers(0, 65, size=nq).astype(np.int32)
+        vbs[0] = 64
+    vbs = np.asarray(vbs, np.int32)
+    idx = synth.random_topk(seed, 1, H, nq, topk)
+    return x[0], x[1], x[2], vbs, idx
+
+
+def test_cube_sums_exact(oracle_lib):
+    """Sums of small integers are exact in FP64 and in bf16 (below 256); pads and empty cubes add nothing."""
+    g = np.random.default_rng(4)
+    v = g.integers(-3, 4, size=(1, 64 * 3, 2, 128)).astype(np.float32)
+    vbs = np.array([64, 17, 0], np.int32)
+    vb = synth.f32_to_bf16_bits(v)
+    got = oracle_lib.bf16_to_f64(oracle_lib.cube_sums(vb, vbs))
+    for c in range(3):
+        want = v[0, 64 * c: 64 * c + vbs[c]].sum(axis=0)  # [H, D]
+        np.testing.assert_array_equal(got[0, :, c], want)
+
+
+def test_proxy_equals_softmax_over_exact_and_proxy_keys(oracle_lib):
+    """The same result from a library softmax over the exact tokens and one key per
+    omitted cube (its mean key, log-weight log vbs[j], value vc_j / vbs[j])."""
+    q, k, v, vbs, idx = _proxy_case(11)
+    nq, H = len(vbs), q.shape[2]
+    kc, vc = oracle_lib.cube_means(k, vbs), oracle_lib.cube_sums(v, vbs)
+    sigma = float(np.float32(0.125))
+    items = oracle_lib.all_items(1, H, nq)
+    out, lse = oracle_lib.fwd_proxy_items(q, k, v, kc, vc, idx, vbs, 0.125, items)
+    f = lambda a: torch.from_numpy(oracle_lib.bf16_to_f64(a))
+    Q, K, V, KC, VC = f(q)[0], f(k)[0], f(v)[0], f(kc)[0], f(vc)[0]
+    for n, (b, h, i) in enumerate(items):
+        sel = idx[0, h, i].tolist()
+        toks = [64 * j + u for j in sel for u in range(vbs[j])]
+        om = [j for j in range(nq) if j not in sel and vbs[j] > 0]
+        qs = Q[64 * i: 64 * i + 64, h]
+        logits = torch.cat([sigma * qs @ K[toks, h].T,
+                            sigma * qs @ KC[h, om].T + torch.log(torch.tensor(vbs[om], dtype=torch.float64))], dim=1)
+        vals = torch.cat([V[toks, h], VC[h, om] / torch.tensor(vbs[om], dtype=torch.float64)[:, None]], dim=0)
+        want = torch.softmax(logits, dim=1) @ vals
+        assert np.allclose(out[n], want.numpy(), rtol=0, atol=1e-12)
+        assert np.allclose(lse[n], torch.logsumexp(logits, dim=1).numpy(), rtol=0, atol=1e-12)
+
+
+def test_proxy_with_every_cube_selected_is_the_plain_forward(oracle_lib):
+    q, k, v, vbs, _ = _proxy_case(12, nq=5, topk=5)
+    idx = np.broadcast_to(np.arange(5, dtype=np.int32), (1, 2, 5, 5)).copy()
+    kc, vc = oracle_lib.cube_means(k, vbs), oracle_lib.cube_sums(v, vbs)
+    items = oracle_lib.all_items(1, 2, 5)
+    o1, l1 = oracle_lib.fwd_proxy_items(q, k, v, kc, vc, idx, vbs, 0.1, items)
+    o2, l2 = oracle_lib.fwd_items(q, k, v, idx, vbs, 0.1, items)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_proxy_is_exact_when_every_cube_is_constant(oracle_lib):
+    """When the keys of each cube are all equal (its mean is that key) and the value
+    sums are exact, proxies reproduce the omitted cubes exactly: the result equals
+    dense attention over every cube, for any selection."""
+    g = np.random.default_rng(13)
+    nq, H = 6, 2
+    vbs = np.array([64, 40, 1, 64, 17, 33], np.int32)
+    q = synth.f32_to_bf16_bits((g.standard_normal((1, 64 * nq, H, 128))).astype(np.float32))
+    kcube = g.standard_normal((nq, H, 128)).astype(np.float32)
+    k = synth.f32_to_bf16_bits(np.repeat(kcube, 64, axis=0)[None])
+    v = synth.f32_to_bf16_bits(g.integers(-2, 3, size=(1, 64 * nq, H, 128)).astype(np.float32))
+    kc, vc = oracle_lib.cube_means(k, vbs), oracle_lib.cube_sums(v, vbs)
+    items = oracle_lib.all_items(1, H, nq)
+    dense = np.broadcast_to(np.arange(nq, dtype=np.int32), (1, H, nq, nq)).copy()
+    o_dense, l_dense = oracle_lib.fwd_items(q, k, v, dense, vbs, 0.2, items)
+    for topk in (1, 3):
+        idx = synth.random_topk(topk, 1, H, nq, topk)
+        o, l = oracle_lib.fwd_proxy_items(q, k, v, kc, vc, idx, vbs, 0.2, items)
+        assert np.allclose(o, o_dense, rtol=0, atol=1e-12)
+        assert np.allclose(l, l_dense, rtol=0, atol=1e-12)
+
+
+def test_proxy_uniform_logits_closed_form(oracle_lib):
+    """q = 0: every weight is equal, so out = (sum of the selected values + the omitted
+    cubes' summed values) / (selected tokens + omitted tokens) and lse = log of that count."""
+    _, k, v, vbs, idx = _proxy_case(14, nq=7, topk=3)
+    q = np.zeros_like(k)
+    kc, vc = oracle_lib.cube_means(k, vbs), oracle_lib.cube_sums(v, vbs)
+    items = oracle_lib.all_items(1, 2, 7)
+    out, lse = oracle_lib.fwd_proxy_items(q, k, v, kc, vc, idx, vbs, 0.3, items)
+    V, VC = oracle_lib.bf16_to_f64(v)[0], oracle_lib.bf16_to_f64(vc)[0]
+    for n, (b, h, i) in enumerate(items):
+        sel = idx[0, h, i].tolist()
+        om = [j for j in range(7) if j not in sel and vbs[j] > 0]
+        num = sum(V[64 * j: 64 * j + vbs[j], h].sum(axis=0) for j in sel) + sum(VC[h, j] for j in om)
+        cnt = sum(int(vbs[j]) for j in sel) + sum(int(vbs[j]) for j in om)
+        assert np.allclose(out[n], np.broadcast_to(num / cnt, (64, 128)), rtol=0, atol=1e-13)
+        assert np.allclose(lse[n], math.log(cnt), rtol=0, atol=1e-13)
