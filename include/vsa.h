@@ -80,9 +80,10 @@ VSA_API int vsa_can_implement(int D, int sm_version);
  * Numerics (default mode): logits and the P.V product accumulate in fp32;
  * each softmax weight enters the P.V product rounded to bf16 and the row
  * sum adds the same rounded weights, so out is a softmax-weighted mean of
- * the selected v rows with each weight off by at most 2^-9 of itself, then
- * rounded to bf16; lse is the log of that same row sum (within 2e-3 of
- * exact, plus the fp32 logit error).  VSA_FWD_PRECISE_P tightens both.
+ * the selected v rows with each weight off by at most 2^-8 of itself (bf16
+ * keeps 8 significant bits), then rounded to bf16; lse is the log of that
+ * same row sum (within -ln(1 - 2^-8) < 4e-3 of exact, plus the fp32 logit
+ * error).  VSA_FWD_PRECISE_P tightens both.
  *
  * Real (non-pad) V rows must be finite: two query cubes share a tile, and a
  * KV cube that only one of them selects enters the other's P.V product with
@@ -118,7 +119,7 @@ enum vsa_fwd_flags {
     VSA_FWD_DEFAULT = 0,
     /* Carry the softmax weights P into the P.V product as a bf16 pair
      * (P = hi + lo, within 2^-17 of P) instead of one bf16 value (within
-     * 2^-9): the output is then within a small fraction of a bf16 ulp of the
+     * 2^-8): the output is then within a small fraction of a bf16 ulp of the
      * exact result, where the default's weight rounding can move an output
      * element by up to 2^-8 * sum_u w_u |v_u - out| before its own rounding
      * (one ulp at large outputs of spread-out softmax rows).  Costs a second
@@ -152,6 +153,35 @@ VSA_API int vsa_fwd_ex(const vsa_bf16 *q, const vsa_bf16 *k, const vsa_bf16 *v, 
 VSA_API int vsa_fwd_planned(const vsa_bf16 *q, const vsa_bf16 *k, const vsa_bf16 *v, const int32_t *topk_idx,
                             const int32_t *vbs, const int32_t *plan, vsa_bf16 *out, float *lse, int B, int S,
                             int H, int D, int Nq, int topk, float sm_scale, int flags, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * vsa_fwd_proxy -- proxy-compensated fine forward.
+ *
+ * TensorRT-LLM PR #7 (the embedded FlashInfer PR "support proxy-compensated
+ * block-sparse attention") and TensorRT-Edge-LLM "Video Sparse Attention
+ * Runner": the selected cubes are attended exactly, and every cube a query
+ * cube did not select contributes through its mean key and summed value,
+ * weighted by the number of tokens it stands for.  For query row s of cube i
+ * (E its selected tokens, multiplicity kept; O the cubes j with vbs[j] > 0
+ * that i did not select -- a selected cube has no proxy):
+ *   out = (sum_{u in E} e^{x_u} v_u + sum_{j in O} e^{y_j} vc_j)
+ *         / (sum_{u in E} e^{x_u} + sum_{j in O} vbs[j] e^{y_j}),
+ *   x_u = sm_scale q_s . k_u,  y_j = sm_scale q_s . kc_j,
+ * lse = the log of that denominator (natural).
+ *
+ *   kc, vc  [B, H, Nq, D] bf16 in: the cubes' mean keys and summed values
+ *           (the bf16 cube means of k and cube sums of v; vsa_tile_qkv forms
+ *           both), caller-owned
+ *   plan    optional tile plan as for vsa_fwd_planned (NULL: consecutive
+ *           pairs)
+ *   other arguments, numerics and errors as vsa_fwd_planned / vsa_fwd_ex,
+ *   plus VSA_ERR_NULL for a NULL kc or vc.  Each tile walks its selected
+ *   cubes, then ceil(Nq / 128) steps of proxy keys.
+ * ---------------------------------------------------------------------- */
+VSA_API int vsa_fwd_proxy(const vsa_bf16 *q, const vsa_bf16 *k, const vsa_bf16 *v, const int32_t *topk_idx,
+                          const int32_t *vbs, const vsa_bf16 *kc, const vsa_bf16 *vc, const int32_t *plan,
+                          vsa_bf16 *out, float *lse, int B, int S, int H, int D, int Nq, int topk, float sm_scale,
+                          int flags, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
  * vsa_route -- cube-mean q.k routing that builds topk_idx.
@@ -286,17 +316,20 @@ VSA_API int vsa_untile(const vsa_bf16 *x_tiled, vsa_bf16 *x_grid, int B, int T, 
  *   qc, kc  [B, H, Nq, D] bf16 out: the cube means of q and k with
  *           vsa_route's arithmetic (slots past a cube's real tokens count as
  *           zeros), bit-identical to the means vsa_route forms from the
- *           tiled tensors; both NULL to tile only
+ *           tiled tensors; both NULL to skip them
+ *   vc      [B, H, Nq, D] bf16 out: the cube sums of v (sequential FP64 sum
+ *           over the first vbs[c] tokens, rounded to bf16 once), the summed
+ *           values of vsa_fwd_proxy; NULL to skip them
  *
  * Errors: as vsa_tile for each of the three tensors; VSA_ERR_ARG if exactly
- * one of qc, kc is NULL, or if means are asked for and D != 128;
- * VSA_ERR_NULL for vbs NULL while means are asked for; VSA_ERR_ALIGN for
- * qc, kc or vbs not 16-byte aligned.  A vbs value outside [0, 64] latches
- * device error 2 and gives a zero mean.
+ * one of qc, kc is NULL, or if means or sums are asked for and D != 128;
+ * VSA_ERR_NULL for vbs NULL while means or sums are asked for;
+ * VSA_ERR_ALIGN for qc, kc, vc or vbs not 16-byte aligned.  A vbs value
+ * outside [0, 64] latches device error 2 and gives a zero mean and sum.
  * ---------------------------------------------------------------------- */
 VSA_API int vsa_tile_qkv(const vsa_bf16 *q_grid, const vsa_bf16 *k_grid, const vsa_bf16 *v_grid, vsa_bf16 *q_tiled,
-                         vsa_bf16 *k_tiled, vsa_bf16 *v_tiled, const int32_t *vbs, vsa_bf16 *qc, vsa_bf16 *kc, int B,
-                         int T, int Hh, int W, int H, int D, cudaStream_t stream);
+                         vsa_bf16 *k_tiled, vsa_bf16 *v_tiled, const int32_t *vbs, vsa_bf16 *qc, vsa_bf16 *kc,
+                         vsa_bf16 *vc, int B, int T, int Hh, int W, int H, int D, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
  * vsa_route_means -- the scoring and top-k steps of vsa_route, on cube means

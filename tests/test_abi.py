@@ -122,17 +122,32 @@ def test_tile_qkv_and_route_means_reject_bad_arguments_without_a_device(vsa):
     p = _fake(1 << 20)
     lib = vsa.get_lib()
     # grid 5x6x7, B=1, H=2, D=128
-    assert lib.vsa_tile_qkv(p, p, p, p, p, p, p, p, None, 1, 5, 6, 7, 2, 128, None) == -1  # kc missing
-    assert lib.vsa_tile_qkv(p, p, p, p, p, p, p, p, p, 1, 5, 6, 7, 2, 64, None) == -1  # means need D = 128
-    assert lib.vsa_tile_qkv(p, p, p, p, p, p, None, p, p, 1, 5, 6, 7, 2, 128, None) == -2  # means need vbs
-    assert lib.vsa_tile_qkv(p, p, None, p, p, p, None, None, None, 1, 5, 6, 7, 2, 128, None) == -2
-    assert lib.vsa_tile_qkv(p, p, p, p, p, p, None, None, None, 1, 0, 6, 7, 2, 128, None) == -1
-    assert lib.vsa_tile_qkv(p, p, p, p, p, _fake((1 << 20) + 4), None, None, None, 1, 5, 6, 7, 2, 128, None) == -3
+    assert lib.vsa_tile_qkv(p, p, p, p, p, p, p, p, None, None, 1, 5, 6, 7, 2, 128, None) == -1  # kc missing
+    assert lib.vsa_tile_qkv(p, p, p, p, p, p, p, p, p, None, 1, 5, 6, 7, 2, 64, None) == -1  # means need D = 128
+    assert lib.vsa_tile_qkv(p, p, p, p, p, p, p, None, None, p, 1, 5, 6, 7, 2, 64, None) == -1  # sums too
+    assert lib.vsa_tile_qkv(p, p, p, p, p, p, None, p, p, None, 1, 5, 6, 7, 2, 128, None) == -2  # means need vbs
+    assert lib.vsa_tile_qkv(p, p, p, p, p, p, None, None, None, p, 1, 5, 6, 7, 2, 128, None) == -2  # sums need vbs
+    assert lib.vsa_tile_qkv(p, p, None, p, p, p, None, None, None, None, 1, 5, 6, 7, 2, 128, None) == -2
+    assert lib.vsa_tile_qkv(p, p, p, p, p, p, None, None, None, None, 1, 0, 6, 7, 2, 128, None) == -1
+    assert lib.vsa_tile_qkv(p, p, p, p, p, _fake((1 << 20) + 4), None, None, None, None, 1, 5, 6, 7, 2, 128,
+                            None) == -3
+    assert lib.vsa_tile_qkv(p, p, p, p, p, p, p, None, None, _fake((1 << 20) + 4), 1, 5, 6, 7, 2, 128, None) == -3
     assert lib.vsa_route_means(p, p, p, 1, 2, 128, 8, 9, None) == -1  # topk > Nq
     assert lib.vsa_route_means(p, p, p, 1, 2, 64, 8, 2, None) == -1  # D != 128
     assert lib.vsa_route_means(p, p, p, 1, 2, 128, 5000, 2, None) == -1  # Nq > 4096
     assert lib.vsa_route_means(p, None, p, 1, 2, 128, 8, 2, None) == -2
     assert lib.vsa_route_means(p, p, _fake((1 << 20) + 4), 1, 2, 128, 8, 2, None) == -3
+
+
+def test_fwd_proxy_rejects_bad_arguments_without_a_device(vsa):
+    p = _fake(1 << 20)
+    lib = vsa.get_lib()
+    args = (1, 512, 2, 128, 8, 2, 0.1, 0, None)  # B, S, H, D, Nq, topk, scale, flags, stream
+    assert lib.vsa_fwd_proxy(p, p, p, p, p, None, p, None, p, None, *args) == -2  # kc missing
+    assert lib.vsa_fwd_proxy(p, p, p, p, p, p, None, None, p, None, *args) == -2  # vc missing
+    assert lib.vsa_fwd_proxy(p, p, p, p, p, p, _fake((1 << 20) + 2), None, p, None, *args) == -3
+    assert lib.vsa_fwd_proxy(p, p, p, p, p, p, p, None, p, None, 1, 512, 2, 64, 8, 2, 0.1, 0, None) == -1
+    assert lib.vsa_fwd_proxy(p, p, p, p, p, p, p, None, p, None, 1, 512, 2, 128, 8, 2, 0.1, 2, None) == -1  # flag
 
 
 def test_route_noalloc_checks_arguments_before_its_array_limit(vsa):

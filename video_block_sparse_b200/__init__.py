@@ -30,7 +30,7 @@ _STATUS = {0: "VSA_OK", -1: "VSA_ERR_ARG", -2: "VSA_ERR_NULL", -3: "VSA_ERR_ALIG
            -5: "VSA_ERR_ARCH", -6: "VSA_ERR_LAUNCH", -7: "VSA_ERR_DEVICE"}
 
 # every symbol include/vsa.h declares
-EXPORTS = ("vsa_status_string", "vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_fwd_planned",
+EXPORTS = ("vsa_status_string", "vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_fwd_planned", "vsa_fwd_proxy",
            "vsa_plan_workspace_size", "vsa_plan", "vsa_route_workspace_size", "vsa_route", "vsa_route_means",
            "vsa_route_noalloc", "vsa_cube_counts", "vsa_tile", "vsa_tile_qkv", "vsa_untile", "vsa_stall_check",
            "vsa_device_status")
@@ -63,11 +63,12 @@ def _load():
     lib.vsa_cube_counts.argtypes = [I, I, I, P, P]
     lib.vsa_tile.argtypes = [P, P, I, I, I, I, I, I, P]
     lib.vsa_untile.argtypes = [P, P, I, I, I, I, I, I, P]
-    lib.vsa_tile_qkv.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, P]
+    lib.vsa_tile_qkv.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, P]
+    lib.vsa_fwd_proxy.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.vsa_route_means.argtypes = [P, P, P, I, I, I, I, I, P]
     lib.vsa_device_status.argtypes = [P, P]
     lib.vsa_stall_check.argtypes = [P, P]
-    for name in ("vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_fwd_planned", "vsa_plan", "vsa_route",
+    for name in ("vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_fwd_planned", "vsa_fwd_proxy", "vsa_plan", "vsa_route",
                  "vsa_route_means", "vsa_route_noalloc", "vsa_cube_counts", "vsa_tile", "vsa_tile_qkv", "vsa_untile",
                  "vsa_device_status", "vsa_stall_check"):
         getattr(lib, name).restype = I
@@ -156,11 +157,12 @@ def untile(x_tiled: torch.Tensor, grid, out: torch.Tensor | None = None, stream=
 
 
 def tile_qkv(q_grid: torch.Tensor, k_grid: torch.Tensor, v_grid: torch.Tensor, grid, vbs: torch.Tensor | None = None,
-             means: bool = True, out=None, stream=None):
+             means: bool = True, out=None, sums: bool = False, stream=None):
     """vsa_tile_qkv: tile q, k, v ([B, T*Hh*W, H, D] raster) in one launch and,
-    if `means`, form the cube means of q and k ([B, H, Nq, D]) in the same pass.
-    Returns (q_tiled, k_tiled, v_tiled, qc, kc) (qc, kc None without means).
-    `out` may hold preallocated tensors in that order."""
+    if `means`, form the cube means of q and k ([B, H, Nq, D]) in the same pass,
+    and if `sums` the cube sums of v (the summed values of vsa_fwd_proxy).
+    Returns (q_tiled, k_tiled, v_tiled, qc, kc), plus vc with `sums` (None
+    for what was not asked).  `out` may hold preallocated tensors in that order."""
     T, Hh, W = grid
     B, L, H, D = q_grid.shape
     for t, n in ((q_grid, "q_grid"), (k_grid, "k_grid"), (v_grid, "v_grid")):
@@ -174,15 +176,21 @@ def tile_qkv(q_grid: torch.Tensor, k_grid: torch.Tensor, v_grid: torch.Tensor, g
         dev = q_grid.device
         out = [torch.empty(B, 64 * nq, H, D, dtype=q_grid.dtype, device=dev) for _ in range(3)]
         out += [torch.empty(B, H, nq, D, dtype=q_grid.dtype, device=dev) for _ in range(2)] if means else [None, None]
-    qt, kt, vt, qc, kc = out
+        out += [torch.empty(B, H, nq, D, dtype=q_grid.dtype, device=dev) if sums else None]
+    out = list(out) + [None] * (6 - len(out))
+    qt, kt, vt, qc, kc, vc = out
+    if sums and (vc is None or vc.shape != (B, H, nq, D) or vbs is None):
+        raise ValueError("tile_qkv: sums need vbs and a [B, H, Nq, D] output")
     if L != T * Hh * W or any(x.shape != (B, 64 * nq, H, D) for x in (qt, kt, vt)):
         raise ValueError("tile_qkv: shape mismatch")
     if means and (vbs is None or qc is None or kc is None or qc.shape != (B, H, nq, D) or kc.shape != qc.shape):
         raise ValueError("tile_qkv: means need vbs and [B, H, Nq, D] outputs")
     _check(get_lib().vsa_tile_qkv(_ptr(q_grid), _ptr(k_grid), _ptr(v_grid), _ptr(qt), _ptr(kt), _ptr(vt),
-                                  _ptr(vbs) if means else None, _ptr(qc) if means else None,
-                                  _ptr(kc) if means else None, B, T, Hh, W, H, D, _stream(stream)), "vsa_tile_qkv")
-    return (qt, kt, vt, qc, kc) if means else (qt, kt, vt, None, None)
+                                  _ptr(vbs) if (means or sums) else None, _ptr(qc) if means else None,
+                                  _ptr(kc) if means else None, _ptr(vc) if sums else None, B, T, Hh, W, H, D,
+                                  _stream(stream)), "vsa_tile_qkv")
+    res = (qt, kt, vt, qc if means else None, kc if means else None)
+    return res + (vc,) if sums else res
 
 
 def route_means(qc: torch.Tensor, kc: torch.Tensor, topk: int, out: torch.Tensor | None = None,
@@ -280,6 +288,35 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk_idx: torch.Tenso
         _check(get_lib().vsa_fwd_planned(_ptr(q), _ptr(k), _ptr(v), _ptr(topk_idx), _ptr(vbs), _ptr(plan), _ptr(out),
                                          _ptr(lse), B, S, H, D, nq, topk, float(sm_scale), int(flags),
                                          _stream(stream)), "vsa_fwd_planned")
+    return (out, lse) if (want_lse or lse is not None) else out
+
+
+def fwd_proxy(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk_idx: torch.Tensor, vbs: torch.Tensor,
+              kc: torch.Tensor, vc: torch.Tensor, sm_scale: float | None = None, out: torch.Tensor | None = None,
+              lse: torch.Tensor | None = None, want_lse: bool = False, flags: int = FWD_DEFAULT,
+              plan: torch.Tensor | None = None, stream=None):
+    """vsa_fwd_proxy: the fine forward with every omitted cube represented by its
+    mean key kc and summed value vc ([B, H, Nq, D] bf16); returns out (and lse)."""
+    B, S, H, D = q.shape
+    nq = S // 64
+    topk = topk_idx.shape[-1]
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (kc, "kc"), (vc, "vc")):
+        _bf16(t, n)
+    if kc.shape != (B, H, nq, D) or vc.shape != kc.shape:
+        raise ValueError("kc and vc must be [B, H, Nq, D]")
+    if topk_idx.dtype != torch.int32 or vbs.dtype != torch.int32:
+        raise ValueError("topk_idx and vbs must be int32")
+    if plan is not None and (plan.dtype != torch.int32 or plan.numel() != B * H * ((nq + 1) // 2) * 2):
+        raise ValueError("plan must be int32 [B*H, ceil(Nq/2), 2]")
+    if sm_scale is None:
+        sm_scale = D ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, H, S, dtype=torch.float32, device=q.device)
+    _check(get_lib().vsa_fwd_proxy(_ptr(q), _ptr(k), _ptr(v), _ptr(topk_idx), _ptr(vbs), _ptr(kc), _ptr(vc),
+                                   _ptr(plan), _ptr(out), _ptr(lse), B, S, H, D, nq, topk, float(sm_scale),
+                                   int(flags), _stream(stream)), "vsa_fwd_proxy")
     return (out, lse) if (want_lse or lse is not None) else out
 
 

@@ -79,8 +79,9 @@ int check_bshd(int B, int S, int H, int D, int Nq)
 }
 
 int fwd_dispatch(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const int32_t* topk_idx,
-                 const int32_t* vbs, const int32_t* plan, vsa_bf16* out, float* lse, int B, int S, int H, int D,
-                 int Nq, int topk, float sm_scale, int flags, cudaStream_t stream);
+                 const int32_t* vbs, const int32_t* plan, const vsa_bf16* kc, const vsa_bf16* vc, vsa_bf16* out,
+                 float* lse, int B, int S, int H, int D, int Nq, int topk, float sm_scale, int flags,
+                 cudaStream_t stream);
 
 }  // namespace
 
@@ -107,10 +108,11 @@ int vsa_can_implement(int D, int sm_version) { return (D == 128 && sm_version ==
 
 namespace {
 
-// Shared by vsa_fwd_ex and vsa_fwd_planned: checks, then the kernel the flags name.
+// Shared by vsa_fwd_ex, vsa_fwd_planned and vsa_fwd_proxy: checks, then the kernel.
 int fwd_dispatch(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const int32_t* topk_idx,
-                 const int32_t* vbs, const int32_t* plan, vsa_bf16* out, float* lse, int B, int S, int H, int D,
-                 int Nq, int topk, float sm_scale, int flags, cudaStream_t stream)
+                 const int32_t* vbs, const int32_t* plan, const vsa_bf16* kc, const vsa_bf16* vc, vsa_bf16* out,
+                 float* lse, int B, int S, int H, int D, int Nq, int topk, float sm_scale, int flags,
+                 cudaStream_t stream)
 {
     int rc = check_bshd(B, S, H, D, Nq);
     if (rc != VSA_OK) return rc;
@@ -119,13 +121,14 @@ int fwd_dispatch(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const 
     if ((int64_t)B * H * Nq * topk > INT32_MAX) return VSA_ERR_ARG;
     if (!q || !k || !v || !topk_idx || !vbs || !out) return VSA_ERR_NULL;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(topk_idx) ||
-        !aligned16(vbs) || (lse && !aligned16(lse)) || (plan && !aligned16(plan)))
+        !aligned16(vbs) || (lse && !aligned16(lse)) || (plan && !aligned16(plan)) || (kc && !aligned16(kc)) ||
+        (vc && !aligned16(vc)))
         return VSA_ERR_ALIGN;
     if ((rc = check_arch()) != VSA_OK) return rc;
     int* err;
     if ((rc = device_error_word(&err)) != VSA_OK) return rc;
     const bool precise = (flags & VSA_FWD_PRECISE_P) != 0;
-    return launch_status(vsa::launch_fwd_pair(q, k, v, topk_idx, vbs, plan, out, lse, B, S, H, Nq, topk, sm_scale,
+    return launch_status(vsa::launch_fwd_pair(q, k, v, topk_idx, vbs, plan, kc, vc, out, lse, B, S, H, Nq, topk, sm_scale,
                                               precise, err, stream));
 }
 
@@ -153,7 +156,8 @@ int vsa_fwd_ex(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const in
                vsa_bf16* out, float* lse, int B, int S, int H, int D, int Nq, int topk, float sm_scale, int flags,
                cudaStream_t stream)
 {
-    return fwd_dispatch(q, k, v, topk_idx, vbs, nullptr, out, lse, B, S, H, D, Nq, topk, sm_scale, flags, stream);
+    return fwd_dispatch(q, k, v, topk_idx, vbs, nullptr, nullptr, nullptr, out, lse, B, S, H, D, Nq, topk, sm_scale,
+                        flags, stream);
 }
 
 int vsa_fwd_planned(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const int32_t* topk_idx,
@@ -161,7 +165,18 @@ int vsa_fwd_planned(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, con
                     int Nq, int topk, float sm_scale, int flags, cudaStream_t stream)
 {
     if (!plan) return VSA_ERR_NULL;
-    return fwd_dispatch(q, k, v, topk_idx, vbs, plan, out, lse, B, S, H, D, Nq, topk, sm_scale, flags, stream);
+    return fwd_dispatch(q, k, v, topk_idx, vbs, plan, nullptr, nullptr, out, lse, B, S, H, D, Nq, topk, sm_scale,
+                        flags, stream);
+}
+
+int vsa_fwd_proxy(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const int32_t* topk_idx,
+                  const int32_t* vbs, const vsa_bf16* kc, const vsa_bf16* vc, const int32_t* plan, vsa_bf16* out,
+                  float* lse, int B, int S, int H, int D, int Nq, int topk, float sm_scale, int flags,
+                  cudaStream_t stream)
+{
+    if (!kc || !vc) return VSA_ERR_NULL;
+    return fwd_dispatch(q, k, v, topk_idx, vbs, plan, kc, vc, out, lse, B, S, H, D, Nq, topk, sm_scale, flags,
+                        stream);
 }
 
 int vsa_fwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const int32_t* topk_idx, const int32_t* vbs,
@@ -269,19 +284,20 @@ int vsa_untile(const vsa_bf16* x_tiled, vsa_bf16* x_grid, int B, int T, int Hh, 
 }
 
 int vsa_tile_qkv(const vsa_bf16* q_grid, const vsa_bf16* k_grid, const vsa_bf16* v_grid, vsa_bf16* q_tiled,
-                 vsa_bf16* k_tiled, vsa_bf16* v_tiled, const int32_t* vbs, vsa_bf16* qc, vsa_bf16* kc, int B, int T,
-                 int Hh, int W, int H, int D, cudaStream_t stream)
+                 vsa_bf16* k_tiled, vsa_bf16* v_tiled, const int32_t* vbs, vsa_bf16* qc, vsa_bf16* kc, vsa_bf16* vc,
+                 int B, int T, int Hh, int W, int H, int D, cudaStream_t stream)
 {
     const bool means = qc != nullptr || kc != nullptr;
     if (means && (qc == nullptr || kc == nullptr)) return VSA_ERR_ARG;
-    if (means && D != 128) return VSA_ERR_ARG;
+    if ((means || vc != nullptr) && D != 128) return VSA_ERR_ARG;
     int rc;
     if ((rc = check_tile_pair(q_grid, q_tiled, B, T, Hh, W, H, D)) != VSA_OK) return rc;
     if ((rc = check_tile_pair(k_grid, k_tiled, B, T, Hh, W, H, D)) != VSA_OK) return rc;
     if ((rc = check_tile_pair(v_grid, v_tiled, B, T, Hh, W, H, D)) != VSA_OK) return rc;
-    if (means) {
+    if (means || vc != nullptr) {
         if (!vbs) return VSA_ERR_NULL;
-        if (!aligned16(vbs) || !aligned16(qc) || !aligned16(kc)) return VSA_ERR_ALIGN;
+        if (!aligned16(vbs) || (means && (!aligned16(qc) || !aligned16(kc))) || (vc && !aligned16(vc)))
+            return VSA_ERR_ALIGN;
     }
     if ((rc = check_arch()) != VSA_OK) return rc;
     int* err;
@@ -295,7 +311,9 @@ int vsa_tile_qkv(const vsa_bf16* q_grid, const vsa_bf16* k_grid, const vsa_bf16*
     }
     job.means[0] = qc;
     job.means[1] = kc;
-    job.means[2] = nullptr;
+    job.means[2] = vc;
+    job.sums[0] = job.sums[1] = 0;
+    job.sums[2] = 1;
     return launch_status(vsa::launch_tile_cubes(job, 3, vbs, B, vsa::make_geom(T, Hh, W), H, D, err, stream));
 }
 

@@ -14,8 +14,16 @@
 // both tcgen05.mma (bf16 in, fp32 accumulate in TMEM); P is written over S
 // in TMEM as bf16 and is the A operand of the second product.  A KV cube
 // that only one of the two query cubes selected has weight 0 for the other
-// cube's rows.  Cubes both lists name are walked first and loaded once for
-// both; vsa_plan pairs query cubes whose lists overlap most.
+// cube's rows.  A cube both lists name is loaded once for both; vsa_plan
+// pairs query cubes whose lists overlap most.
+//
+// Proxy compensation (vsa_fwd_proxy; TensorRT-LLM PR #7, the embedded FlashInfer
+// PR "support proxy-compensated block-sparse attention"): after a tile's
+// selected cubes come ceil(Nq / 128) proxy steps whose keys are the cubes'
+// mean keys and whose values are their summed values; a row uses the proxy of
+// every cube with valid tokens that its query cube did not select, with its
+// weight counted vbs[j] times in the row sum.  PROXY is a template parameter:
+// the plain kernels hold none of it.
 //
 // Pipeline.  TMEM holds three S/P buffers (columns 0, 128, 256) and O
 // (columns 384-511).  Step g uses buffer g % 3, and the two MMA issuers run
@@ -32,8 +40,9 @@
 //   warps 12-15 O correction and epilogue (thread = row): rescale the rows
 //               whose running offset rose, once the previous PV has finished;
 //               at a tile's end, O / l -> out and the log-sum-exp -> lse
-//   warp 16     TMA producer of Q and K: builds each tile's step list (shared
-//               cubes first) from lists copied in one tile ahead, streams Q
+//   warp 16     TMA producer of Q and K: builds each tile's step list (list 1,
+//               then list 2's other cubes) over the tile's list 1, from lists
+//               copied in one tile ahead, streams Q
 //               (one buffer; loaded after the tile's first K pair) and K pairs
 //               (ring of 3) and posts each step's V pair to warp 18
 //   warp 17     PV MMA issuer (the whole warp runs the schedule, one elected
@@ -75,6 +84,7 @@ constexpr int kKBuf = 3;  // K ring depth
 constexpr int kVBuf = 2;  // V ring depth
 constexpr uint32_t kOCol = 384;
 constexpr uint32_t kFinal = 1u << 22;  // step word: last step of the CTA's last tile
+constexpr uint32_t kProxyStep = 1u << 23;  // step word: the keys are proxies of omitted cubes
 
 // Pairs (bit c: columns 2c, 2c+1 of each 32-column chunk) whose exp2 runs on
 // the FMA pipe instead of the multi-function unit.  None by default: with three
@@ -110,6 +120,12 @@ struct Misc {
     uint32_t v_meta[kVBuf];  // step word of the V pair in each V buffer
     uint32_t k_meta[kKBuf];  // step word of the K pair in each K buffer
     uint32_t s_meta[kSBuf];  // step word of each S buffer
+    // proxy steps: which of the step's 128 proxy keys each query cube may use
+    // ([cube][key half][32-key word]) and the first proxy key's cube index
+    uint32_t k_pmask[kKBuf][8];
+    int k_pbase[kKBuf];
+    uint32_t s_pmask[kSBuf][8];
+    int s_pbase[kSBuf];
     uint32_t tmem_base;
     int abort;
     int end_g;  // the CTA's last step, once its softmax is done (the other softmax warps stop there)
@@ -124,7 +140,7 @@ struct Misc {
     uint32_t bits2[kMaxNq / 32];
     int32_t list1[2][kMaxTopk];           // [tile parity]: the tile's two selection lists
     int32_t list2[2][kMaxTopk];           // (the next tile's are copied in while this one runs)
-    uint8_t vbs8[kMaxNq];                 // the valid counts (255: out of range)
+    alignas(16) uint8_t vbs8[kMaxNq];     // the valid counts (255: out of range)
 };
 
 struct Layout {
@@ -137,10 +153,19 @@ struct Layout {
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-template <bool NEG, bool PRECISE>
+template <bool B>
+struct Flag {
+    static constexpr bool value = B;
+};
+
+// PROXY: the kernel runs the proxy steps after each tile's selected cubes.  It is a
+// template parameter so that the plain kernels hold none of that code: the extra
+// instructions cost the plain forward ~25% through instruction fetches alone.
+template <bool NEG, bool PRECISE, bool PROXY>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                    const __grid_constant__ CUtensorMap tmv, const int32_t* __restrict__ topk_idx,
+                    const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmkc,
+                    const __grid_constant__ CUtensorMap tmvc, const int32_t* __restrict__ topk_idx,
                     const int32_t* __restrict__ vbs, const int32_t* __restrict__ plan, uint16_t* __restrict__ out,
                     float* __restrict__ lse, int S, int H, int nq, int topk, int tiles_per_bh, int n_tiles,
                     float scale_log2, int* err)
@@ -210,6 +235,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tmq);
         prefetch_tmap(&tmk);
         prefetch_tmap(&tmv);
+        if (PROXY) {
+            prefetch_tmap(&tmkc);
+            prefetch_tmap(&tmvc);
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -220,9 +249,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ TMA producer of Q and K
         // (it posts each step's V pair to the V producer, so that K loads never wait
         // behind a V buffer)
-        ListGen gen;
         int kc = 0;
         int armed_q = -1, armed_k = -1, armed_kb = 0;
+        const uint64_t l2_keep = PROXY ? l2_policy_evict_last() : 0ull;
         bool aborted = false;
         uint8_t* qdst = tiles_ptr + L::Q_OFF;
         TileRef t_next;
@@ -234,54 +263,54 @@ __global__ void __launch_bounds__(kThreads, 1)
             const TileRef t = t_next;
             int32_t* l1 = m.list1[n & 1];
             int32_t* l2 = m.list2[n & 1];
-            gen_start(gen, t, m.vbs8, nq, topk, l1, l2, m.bits1, m.bits2, err, lane);
+            const int n_ent = steps_build(t, m.vbs8, nq, topk, l1, l2, m.bits1, m.bits2, err, lane);
+            const uint16_t* ent = reinterpret_cast<const uint16_t*>(l1);  // written over list 1
             const int tok0 = t.b * S;
-            bool q_pending = true;  // Q is loaded after the tile's first K pair (which needs no Q buffer)
-            bool first = true;
-            while (!aborted) {
-                const Entry ea = gen.next;
-                Entry eb{0, 0, 0};
-                if (ea.mem != 0) {
-                    gen.next = gen_pull(gen, l1, l2, m.bits1, m.bits2, m.vbs8, lane);
-                    eb = gen.next;
-                    if (eb.mem != 0) gen.next = gen_pull(gen, l1, l2, m.bits1, m.bits2, m.vbs8, lane);
-                }
-                const bool last = gen.next.mem == 0;
-                StepMeta meta;
-                meta.ja = ea.j;
-                meta.jb = eb.j;
-                meta.na = ea.n;
-                meta.nb = eb.n;
-                meta.ma = ea.mem;
-                meta.mb = eb.mem;
-                meta.flags = (first ? 1 : 0) | (last ? 2 : 0);
-                first = false;
-                const uint32_t word = step_word(meta) | (last && n == my_tiles - 1 ? kFinal : 0u);
-                const uint32_t bytes = 2 * kHalfBox * ((meta.na > 0) + (meta.nb > 0));
+            // proxy mode: after the selected cubes, ceil(nq / 128) steps over the proxy keys
+            // (cube j's mean key and summed value), 128 cubes per step; a tile without
+            // entries then has no plain step (else it takes one empty step)
+            const int n_proxy = PROXY ? (nq + 127) / 128 : 0;
+            const int n_plain = PROXY ? (n_ent + 1) / 2 : max(1, (n_ent + 1) / 2);
+            const int n_steps = n_plain + n_proxy;
+            // Step s of the tile: its K pair (rows ka, kb of head kh of map kmap; -1: none),
+            // its V request, and with the tile's first step the tile's Q and the next tile's
+            // lists.  Inlined at two sites, each with a fixed map.
+            auto issue = [&](int s, const CUtensorMap* kmap, int kh, int ka, int kb2, int vh, uint32_t word,
+                             const uint32_t* pmw, int pbase) {
+                const uint32_t bytes = 2 * kHalfBox * ((ka >= 0) + (kb2 >= 0));
                 const int kb = kc % kKBuf, vr = kc % kVReq;
                 if (lane == 0) {
                     // K pair of the step: its buffer is free once the QK two steps back finished
                     if (wait_bar(&bb.k_empty[kb], ((kc / kKBuf) & 1) ^ 1, &m.abort, err)) {
-                        m.k_meta[kb] = word;
+                        if (pmw != nullptr) {
+#pragma unroll
+                            for (int w = 0; w < 8; ++w) m.k_pmask[kb][w] = pmw[w];
+                            m.k_pbase[kb] = pbase;
+                        }
+                        m.k_meta[kb] = word;  // published, with the masks, by the expect-tx arrival
                         mbar_expect_tx(&bb.k_full[kb], bytes);
                         armed_k = (kc / kKBuf) & 1;
                         armed_kb = kb;
                         uint8_t* kdst = tiles_ptr + L::K_OFF + kb * kTileBytes;
-                        if (meta.na > 0) load_cube(&tmk, &bb.k_full[kb], kdst, 0, t.h, tok0 + 64 * meta.ja);
-                        if (meta.nb > 0) load_cube(&tmk, &bb.k_full[kb], kdst, 1, t.h, tok0 + 64 * meta.jb);
+                        if (pmw != nullptr) {  // mean keys: every tile of the head reads them
+                            if (ka >= 0) load_cube_keep(kmap, &bb.k_full[kb], kdst, 0, kh, ka, l2_keep);
+                            if (kb2 >= 0) load_cube_keep(kmap, &bb.k_full[kb], kdst, 1, kh, kb2, l2_keep);
+                        } else {
+                            if (ka >= 0) load_cube(kmap, &bb.k_full[kb], kdst, 0, kh, ka);
+                            if (kb2 >= 0) load_cube(kmap, &bb.k_full[kb], kdst, 1, kh, kb2);
+                        }
                     } else {
                         aborted = true;
                     }
-                    // the step's V pair, for the V producer
+                    // the step's V pair, for the V producer (same rows as the K pair)
                     if (!aborted && wait_bar(&bb.vr_empty[vr], ((kc / kVReq) & 1) ^ 1, &m.abort, err)) {
-                        m.vreq[vr] = make_int4(meta.na > 0 ? tok0 + 64 * meta.ja : -1,
-                                               meta.nb > 0 ? tok0 + 64 * meta.jb : -1, t.h, (int)word);
+                        m.vreq[vr] = make_int4(ka, kb2, vh, (int)word);
                         mbar_arrive(&bb.vr_full[vr]);
                     } else {
                         aborted = true;
                     }
                     // the tile's Q, once the previous tile's last QK has released the buffer
-                    if (!aborted && q_pending) {
+                    if (!aborted && s == 0) {
                         if (wait_bar(&bb.q_empty, (n & 1) ^ 1, &m.abort, err)) {
                             mbar_expect_tx(&bb.q_full, 2 * kHalfBox * ((t.i1 >= 0) + (t.i2 >= 0)));
                             armed_q = n & 1;
@@ -292,25 +321,76 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-                if (q_pending && n + 1 < my_tiles) {
+                if (s == 0 && n + 1 < my_tiles) {
                     // the next tile, once this one's first loads are out: its lists copied
                     // into the other list buffer and its Q cubes prefetched into L2
                     t_next = checked_tile(blockIdx.x + (n + 1) * gridDim.x, H, nq, tiles_per_bh, plan,
                                           lane == 0 ? err : nullptr);
                     lists_fetch(t_next, topk_idx, H, nq, topk, m.list1[(n + 1) & 1], m.list2[(n + 1) & 1], lane);
                     if (lane == 0) {
-                        for (int s = 0; s < 2; ++s) {
-                            const int i = s == 0 ? t_next.i1 : t_next.i2;
+                        for (int q2 = 0; q2 < 2; ++q2) {
+                            const int i = q2 == 0 ? t_next.i1 : t_next.i2;
                             if (i < 0) continue;
                             tma_prefetch_3d(&tmq, 0, t_next.h, t_next.b * S + 64 * i);
                             tma_prefetch_3d(&tmq, 64, t_next.h, t_next.b * S + 64 * i);
                         }
                     }
                 }
-                q_pending = false;
                 aborted = __shfl_sync(0xffffffffu, aborted, 0);
                 ++kc;
-                if (last) break;
+            };
+            // the selected cubes, two entries a step (one 32-bit load: 2 s is even)
+            for (int s = 0; s < n_plain && !aborted; ++s) {
+                const uint32_t pair = 2 * s < n_ent ? *reinterpret_cast<const uint32_t*>(ent + 2 * s) : 0u;
+                const uint32_t ea = pair & 0xffffu;
+                const uint32_t eb = 2 * s + 1 < n_ent ? pair >> 16 : 0u;
+                const int ja = (int)(ea & 0x1fffu), jb = (int)(eb & 0x1fffu);
+                StepMeta meta;
+                meta.ma = (int)(ea >> 14);
+                meta.mb = (int)(eb >> 14);
+                meta.na = meta.ma != 0 ? m.vbs8[ja] : 0;
+                meta.nb = meta.mb != 0 ? m.vbs8[jb] : 0;
+                const bool last = s + 1 == n_steps;
+                meta.flags = (s == 0 ? 1 : 0) | (last ? 2 : 0);
+                const uint32_t word = step_word(meta) | (last && n == my_tiles - 1 ? kFinal : 0u);
+                issue(s, &tmk, t.h, meta.na > 0 ? tok0 + 64 * ja : -1, meta.nb > 0 ? tok0 + 64 * jb : -1, t.h, word,
+                      nullptr, 0);
+            }
+            if constexpr (PROXY) {
+                // proxy keys pbase .. pbase + 127 (rows of the [B*H*nq, D] means and sums): key
+                // j may be used by query cube q iff cube j has valid tokens and q did not
+                // select it (no double count)
+                const int cubes_here = (t.i1 >= 0 ? 1 : 0) | (t.i2 >= 0 ? 2 : 0);
+                for (int pc = 0; pc < n_proxy && !aborted; ++pc) {
+                    const int s = n_plain + pc, pbase = 128 * pc;
+                    StepMeta meta;
+                    meta.na = min(64, nq - pbase);
+                    meta.nb = min(64, max(0, nq - pbase - 64));
+                    meta.ma = cubes_here;
+                    meta.mb = meta.nb > 0 ? cubes_here : 0;
+                    uint32_t pm = 0;  // lane w < 8: mask word w, [cube][key half][32-key word]
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const int j = pbase + 32 * w + (int)lane;
+                        const int nj = j < nq ? (int)m.vbs8[j] : 0;
+                        const uint32_t valid = __ballot_sync(0xffffffffu, nj >= 1 && nj <= 64);
+                        const int word = (pbase >> 5) + w;
+                        const bool in_range = pbase + 32 * w < nq;
+                        const uint32_t m1 = t.i1 >= 0 && in_range ? valid & ~m.bits1[word] : 0u;
+                        const uint32_t m2 = t.i2 >= 0 && in_range ? valid & ~m.bits2[word] : 0u;
+                        if ((int)lane == w) pm = m1;
+                        if ((int)lane == 4 + w) pm = m2;
+                    }
+                    uint32_t pmw[8];  // in every lane (lane 0 stores them with the K pair)
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) pmw[w] = __shfl_sync(0xffffffffu, pm, w);
+                    const bool last = s + 1 == n_steps;
+                    meta.flags = (s == 0 ? 1 : 0) | (last ? 2 : 0);
+                    const uint32_t word =
+                        step_word(meta) | (last && n == my_tiles - 1 ? kFinal : 0u) | kProxyStep;
+                    const int row = (t.b * H + t.h) * nq + pbase;
+                    issue(s, &tmkc, 0, row, meta.nb > 0 ? row + 64 : -1, 0, word, pmw, pbase);
+                }
             }
         }
         cp_async_wait_all();  // a list copy still in flight after an abort
@@ -322,6 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kWarpVProd) {
         // ------------------------------------------------------------ TMA producer of V
         int armed_v = -1, armed_vb = 0;
+        const uint64_t l2_keep = PROXY ? l2_policy_evict_last() : 0ull;
         for (int vc = 0; my_tiles > 0 && lane == 0; ++vc) {
             const int vr = vc % kVReq, vb = vc % kVBuf;
             if (!wait_bar(&bb.vr_full[vr], (vc / kVReq) & 1, &m.abort, err)) break;
@@ -334,8 +415,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             armed_v = (vc / kVBuf) & 1;
             armed_vb = vb;
             uint8_t* vdst = tiles_ptr + L::V_OFF + vb * kTileBytes;
-            if (rq.x >= 0) load_cube(&tmv, &bb.v_full[vb], vdst, 0, rq.z, rq.x);
-            if (rq.y >= 0) load_cube(&tmv, &bb.v_full[vb], vdst, 1, rq.z, rq.y);
+            if (PROXY && ((uint32_t)rq.w & kProxyStep)) {
+                // summed values: every tile of the head reads them, so they stay in L2
+                if (rq.x >= 0) load_cube_keep(&tmvc, &bb.v_full[vb], vdst, 0, rq.z, rq.x, l2_keep);
+                if (rq.y >= 0) load_cube_keep(&tmvc, &bb.v_full[vb], vdst, 1, rq.z, rq.y, l2_keep);
+            } else {
+                if (rq.x >= 0) load_cube(&tmv, &bb.v_full[vb], vdst, 0, rq.z, rq.x);
+                if (rq.y >= 0) load_cube(&tmv, &bb.v_full[vb], vdst, 1, rq.z, rq.y);
+            }
             if ((uint32_t)rq.w & kFinal) break;  // the CTA's last step
         }
         if (lane == 0 && armed_v >= 0 && aborted_flag(&m.abort)) drain_wait(&bb.v_full[armed_vb], armed_v);
@@ -372,6 +459,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (j >= kSBuf && !wait_warp(&bb.pv_issued[sb], ((j - kSBuf) / kSBuf) & 1, &m.abort, err)) {
                     aborted = true;
                     break;
+                }
+                if (PROXY && (meta & kProxyStep)) {
+                    // every lane stores the same words, so the elected arrival publishes them
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) m.s_pmask[sb][w] = m.k_pmask[kb][w];
+                    m.s_pbase[sb] = m.k_pbase[kb];
                 }
                 m.s_meta[sb] = meta;                // every lane stores the same word
                 mbar_arrive_elect(&bb.s_full[sb]);  // publishes it (release)
@@ -575,30 +668,45 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nv0 = ((sw_ma(meta) >> qbit) & 1) ? na : 0;  // valid keys of each half
             const int nv1 = ((sw_mb(meta) >> qbit) & 1) ? nb : 0;  // for this row (warp-uniform)
             const uint32_t s_addr = lane_base + 128u * b;
+            // proxy step: the keys are mean keys of cubes pbase .. pbase + 127; chunk ch's
+            // mask word (which of them this row's query cube may use) and their token counts
+            const bool pstep = PROXY && (meta & kProxyStep) != 0;
+            const uint32_t* pmask = m.s_pmask[b] + 4 * qbit;
+            const int pbase = pstep ? m.s_pbase[b] : 0;
 
             // pass 1: extreme of the selected logits, one 32-column chunk at a time
-            // (chunk ch: columns 32 ch .. +31, key half ch / 2)
-            float e4[4] = {kNeutral, kNeutral, kNeutral, kNeutral};
+            // (chunk ch: columns 32 ch .. +31, key half ch / 2).  Both passes come in two
+            // instantiations: a proxy step masks by its bits, a plain step only its ragged
+            // tail, and plain steps run none of the proxy code.
+            auto pass1 = [&](auto px) -> float {
+                constexpr bool PX = decltype(px)::value;
+                float e4[4] = {kNeutral, kNeutral, kNeutral, kNeutral};
 #pragma unroll 1
-            for (int ch = 0; ch < 4; ++ch) {
-                const int nv = (ch < 2 ? nv0 : nv1) - 32 * (ch & 1);  // valid columns of the chunk
-                if (nv <= 0) continue;
-                float sc[32];
-                tmem_ld32(s_addr + 32 * ch, reinterpret_cast<uint32_t*>(sc));
-                tmem_ld_wait();
-                if (nv < 32) {
+                for (int ch = 0; ch < 4; ++ch) {
+                    const int nv = (ch < 2 ? nv0 : nv1) - 32 * (ch & 1);  // valid columns of the chunk
+                    if (nv <= 0) continue;
+                    float sc[32];
+                    tmem_ld32(s_addr + 32 * ch, reinterpret_cast<uint32_t*>(sc));
+                    tmem_ld_wait();
+                    if constexpr (PX) {
+                        const uint32_t mw = pmask[ch];
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) sc[c] = c < nv ? sc[c] : kNeutral;
+                        for (int c = 0; c < 32; ++c) sc[c] = (mw >> c) & 1u ? sc[c] : kNeutral;
+                    } else if (nv < 32) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) sc[c] = c < nv ? sc[c] : kNeutral;
+                    }
+#pragma unroll
+                    for (int c = 0; c < 32; c += 8) {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            e4[u] = NEG ? min3(e4[u], sc[c + 2 * u], sc[c + 2 * u + 1])
+                                        : max3(e4[u], sc[c + 2 * u], sc[c + 2 * u + 1]);
+                    }
                 }
-#pragma unroll
-                for (int c = 0; c < 32; c += 8) {
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        e4[u] = NEG ? min3(e4[u], sc[c + 2 * u], sc[c + 2 * u + 1])
-                                    : max3(e4[u], sc[c + 2 * u], sc[c + 2 * u + 1]);
-                }
-            }
-            const float ext = NEG ? min3(fminf(e4[0], e4[1]), e4[2], e4[3]) : max3(fmaxf(e4[0], e4[1]), e4[2], e4[3]);
+                return NEG ? min3(fminf(e4[0], e4[1]), e4[2], e4[3]) : max3(fmaxf(e4[0], e4[1]), e4[2], e4[3]);
+            };
+            const float ext = PROXY && pstep ? pass1(Flag<PROXY>{}) : pass1(Flag<false>{});
 
             // decision: the row's offset after this step (lazy: raised by more than kTau only)
             if (g > 0) {
@@ -630,54 +738,83 @@ __global__ void __launch_bounds__(kThreads, 1)
             // bf16 parts (lo = bf16(P - hi), so hi + lo is within 2^-17 of P) in the
             // chunk's own columns 32 ch .. +15 and +16 .. +31
             const float mu = m_run == -INFINITY ? 0.f : m_run;
-            float ls0 = 0.f, ls1 = 0.f;
+            auto pass2 = [&](auto px) -> float2 {
+                constexpr bool PX = decltype(px)::value;
+                float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll 1
-            for (int ch = 0; ch < 4; ++ch) {
-                const int nv = (ch < 2 ? nv0 : nv1) - 32 * (ch & 1);
-                uint32_t pk[16], pl[16];
-                if (nv > 0) {
-                    float sc[32];
-                    tmem_ld32(s_addr + 32 * ch, reinterpret_cast<uint32_t*>(sc));
-                    tmem_ld_wait();
-                    if (nv < 32) {
+                for (int ch = 0; ch < 4; ++ch) {
+                    const int nv = (ch < 2 ? nv0 : nv1) - 32 * (ch & 1);
+                    uint32_t pk[16], pl[16];
+                    if (nv > 0) {
+                        float sc[32];
+                        tmem_ld32(s_addr + 32 * ch, reinterpret_cast<uint32_t*>(sc));
+                        tmem_ld_wait();
+                        if constexpr (PX) {
+                            const uint32_t mw = pmask[ch];
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) sc[c] = c < nv ? sc[c] : kNeutral;
-                    }
+                            for (int c = 0; c < 32; ++c) sc[c] = (mw >> c) & 1u ? sc[c] : kNeutral;
+                        } else if (nv < 32) {
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        float x0, x1, p0, p1;
-                        ffma2(x0, x1, sc[2 * c], sc[2 * c + 1], scale_log2, scale_log2, -mu, -mu);
-                        if ((kPolyPairs >> (c & 15)) & 1) {
-                            // weights below 2^-125 (masked keys included) become 2^-125
-                            const float2 pp = ex2_fma2(make_float2(fmaxf(x0, -125.f), fmaxf(x1, -125.f)));
-                            p0 = pp.x;
-                            p1 = pp.y;
-                        } else {
-                            p0 = ex2(x0);
-                            p1 = ex2(x1);
+                            for (int c = 0; c < 32; ++c) sc[c] = c < nv ? sc[c] : kNeutral;
                         }
-                        pk[c] = pack_bf16(p0, p1);
-                        const float h0 = __uint_as_float(pk[c] << 16), h1 = __uint_as_float(pk[c] & 0xffff0000u);
-                        if (PRECISE) {
-                            pl[c] = pack_bf16(p0 - h0, p1 - h1);  // the differences are exact in fp32
-                            fadd2(ls0, ls1, p0, p1);
-                        } else {
-                            // the row sum adds the bf16 weights the P.V product sees, so that
-                            // numerator and denominator carry the same rounding
-                            fadd2(ls0, ls1, h0, h1);
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) {
+                            float x0, x1, p0, p1;
+                            ffma2(x0, x1, sc[2 * c], sc[2 * c + 1], scale_log2, scale_log2, -mu, -mu);
+                            if ((kPolyPairs >> (c & 15)) & 1) {
+                                // weights below 2^-125 (masked keys included) become 2^-125
+                                const float2 pp = ex2_fma2(make_float2(fmaxf(x0, -125.f), fmaxf(x1, -125.f)));
+                                p0 = pp.x;
+                                p1 = pp.y;
+                            } else {
+                                p0 = ex2(x0);
+                                p1 = ex2(x1);
+                            }
+                            pk[c] = pack_bf16(p0, p1);
+                            if (PRECISE) {
+                                const float h0 = __uint_as_float(pk[c] << 16), h1 = __uint_as_float(pk[c] & 0xffff0000u);
+                                pl[c] = pack_bf16(p0 - h0, p1 - h1);  // the differences are exact in fp32
+                                fadd2(ls0, ls1, p0, p1);
+                            } else {
+                                // the row sum adds the bf16 weights the P.V product sees, so that
+                                // numerator and denominator carry the same rounding
+                                add_bf16x2_f32(ls0, ls1, pk[c]);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) pk[c] = pl[c] = 0u;
+                    }
+                    if (PRECISE) {
+                        tmem_st16(s_addr + 32 * ch, pk);
+                        tmem_st16(s_addr + 32 * ch + 16, pl);
+                    } else {
+                        tmem_st16(s_addr + 64 * (ch >> 1) + 16 * (ch & 1), pk);
+                    }
+                    if (PX && nv > 0) {
+                        // a proxy stands for vbs[j] tokens: the loop above added its weight once,
+                        // this adds it vbs[j] - 1 more times (its summed value enters P.V once)
+                        const uint4 wa = *reinterpret_cast<const uint4*>(m.vbs8 + pbase + 32 * ch);
+                        const uint4 wb = *reinterpret_cast<const uint4*>(m.vbs8 + pbase + 32 * ch + 16);
+                        const uint32_t wn[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) {
+                            // the counts as floats: byte k of the word under the exponent of 2^23
+                            const uint32_t w = wn[c >> 1], k = 2 * (c & 1);
+                            float n0 = __uint_as_float(__byte_perm(w, 0x4B000000u, k | 0x7540u));
+                            float n1 = __uint_as_float(__byte_perm(w, 0x4B000000u, (k + 1) | 0x7540u));
+                            fadd2(n0, n1, -8388609.f, -8388609.f);  // vbs[j] - 1
+                            float h0 = __uint_as_float(pk[c] << 16), h1 = __uint_as_float(pk[c] & 0xffff0000u);
+                            if (PRECISE)  // the weight is hi + lo
+                                fadd2(h0, h1, __uint_as_float(pl[c] << 16), __uint_as_float(pl[c] & 0xffff0000u));
+                            ffma2(ls0, ls1, h0, h1, n0, n1, ls0, ls1);
                         }
                     }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) pk[c] = pl[c] = 0u;
                 }
-                if (PRECISE) {
-                    tmem_st16(s_addr + 32 * ch, pk);
-                    tmem_st16(s_addr + 32 * ch + 16, pl);
-                } else {
-                    tmem_st16(s_addr + 64 * (ch >> 1) + 16 * (ch & 1), pk);
-                }
-            }
+                return make_float2(ls0, ls1);
+            };
+            const float2 lsum = PROXY && pstep ? pass2(Flag<PROXY>{}) : pass2(Flag<false>{});
+            const float ls0 = lsum.x, ls1 = lsum.y;
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&bb.p_full[b]);
@@ -725,12 +862,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kWarpMma) tmem_dealloc(tbase, 512);
 }
 
-template <bool NEG, bool PRECISE>
-cudaError_t launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const int32_t* topk_idx,
-                   const int32_t* vbs, const int32_t* plan, uint16_t* out, float* lse, int B, int S, int H, int nq,
-                   int topk, float scale_log2, int* err, cudaStream_t s)
+// The maps of one forward call: q, k, v ([B*S tokens][H][D]) and, for proxy
+// compensation, the mean keys and summed values ([B*H*Nq rows][1][D]).
+struct FwdMaps {
+    CUtensorMap q, k, v, kc, vc;
+};
+
+template <bool NEG, bool PRECISE, bool PROXY>
+cudaError_t launch(const FwdMaps& mp, const int32_t* topk_idx, const int32_t* vbs, const int32_t* plan, uint16_t* out,
+                   float* lse, int B, int S, int H, int nq, int topk, float scale_log2, int* err, cudaStream_t s)
 {
-    auto kern = fwd_pair_kernel<NEG, PRECISE>;
+    auto kern = fwd_pair_kernel<NEG, PRECISE, PROXY>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Layout::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
@@ -739,8 +881,8 @@ cudaError_t launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
     const int tiles_per_bh = (nq + 1) / 2;
     const int n_tiles = B * H * tiles_per_bh;
     const int grid = n_tiles < sms ? n_tiles : sms;
-    kern<<<grid, kThreads, Layout::SMEM_BYTES, s>>>(mq, mk, mv, topk_idx, vbs, plan, out, lse, S, H, nq, topk,
-                                                    tiles_per_bh, n_tiles, scale_log2, err);
+    kern<<<grid, kThreads, Layout::SMEM_BYTES, s>>>(mp.q, mp.k, mp.v, mp.kc, mp.vc, topk_idx, vbs, plan, out,
+                                                    lse, S, H, nq, topk, tiles_per_bh, n_tiles, scale_log2, err);
     return cudaGetLastError();
 }
 
@@ -749,21 +891,31 @@ cudaError_t launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
 bool fwd_pair_supported(int nq, int topk) { return nq <= kMaxNq && topk <= kMaxTopk; }
 
 cudaError_t launch_fwd_pair(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* topk_idx,
-                            const int32_t* vbs, const int32_t* plan, uint16_t* out, float* lse, int B, int S, int H,
-                            int nq, int topk, float sm_scale, bool precise_p, int* err, cudaStream_t s)
+                            const int32_t* vbs, const int32_t* plan, const uint16_t* kc, const uint16_t* vc,
+                            uint16_t* out, float* lse, int B, int S, int H, int nq, int topk, float sm_scale,
+                            bool precise_p, int* err, cudaStream_t s)
 {
-    CUtensorMap mq, mk, mv;
+    FwdMaps mp;
     const int64_t tokens = (int64_t)B * S;
-    if (!make_map(&mq, q, tokens, H) || !make_map(&mk, k, tokens, H) || !make_map(&mv, v, tokens, H))
+    if (!make_map(&mp.q, q, tokens, H) || !make_map(&mp.k, k, tokens, H) || !make_map(&mp.v, v, tokens, H))
         return cudaErrorInvalidValue;
+    const bool proxy = kc != nullptr && vc != nullptr;
+    if (proxy) {
+        const int64_t rows = (int64_t)B * H * nq;
+        if (!make_map(&mp.kc, kc, rows, 1) || !make_map(&mp.vc, vc, rows, 1)) return cudaErrorInvalidValue;
+    } else {
+        mp.kc = mp.k;  // not read
+        mp.vc = mp.v;
+    }
     const float scale_log2 = sm_scale * 1.4426950408889634f;
-    if (precise_p)
-        return scale_log2 < 0.f
-                   ? launch<true, true>(mq, mk, mv, topk_idx, vbs, plan, out, lse, B, S, H, nq, topk, scale_log2, err, s)
-                   : launch<false, true>(mq, mk, mv, topk_idx, vbs, plan, out, lse, B, S, H, nq, topk, scale_log2, err, s);
-    return scale_log2 < 0.f
-               ? launch<true, false>(mq, mk, mv, topk_idx, vbs, plan, out, lse, B, S, H, nq, topk, scale_log2, err, s)
-               : launch<false, false>(mq, mk, mv, topk_idx, vbs, plan, out, lse, B, S, H, nq, topk, scale_log2, err, s);
+    // one kernel per (sign of the scale, weight precision, proxy steps)
+    using Launch = cudaError_t (*)(const FwdMaps&, const int32_t*, const int32_t*, const int32_t*, uint16_t*, float*,
+                                   int, int, int, int, int, float, int*, cudaStream_t);
+    static constexpr Launch table[8] = {
+        launch<false, false, false>, launch<true, false, false>, launch<false, true, false>, launch<true, true, false>,
+        launch<false, false, true>,  launch<true, false, true>,  launch<false, true, true>,  launch<true, true, true>};
+    const int which = (scale_log2 < 0.f ? 1 : 0) | (precise_p ? 2 : 0) | (proxy ? 4 : 0);
+    return table[which](mp, topk_idx, vbs, plan, out, lse, B, S, H, nq, topk, scale_log2, err, s);
 }
 
 }  // namespace vsa

@@ -31,18 +31,14 @@ constexpr int kMaxNq = 8192;    // per-slot membership bitmaps in shared memory
 
 // Per-step description, produced by the producer warp with each K pair.
 struct StepMeta {
-    int32_t ja, jb;   // cube ids of key halves 0 (keys 0-63) and 1 (keys 64-127)
-    int32_t na, nb;   // valid keys of each half (0: nothing loaded)
+    int32_t na, nb;   // valid keys of key halves 0 (keys 0-63) and 1 (64-127); 0: nothing loaded
     int32_t ma, mb;   // membership: bit 0 = query cube i1 selects it, bit 1 = i2
     int32_t flags;    // bit 0 first step of the tile, bit 1 last step
-    int32_t vslot;    // V ring slot of this step's V pair (set by the MMA issuer)
-    int32_t vpar;     // its phase parity
-    int32_t pad[3];
 };
-static_assert(sizeof(StepMeta) == 48, "StepMeta layout");
 
 // The fields the other roles need, packed in one 32-bit word in shared memory:
-// na [0,7) nb [7,14) ma [14,16) mb [16,18) flags [18,20) vslot [20] vpar [21].
+// na [0,7) nb [7,14) ma [14,16) mb [16,18) flags [18,20); the kernel adds its
+// own flags above bit 21.
 __device__ __forceinline__ uint32_t step_word(const StepMeta& s)
 {
     return (uint32_t)s.na | ((uint32_t)s.nb << 7) | ((uint32_t)s.ma << 14) | ((uint32_t)s.mb << 16) |
@@ -53,8 +49,6 @@ __device__ __forceinline__ int sw_nb(uint32_t w) { return (int)((w >> 7) & 127u)
 __device__ __forceinline__ int sw_ma(uint32_t w) { return (int)((w >> 14) & 3u); }
 __device__ __forceinline__ int sw_mb(uint32_t w) { return (int)((w >> 16) & 3u); }
 __device__ __forceinline__ int sw_flags(uint32_t w) { return (int)((w >> 18) & 3u); }
-__device__ __forceinline__ int sw_vslot(uint32_t w) { return (int)((w >> 20) & 1u); }
-__device__ __forceinline__ int sw_vpar(uint32_t w) { return (int)((w >> 21) & 1u); }
 
 
 __device__ __forceinline__ float ex2(float x)
@@ -205,6 +199,19 @@ __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1)
         : "f"(a0), "f"(a1));
 }
 
+// d0 += the low bf16 of w, d1 += its high bf16: each widened exactly and added
+// with one fp32 rounding (the same sums as unpacking to fp32 first, in fewer
+// instructions).
+__device__ __forceinline__ void add_bf16x2_f32(float& d0, float& d1, uint32_t w)
+{
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "mov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\t"
+        "add.rn.f32.bf16 %1, hi, %1;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "r"(w));
+}
+
 
 __device__ __forceinline__ bool aborted_flag(int* abort) { return *reinterpret_cast<volatile int*>(abort) != 0; }
 
@@ -331,72 +338,14 @@ __device__ __forceinline__ TileRef tile_ref(int t, int H, int nq, int tiles_per_
 
 // ------------------------------------------------------------------ step lists
 //
-// The union of a tile's two selection lists, walked in three phases:
-//   0: entries of list 2 whose cube list 1 also names   (both query cubes)
-//   1: entries of list 1 whose cube list 2 does not name (query cube i1 only)
-//   2: entries of list 2 whose cube list 1 does not name (query cube i2 only)
-// A list that names a cube twice disables the sharing (phase 0 is empty and
-// phases 1/2 take every entry), which keeps every multiplicity.  Entries
-// whose cube has no valid token are skipped.  The generator is run by the
-// whole producer warp; `next` keeps a one-entry lookahead so that each step
-// knows whether it is the tile's last.
-struct Entry {
-    int j, n, mem;  // cube, valid tokens, membership bits; mem = 0: none
-};
-
-struct ListGen {
-    int phase, base;
-    uint32_t mask;   // qualifying entries of the 32-entry window at `base`
-    bool dedupe;
-    int len1, len2;  // list lengths (0 if the query cube is absent)
-    Entry next;
-};
-
+// A tile's keys are the union of its two selection lists, as 16-bit entries
+// (cube j in bits 0-12, membership in bits 14-15: 1 = query cube i1, 2 = i2,
+// 3 = both), in this order: every entry of list 1 (membership 3 when list 2
+// names the same cube), then the entries of list 2 that list 1 does not name.
+// A list that names a cube twice disables the sharing (list 1's entries are
+// all membership 1 and list 2's all membership 2), which keeps every
+// multiplicity.  Entries whose cube has no valid token are left out.
 __device__ __forceinline__ bool test_bit(const uint32_t* bits, int j) { return (bits[j >> 5] >> (j & 31)) & 1u; }
-
-// Scan forward to the next qualifying entry (warp-uniform result).
-__device__ Entry gen_pull(ListGen& g, const int32_t* l1, const int32_t* l2, const uint32_t* b1, const uint32_t* b2,
-                          const uint8_t* vbs8, uint32_t lane)
-{
-    Entry e{0, 0, 0};
-    for (;;) {
-        if (g.phase > 2) return e;
-        const int len = g.phase == 1 ? g.len1 : g.len2;
-        const int32_t* list = g.phase == 1 ? l1 : l2;
-        if (g.mask == 0) {
-            if (g.base >= len) {
-                ++g.phase;
-                g.base = 0;
-                continue;
-            }
-            const int idx = g.base + (int)lane;
-            bool q = false;
-            if (idx < len) {
-                const int j = list[idx];
-                const int n = j >= 0 ? vbs8[j] : 0;
-                if (n > 0 && n <= 64) {
-                    if (g.phase == 0)
-                        q = g.dedupe && test_bit(b1, j);
-                    else if (g.phase == 1)
-                        q = !g.dedupe || !test_bit(b2, j);
-                    else
-                        q = !g.dedupe || !test_bit(b1, j);
-                }
-            }
-            g.mask = __ballot_sync(0xffffffffu, q);
-            g.base += 32;
-            if (g.mask == 0) continue;
-        }
-        const int l = __ffs(g.mask) - 1;
-        g.mask &= g.mask - 1;
-        const int idx = g.base - 32 + l;
-        const int j = list[idx];
-        e.j = j;
-        e.n = vbs8[j];
-        e.mem = g.phase == 0 ? 3 : (g.phase == 1 ? 1 : 2);
-        return e;
-    }
-}
 
 // The valid counts as bytes in shared memory (read for every list entry); a
 // count outside [0, 64] is kept as 255, which the list code treats as an
@@ -410,7 +359,7 @@ __device__ __forceinline__ void vbs_stage(const int32_t* __restrict__ vbs, int n
 }
 
 // Copy a tile's two selection lists into shared memory asynchronously
-// (cp.async, one entry per lane and pass); gen_start waits for them.  Run one
+// (cp.async, one entry per lane and pass); steps_build waits for them.  Run one
 // tile ahead, so that the copies overlap the previous tile's steps.
 __device__ __forceinline__ void lists_fetch(const TileRef& t, const int32_t* __restrict__ topk_idx, int H, int nq,
                                             int topk, int32_t* l1, int32_t* l2, uint32_t lane)
@@ -425,28 +374,31 @@ __device__ __forceinline__ void lists_fetch(const TileRef& t, const int32_t* __r
     cp_async_commit();
 }
 
-// Build a tile's membership bitmaps from its lists (fetched by lists_fetch)
-// and prime the generator.  Invalid cube ids latch an error and are dropped
-// (stored as -1); invalid vbs values latch an error and count as empty cubes.
-// vbs8: the valid counts staged in shared memory (vbs_stage).
-__device__ void gen_start(ListGen& g, const TileRef& t, const uint8_t* vbs8, int nq, int topk, int32_t* l1,
-                          int32_t* l2, uint32_t* b1, uint32_t* b2, int* err, uint32_t lane)
+// Build a tile's membership bitmaps and its entry list from its two selection
+// lists (fetched by lists_fetch), by the whole producer warp.  The entries are
+// written over list 1 (each 32-entry window of it is read before any entry
+// lands on it: after window w at most 32 (w + 1) entries exist, which end
+// within its first w + 1 windows' bytes).  Invalid cube ids latch an error
+// and are dropped; invalid vbs values latch an error and count as empty
+// cubes.  vbs8: the valid counts staged in shared memory (vbs_stage).
+// Returns the number of entries (warp-uniform).
+__device__ int steps_build(const TileRef& t, const uint8_t* vbs8, int nq, int topk, int32_t* l1, int32_t* l2,
+                           uint32_t* b1, uint32_t* b2, int* err, uint32_t lane)
 {
     const int words = (nq + 31) >> 5;
     for (int w = lane; w < words; w += 32) {
         b1[w] = 0u;
         b2[w] = 0u;
     }
-    g.len1 = t.i1 >= 0 ? topk : 0;
-    g.len2 = t.i2 >= 0 ? topk : 0;
+    const int len1 = t.i1 >= 0 ? topk : 0;
+    const int len2 = t.i2 >= 0 ? topk : 0;
     cp_async_wait_all();
     __syncwarp();
     // bitmaps by non-returning shared-memory ORs; a list names a cube twice iff
     // its bitmap holds fewer bits than it has valid entries
     int valid[2] = {0, 0};
     for (int s = 0; s < 2; ++s) {
-        const int len = s == 0 ? g.len1 : g.len2;
-        if (len == 0) continue;
+        const int len = s == 0 ? len1 : len2;
         int32_t* lst = s == 0 ? l1 : l2;
         uint32_t* bits = s == 0 ? b1 : b2;
         for (int e = lane; e < len; e += 32) {
@@ -475,12 +427,33 @@ __device__ void gen_start(ListGen& g, const TileRef& t, const uint8_t* vbs8, int
         set[0] += __shfl_xor_sync(0xffffffffu, set[0], o);
         set[1] += __shfl_xor_sync(0xffffffffu, set[1], o);
     }
-    const bool dup = set[0] != valid[0] || set[1] != valid[1];
-    g.dedupe = !dup && g.len1 > 0 && g.len2 > 0;
-    g.phase = g.dedupe ? 0 : 1;
-    g.base = 0;
-    g.mask = 0;
-    g.next = gen_pull(g, l1, l2, b1, b2, vbs8, lane);
+    const bool share = set[0] == valid[0] && set[1] == valid[1] && len1 > 0 && len2 > 0;
+    uint16_t* ent = reinterpret_cast<uint16_t*>(l1);
+    const uint32_t lt = (1u << lane) - 1u;  // lanes below this one
+    int count = 0;
+    for (int s = 0; s < 2; ++s) {
+        const int len = s == 0 ? len1 : len2;
+        const int32_t* lst = s == 0 ? l1 : l2;
+        for (int base = 0; base < len; base += 32) {
+            const int e = base + (int)lane;
+            const int j = e < len ? lst[e] : -1;
+            const int n = j >= 0 ? vbs8[j] : 0;
+            bool q = n > 0 && n <= 64;
+            uint32_t mem = 1;
+            if (s == 0) {
+                if (q && share && test_bit(b2, j)) mem = 3;
+            } else {
+                mem = 2;
+                q = q && !(share && test_bit(b1, j));
+            }
+            const uint32_t mask = __ballot_sync(0xffffffffu, q);
+            __syncwarp();  // the window is read before entries land on list 1
+            if (q) ent[count + __popc(mask & lt)] = (uint16_t)((uint32_t)j | (mem << 14));
+            count += __popc(mask);
+        }
+    }
+    __syncwarp();
+    return count;
 }
 
 // A tile with an out-of-range plan entry latches an error; the bad cube is dropped.
@@ -504,6 +477,14 @@ __device__ __forceinline__ void load_cube(const CUtensorMap* map, uint64_t* bar,
 {
     tma_load_3d(map, bar, dst + part * kHalfBox, 0, h, tok);
     tma_load_3d(map, bar, dst + 2 * kHalfBox + part * kHalfBox, 64, h, tok);
+}
+
+// The same with an L2 cache policy.
+__device__ __forceinline__ void load_cube_keep(const CUtensorMap* map, uint64_t* bar, uint8_t* dst, int part, int h,
+                                               int tok, uint64_t policy)
+{
+    tma_load_3d_hint(map, bar, dst + part * kHalfBox, 0, h, tok, policy);
+    tma_load_3d_hint(map, bar, dst + 2 * kHalfBox + part * kHalfBox, 64, h, tok, policy);
 }
 
 

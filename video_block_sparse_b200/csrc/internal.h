@@ -31,6 +31,7 @@ struct TileJob {
     const uint4* src[3];   // raster tensors [B, T*Hh*W, H, D]
     uint4* dst[3];         // tiled tensors [B, 64*Nq, H, D]
     uint16_t* means[3];    // cube means [B, H, Nq, D] bf16, or nullptr
+    int sums[3];           // 1: that buffer gets the cube sums instead of the means
 };
 cudaError_t launch_tile_cubes(const TileJob& job, int n_tensors, const int32_t* vbs, int B, const CubeGeom& g, int H,
                               int D, int* err, cudaStream_t s);
@@ -52,9 +53,11 @@ cudaError_t launch_score_topk(const uint16_t* qc, const uint16_t* kc, int32_t* t
 
 // ---- fwd_pair.cu (tcgen05 kernel, two query cubes per 128-row tile)
 bool fwd_pair_supported(int nq, int topk);
+// kc, vc: the proxies' mean keys and summed values [B, H, Nq, 128] (both NULL: no proxies)
 cudaError_t launch_fwd_pair(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* topk_idx,
-                            const int32_t* vbs, const int32_t* plan, uint16_t* out, float* lse, int B, int S, int H,
-                            int nq, int topk, float sm_scale, bool precise_p, int* err, cudaStream_t s);
+                            const int32_t* vbs, const int32_t* plan, const uint16_t* kc, const uint16_t* vc,
+                            uint16_t* out, float* lse, int B, int S, int H, int nq, int topk, float sm_scale,
+                            bool precise_p, int* err, cudaStream_t s);
 
 // ---- plan.cu (pairing of query cubes by selection overlap)
 size_t plan_workspace_bytes(int B, int H, int nq);

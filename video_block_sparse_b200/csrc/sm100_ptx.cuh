@@ -146,6 +146,25 @@ __device__ __forceinline__ void tma_load_3d(const void* tmap, uint64_t* bar, voi
         : "memory");
 }
 
+// The same load with an L2 cache policy (from l2_policy_evict_last).
+__device__ __forceinline__ void tma_load_3d_hint(const void* tmap, uint64_t* bar, void* dst, int c0, int c1, int c2,
+                                                 uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
+        "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
+        : "memory");
+}
+
+// An L2 policy that keeps the lines it touches ahead of normal ones on eviction.
+__device__ __forceinline__ uint64_t l2_policy_evict_last()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
 // L2 prefetch of one tensor-map box (nothing is written to shared memory)
 __device__ __forceinline__ void tma_prefetch_3d(const void* tmap, int c0, int c1, int c2)
 {

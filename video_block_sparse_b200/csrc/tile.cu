@@ -126,7 +126,8 @@ __device__ __forceinline__ void add_bf16x8(double (&acc)[8], const uint4 w)
 // means buffer the same pass also forms the cube mean: FP64 sums over slots
 // 0 .. vbs[c] - 1 in slot order (pads count as zeros), divided by vbs[c] and
 // rounded to bf16, into [B, H, Nq, D] -- the routing's means, without reading
-// the tiled tensor again.
+// the tiled tensor again (for a sums buffer, the sum itself rounded to bf16:
+// the summed values of proxy compensation).
 constexpr int kTileCols = 320;  // 16-byte columns per CTA
 constexpr int kTileUnroll = 8;
 
@@ -141,6 +142,7 @@ __global__ void __launch_bounds__(kTileCols) tile_cubes_kernel(TileJob job, cons
     const uint4* __restrict__ src = t == 0 ? job.src[0] : (t == 1 ? job.src[1] : job.src[2]);
     uint4* __restrict__ dst = t == 0 ? job.dst[0] : (t == 1 ? job.dst[1] : job.dst[2]);
     uint16_t* __restrict__ xm = t == 0 ? job.means[0] : (t == 1 ? job.means[1] : job.means[2]);
+    const int as_sum = t == 0 ? job.sums[0] : (t == 1 ? job.sums[1] : job.sums[2]);
     const int cw = c % g.ncw, ch = (c / g.ncw) % g.nch, ct = c / (g.ncw * g.nch);
     const int et = min(4, g.T - 4 * ct), eh = min(4, g.Hh - 4 * ch), ew = min(4, g.W - 4 * cw);
     const int n_real = et * eh * ew;
@@ -177,10 +179,12 @@ __global__ void __launch_bounds__(kTileCols) tile_cubes_kernel(TileJob job, cons
         }
     }
     if (xm != nullptr) {
+        // the sum rounds as the mean of one (the division by 1 is exact); empty cubes give 0
+        const int div = as_sum ? (n_mean > 0 ? 1 : 0) : n_mean;
         uint32_t o[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-            o[e] = (uint32_t)mean_bf16(acc[2 * e], n_mean) | ((uint32_t)mean_bf16(acc[2 * e + 1], n_mean) << 16);
+            o[e] = (uint32_t)mean_bf16(acc[2 * e], div) | ((uint32_t)mean_bf16(acc[2 * e + 1], div) << 16);
         const int h = (col * 8) / D, d = (col * 8) % D;
         *reinterpret_cast<uint4*>(xm + (((int64_t)b * H + h) * g.nq + c) * D + d) = make_uint4(o[0], o[1], o[2], o[3]);
     }
