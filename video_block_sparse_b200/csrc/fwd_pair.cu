@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         m.end_g = 0x7fffffff;
         fence_mbar_init();
     }
-    vbs_stage(vbs, nq, m.vbs8);
+    vbs_stage(vbs, nq, m.vbs8, err);
     if (warp == kWarpMma) {
         tmem_alloc(&m.tmem_base, 512);
         tmem_relinquish();
@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const TileRef t = t_next;
             int32_t* l1 = m.list1[n & 1];
             int32_t* l2 = m.list2[n & 1];
-            const int n_ent = steps_build(t, m.vbs8, nq, topk, l1, l2, m.bits1, m.bits2, err, lane);
+            const int n_ent = steps_build(t, nq, topk, l1, l2, m.bits1, m.bits2, err, lane);
             const uint16_t* ent = reinterpret_cast<const uint16_t*>(l1);  // written over list 1
             const int tok0 = t.b * S;
             // proxy mode: after the selected cubes, ceil(nq / 128) steps over the proxy keys
@@ -348,8 +348,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 StepMeta meta;
                 meta.ma = (int)(ea >> 14);
                 meta.mb = (int)(eb >> 14);
-                meta.na = meta.ma != 0 ? m.vbs8[ja] : 0;
-                meta.nb = meta.mb != 0 ? m.vbs8[jb] : 0;
+                const int va = m.vbs8[ja], vb = m.vbs8[jb];  // 255: an invalid count, no tokens
+                meta.na = meta.ma != 0 && va <= 64 ? va : 0;
+                meta.nb = meta.mb != 0 && vb <= 64 ? vb : 0;
                 const bool last = s + 1 == n_steps;
                 meta.flags = (s == 0 ? 1 : 0) | (last ? 2 : 0);
                 const uint32_t word = step_word(meta) | (last && n == my_tiles - 1 ? kFinal : 0u);

@@ -344,17 +344,19 @@ __device__ __forceinline__ TileRef tile_ref(int t, int H, int nq, int tiles_per_
 // names the same cube), then the entries of list 2 that list 1 does not name.
 // A list that names a cube twice disables the sharing (list 1's entries are
 // all membership 1 and list 2's all membership 2), which keeps every
-// multiplicity.  Entries whose cube has no valid token are left out.
+// multiplicity.  A cube without valid tokens stays in the list; its half of
+// a step is empty.
 __device__ __forceinline__ bool test_bit(const uint32_t* bits, int j) { return (bits[j >> 5] >> (j & 31)) & 1u; }
 
-// The valid counts as bytes in shared memory (read for every list entry); a
-// count outside [0, 64] is kept as 255, which the list code treats as an
-// empty cube after latching the error.
-__device__ __forceinline__ void vbs_stage(const int32_t* __restrict__ vbs, int nq, uint8_t* vbs8)
+// The valid counts as bytes in shared memory; a count outside [0, 64] latches
+// an error and is kept as 255, which the kernel treats as an empty cube.
+__device__ __forceinline__ void vbs_stage(const int32_t* __restrict__ vbs, int nq, uint8_t* vbs8, int* err)
 {
     for (int c = threadIdx.x; c < nq; c += blockDim.x) {
         const int n = __ldg(vbs + c);
-        vbs8[c] = (uint8_t)(n < 0 || n > 64 ? 255 : n);
+        const bool bad = n < 0 || n > 64;
+        if (bad) atomicCAS(err, 0, (int)kErrVbs);
+        vbs8[c] = (uint8_t)(bad ? 255 : n);
     }
 }
 
@@ -375,15 +377,18 @@ __device__ __forceinline__ void lists_fetch(const TileRef& t, const int32_t* __r
 }
 
 // Build a tile's membership bitmaps and its entry list from its two selection
-// lists (fetched by lists_fetch), by the whole producer warp.  The entries are
-// written over list 1 (each 32-entry window of it is read before any entry
-// lands on it: after window w at most 32 (w + 1) entries exist, which end
-// within its first w + 1 windows' bytes).  Invalid cube ids latch an error
-// and are dropped; invalid vbs values latch an error and count as empty
-// cubes.  vbs8: the valid counts staged in shared memory (vbs_stage).
-// Returns the number of entries (warp-uniform).
-__device__ int steps_build(const TileRef& t, const uint8_t* vbs8, int nq, int topk, int32_t* l1, int32_t* l2,
-                           uint32_t* b1, uint32_t* b2, int* err, uint32_t lane)
+// lists (fetched by lists_fetch), by the whole producer warp.  Shared memory is
+// busy with the tensor core's operands and the TMA copies while this runs, so
+// the work is laid out for few round trips: up to kBuildBatch windows of both
+// lists at once, the first batch kept in registers from the bitmap pass to the
+// emission.  The entries are written over list 1 (each batch of it is read
+// before any entry lands on it: after windows 0 .. w at most 32 (w + 1) entries
+// exist, which end within their bytes).  Invalid cube ids latch an error and
+// are dropped.  Returns the number of entries (warp-uniform).
+constexpr int kBuildBatch = 4;
+
+__device__ int steps_build(const TileRef& t, int nq, int topk, int32_t* l1, int32_t* l2, uint32_t* b1, uint32_t* b2,
+                           int* err, uint32_t lane)
 {
     const int words = (nq + 31) >> 5;
     for (int w = lane; w < words; w += 32) {
@@ -394,62 +399,74 @@ __device__ int steps_build(const TileRef& t, const uint8_t* vbs8, int nq, int to
     const int len2 = t.i2 >= 0 ? topk : 0;
     cp_async_wait_all();
     __syncwarp();
-    // bitmaps by non-returning shared-memory ORs; a list names a cube twice iff
-    // its bitmap holds fewer bits than it has valid entries
-    int valid[2] = {0, 0};
-    for (int s = 0; s < 2; ++s) {
-        const int len = s == 0 ? len1 : len2;
-        int32_t* lst = s == 0 ? l1 : l2;
-        uint32_t* bits = s == 0 ? b1 : b2;
-        for (int e = lane; e < len; e += 32) {
-            int j = lst[e];
-            if (j < 0 || j >= nq) {
-                atomicCAS(err, 0, (int)kErrTopkIdx);
-                j = -1;
-            } else {
-                if (vbs8[j] > 64) atomicCAS(err, 0, (int)kErrVbs);
-                atomicOr(&bits[j >> 5], 1u << (j & 31));  // result unused: a reduction
-                ++valid[s];
+    // bitmaps by shared-memory ORs; a list names a cube twice iff one of its ORs
+    // finds the bit already set
+    bool dup = false;
+    int j0[2][kBuildBatch];  // the first batch (-1: none or invalid)
+    for (int base = 0; base < topk; base += 32 * kBuildBatch) {
+        int j[2][kBuildBatch];
+#pragma unroll
+        for (int s = 0; s < 2; ++s)
+#pragma unroll
+            for (int u = 0; u < kBuildBatch; ++u) {
+                const int e = base + 32 * u + (int)lane;
+                j[s][u] = e < (s == 0 ? len1 : len2) ? (s == 0 ? l1 : l2)[e] : -1;
             }
-            lst[e] = j;
+#pragma unroll
+        for (int s = 0; s < 2; ++s)
+#pragma unroll
+            for (int u = 0; u < kBuildBatch; ++u) {
+                const int e = base + 32 * u + (int)lane;
+                if (e >= (s == 0 ? len1 : len2)) continue;
+                const int jj = j[s][u];
+                if (jj < 0 || jj >= nq) {
+                    atomicCAS(err, 0, (int)kErrTopkIdx);
+                    (s == 0 ? l1 : l2)[e] = -1;
+                    j[s][u] = -1;
+                } else {
+                    const uint32_t bit = 1u << (jj & 31);
+                    dup |= (atomicOr(&(s == 0 ? b1 : b2)[jj >> 5], bit) & bit) != 0u;
+                }
+            }
+        if (base == 0) {
+#pragma unroll
+            for (int s = 0; s < 2; ++s)
+#pragma unroll
+                for (int u = 0; u < kBuildBatch; ++u) j0[s][u] = j[s][u];
         }
     }
     __syncwarp();
-    int set[2] = {0, 0};
-    for (int w = lane; w < words; w += 32) {
-        set[0] += __popc(b1[w]);
-        set[1] += __popc(b2[w]);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        valid[0] += __shfl_xor_sync(0xffffffffu, valid[0], o);
-        valid[1] += __shfl_xor_sync(0xffffffffu, valid[1], o);
-        set[0] += __shfl_xor_sync(0xffffffffu, set[0], o);
-        set[1] += __shfl_xor_sync(0xffffffffu, set[1], o);
-    }
-    const bool share = set[0] == valid[0] && set[1] == valid[1] && len1 > 0 && len2 > 0;
+    const bool share = !__any_sync(0xffffffffu, dup) && len1 > 0 && len2 > 0;
     uint16_t* ent = reinterpret_cast<uint16_t*>(l1);
     const uint32_t lt = (1u << lane) - 1u;  // lanes below this one
     int count = 0;
+#pragma unroll
     for (int s = 0; s < 2; ++s) {
         const int len = s == 0 ? len1 : len2;
         const int32_t* lst = s == 0 ? l1 : l2;
-        for (int base = 0; base < len; base += 32) {
-            const int e = base + (int)lane;
-            const int j = e < len ? lst[e] : -1;
-            const int n = j >= 0 ? vbs8[j] : 0;
-            bool q = n > 0 && n <= 64;
-            uint32_t mem = 1;
-            if (s == 0) {
-                if (q && share && test_bit(b2, j)) mem = 3;
-            } else {
-                mem = 2;
-                q = q && !(share && test_bit(b1, j));
+        for (int base = 0; base < len; base += 32 * kBuildBatch) {
+            bool q[kBuildBatch];
+            uint32_t code[kBuildBatch];
+#pragma unroll
+            for (int u = 0; u < kBuildBatch; ++u) {
+                const int e = base + 32 * u + (int)lane;
+                const int jj = base == 0 ? j0[s][u] : (e < len ? lst[e] : -1);
+                q[u] = jj >= 0;
+                uint32_t mem = s == 0 ? 1u : 2u;
+                if (q[u] && share) {
+                    const bool other = test_bit(s == 0 ? b2 : b1, jj);
+                    if (s == 0 && other) mem = 3u;  // both select it: walked with list 1
+                    if (s == 1 && other) q[u] = false;
+                }
+                code[u] = (uint32_t)jj | (mem << 14);
             }
-            const uint32_t mask = __ballot_sync(0xffffffffu, q);
-            __syncwarp();  // the window is read before entries land on list 1
-            if (q) ent[count + __popc(mask & lt)] = (uint16_t)((uint32_t)j | (mem << 14));
-            count += __popc(mask);
+            __syncwarp();  // the batch is read before entries land on list 1
+#pragma unroll
+            for (int u = 0; u < kBuildBatch; ++u) {
+                const uint32_t mask = __ballot_sync(0xffffffffu, q[u]);
+                if (q[u]) ent[count + __popc(mask & lt)] = (uint16_t)code[u];
+                count += __popc(mask);
+            }
         }
     }
     __syncwarp();
