@@ -317,14 +317,16 @@ def steps_per_tile(idx: np.ndarray, plan: np.ndarray | None, vbs: np.ndarray) ->
     return np.array(out)
 
 
-def time_fwd(vsa, args, n=10, warm=3):
-    """Average forward time (ms) over n calls, CUDA events on the current stream."""
+def time_fwd(vsa, args, n=10, warm=3, fn=None):
+    """Average forward time (ms) over n calls, CUDA events on the current stream
+    (fn: the call, vsa.fwd by default)."""
+    fn = fn or vsa.fwd
     for _ in range(warm):
-        vsa.fwd(*args[0], **args[1])
+        fn(*args[0], **args[1])
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
     for a, b in ev:
         a.record()
-        vsa.fwd(*args[0], **args[1])
+        fn(*args[0], **args[1])
         b.record()
     torch.cuda.synchronize()
     return statistics.mean(a.elapsed_time(b) for a, b in ev)
@@ -332,7 +334,8 @@ def time_fwd(vsa, args, n=10, warm=3):
 
 def run_extras(vsa, dev, cfg, qt, kt, vt, qc, kc, idx, vbs, peak):
     """The forward alone: the headline workload with the consecutive pairing and on
-    random selection lists, then the other configurations."""
+    random selection lists, the proxy-compensated forward, then the other
+    configurations."""
     out = torch.empty_like(qt)
     vbs_h = vbs.cpu().numpy()
     res = {}
@@ -360,6 +363,21 @@ def run_extras(vsa, dev, cfg, qt, kt, vt, qc, kc, idx, vbs, peak):
                         "steps_per_tile_mean": float(spt.mean()), "steps_total": int(spt.sum())}
         cases[name] = row
     res["pairing"] = cases
+
+    # proxy compensation: the same call with every omitted cube's mean key and summed
+    # value (vc formed by the fused tiling from the raster inputs)
+    T, Hh, W = cfg.grid
+    g = [synth.bits_to_torch(x).to(dev) for x in synth.grid_qkv(cfg)]
+    tiled = [torch.empty_like(qt) for _ in range(3)]
+    vc = torch.empty_like(kc)
+    vsa.tile_qkv(*g, cfg.grid, vbs, means=False, sums=True, out=tiled + [None, None, vc])
+    del g, tiled
+    ms_plain = fwd_case(qt, kt, vt, idx, vbs, cfg, plan)
+    ms_proxy = time_fwd(vsa, ((qt, kt, vt, idx, vbs, kc, vc, cfg.sm_scale), {"out": out, "plan": plan}),
+                        fn=vsa.fwd_proxy)
+    res["proxy"] = {"fwd_ms": ms_plain, "fwd_proxy_ms": ms_proxy, "overhead": ms_proxy / ms_plain - 1.0,
+                    "proxy_steps_per_tile": (len(vbs_h) + 127) // 128}
+    del vc
 
     # other configurations: forward alone (inputs tiled and routed by the library first)
     cfgs = {}
@@ -513,11 +531,14 @@ def main():
         import hashlib
 
         t = json.load(open(tpath))
-        src = os.path.join(ROOT, t.get("kernel_source", ""))
-        # the kernel the default forward runs (the traffic of another kernel does not apply)
-        timed = os.path.join(ROOT, "video_block_sparse_b200", "csrc", "fwd_pair.cu")
-        if (os.path.exists(src) and os.path.samefile(src, timed)
-                and hashlib.sha256(open(src, "rb").read()).hexdigest() == t.get("kernel_source_sha256")):
+        # the sources of the kernel the default forward runs, as they were when the
+        # counters were taken (the traffic of another kernel does not apply)
+        srcs = t.get("kernel_sources", {})
+        timed = {"video_block_sparse_b200/csrc/fwd_pair.cu", "video_block_sparse_b200/csrc/fwd_pair_common.cuh"}
+        if set(srcs) == timed and all(
+                os.path.exists(os.path.join(ROOT, f))
+                and hashlib.sha256(open(os.path.join(ROOT, f), "rb").read()).hexdigest() == h
+                for f, h in srcs.items()):
             traffic = t.get("bytes_per_launch")
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
