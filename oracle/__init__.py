@@ -60,9 +60,12 @@ def _load():
         lib.oracle_plan.argtypes = [P, I, I, I, I, P]
         lib.oracle_cube_sums.argtypes = [P, P, P, I, I, I, I, I]
         lib.oracle_fwd_proxy_items.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, ctypes.c_double, P, I64, P, P]
+        lib.oracle_fwd_bsr_items.argtypes = [P, P, P, P, P, P, P, I64, P, I, I, I, I, I, ctypes.c_double, P, I64, P, P,
+                                             P]
         for name in ("oracle_f64_to_bf16", "oracle_bf16_to_f64", "oracle_cube_counts", "oracle_tile",
                      "oracle_untile", "oracle_cube_means", "oracle_route", "oracle_fwd_items", "oracle_fwd_items_ex",
-                     "oracle_num_threads", "oracle_plan", "oracle_cube_sums", "oracle_fwd_proxy_items"):
+                     "oracle_num_threads", "oracle_plan", "oracle_cube_sums", "oracle_fwd_proxy_items",
+                     "oracle_fwd_bsr_items"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -182,6 +185,73 @@ def route(q: np.ndarray, k: np.ndarray, vbs: np.ndarray, topk: int, want_scores:
     _check(_load().oracle_route(_ptr(q), _ptr(k), _ptr(vbs), _ptr(idx), B, S, H, D, nq, topk,
                                 _ptr(scores) if want_scores else None), "route")
     return (idx, scores) if want_scores else idx
+
+
+# ---- route formats (TensorRT-LLM PR #7, the embedded FlashInfer PR, "Bitmask format"):
+# canonical BSR rows and packed UInt32 exact-block bitmaps, one row per (batch, head,
+# query cube); in a bitmap, bit c % 32 of word c / 32 selects cube c (the bit order is a
+# reading: least significant first), and bits at c >= Nq in the last word are ignored.
+
+def lists_to_bsr(topk_idx: np.ndarray):
+    """[B, H, Nq, topk] lists -> (indptr [B*H*Nq + 1], indices) int32, rows in order."""
+    B, H, nq, topk = topk_idx.shape
+    indptr = (np.arange(B * H * nq + 1, dtype=np.int64) * topk).astype(np.int32)
+    return indptr, np.ascontiguousarray(topk_idx.reshape(-1), dtype=np.int32)
+
+
+def bitmask_to_bsr(mask: np.ndarray, nq: int):
+    """[B, H, Nq, W] 32-bit words -> (indptr, indices): each row's selected cubes in
+    ascending order, padding bits ignored."""
+    B, H, rows_nq, W = mask.shape
+    assert rows_nq == nq and W == (nq + 31) // 32
+    words = np.ascontiguousarray(mask).view(np.uint32).reshape(-1, W)
+    indptr = [0]
+    indices = []
+    for row in words:
+        sel = [32 * w + bit for w in range(W) for bit in range(32) if (int(row[w]) >> bit) & 1 and 32 * w + bit < nq]
+        indices.extend(sel)
+        indptr.append(len(indices))
+    return np.asarray(indptr, np.int32), np.asarray(indices, np.int32)
+
+
+def bsr_to_bitmask(indptr: np.ndarray, indices: np.ndarray, B: int, H: int, nq: int) -> np.ndarray:
+    """BSR rows -> [B, H, Nq, ceil(Nq/32)] uint32 bitmaps (a cube named twice sets its
+    bit once)."""
+    W = (nq + 31) // 32
+    out = np.zeros((B * H * nq, W), np.uint32)
+    for r in range(B * H * nq):
+        for c in indices[indptr[r]:indptr[r + 1]]:
+            out[r, c // 32] |= np.uint32(1 << (c % 32))
+    return out.reshape(B, H, nq, W)
+
+
+def fwd_bsr_items(q, k, v, indptr, indices, vbs, sm_scale: float, items: np.ndarray, kc=None, vc=None,
+                  want_wabs: bool = False):
+    """The fine forward with the selections as BSR rows, plain or (kc, vc given)
+    proxy-compensated, for the listed (b, h, query cube) items. Returns out [n, 64, D],
+    lse [n, 64] (and, plain only, the weighted mean of |v| [n, 64, D]), float64.
+    sm_scale is used as the binary32 value a GPU kernel receives."""
+    B, S, H, D = q.shape
+    nq = S // 64
+    arrs = [np.ascontiguousarray(a, dtype=np.uint16) for a in (q, k, v)]
+    kcv = [None, None] if kc is None else [np.ascontiguousarray(a, dtype=np.uint16) for a in (kc, vc)]
+    indptr = np.ascontiguousarray(indptr, dtype=np.int32)
+    indices = np.ascontiguousarray(indices, dtype=np.int32)
+    assert indptr.shape == (B * H * nq + 1,)
+    vbs = np.ascontiguousarray(vbs, dtype=np.int32)
+    items = np.ascontiguousarray(items, dtype=np.int32).reshape(-1, 3)
+    n = items.shape[0]
+    out = np.empty((n, 64, D), dtype=np.float64)
+    lse = np.empty((n, 64), dtype=np.float64)
+    wabs = np.empty((n, 64, D), dtype=np.float64) if want_wabs else None
+    idx_buf = indices if indices.size else np.zeros(1, np.int32)
+    opt = lambda a: None if a is None else _ptr(a)  # noqa: E731
+    _check(_load().oracle_fwd_bsr_items(*(_ptr(a) for a in arrs), opt(kcv[0]), opt(kcv[1]), _ptr(indptr),
+                                        _ptr(idx_buf), int(indices.size), _ptr(vbs), B, S, H, D, nq,
+                                        float(np.float32(sm_scale)), _ptr(items), n, _ptr(out), _ptr(lse),
+                                        opt(wabs)),
+           "fwd_bsr_items")
+    return (out, lse, wabs) if want_wabs else (out, lse)
 
 
 def fwd_items(q, k, v, topk_idx, vbs, sm_scale: float, items: np.ndarray, want_wabs: bool = False):

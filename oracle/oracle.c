@@ -479,6 +479,127 @@ int oracle_fwd_proxy_items(const uint16_t *q, const uint16_t *k, const uint16_t 
     return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
 }
 
+/* ------------------------------------------------------------------ BSR rows
+ *
+ * TensorRT-LLM PR #7 (the embedded FlashInfer PR "support proxy-compensated
+ * block-sparse attention", "Bitmask format"): exact-block selections as
+ * canonical BSR rows (block_indptr / block_indices) or packed UInt32 bitmaps
+ * per (batch, KV head, Q block); both describe the same selection, and a
+ * bitmap is first written out as BSR rows (oracle/__init__.py).  Here a row is
+ * r = (b*H + h)*Nq + i and lists the cubes indices[indptr[r] .. indptr[r+1])
+ * of query cube i, any number of them, multiplicity kept.  Without kc and vc
+ * (both NULL) the result is the fine forward over the listed cubes' valid
+ * tokens; with them, every cube with vbs > 0 that the row does not list adds
+ * its proxy as in oracle_fwd_proxy_items.  wabs (plain mode, may be NULL): the
+ * softmax-weighted mean of |v|. */
+int oracle_fwd_bsr_items(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *kc,
+                         const uint16_t *vc, const int32_t *indptr, const int32_t *indices, int64_t nnz,
+                         const int32_t *vbs, int B, int S, int H, int D, int Nq, double sigma,
+                         const int32_t *items, int64_t n_items, double *out, double *lse, double *wabs)
+{
+    if (B <= 0 || H <= 0 || D <= 0 || Nq <= 0 || S != 64 * Nq || nnz < 0) return ORACLE_ERR_ARG;
+    if ((kc == NULL) != (vc == NULL) || (kc != NULL && wabs != NULL)) return ORACLE_ERR_ARG;
+    for (int c = 0; c < Nq; ++c)
+        if (vbs[c] < 0 || vbs[c] > 64) return ORACLE_ERR_ARG;
+    int64_t maxlen = 0;
+    for (int64_t it = 0; it < n_items; ++it) {
+        int b = items[3 * it], h = items[3 * it + 1], i = items[3 * it + 2];
+        if (b < 0 || b >= B || h < 0 || h >= H || i < 0 || i >= Nq) return ORACLE_ERR_ARG;
+        int64_t r = ((int64_t)b * H + h) * Nq + i;
+        if (indptr[r] < 0 || indptr[r + 1] < indptr[r] || indptr[r + 1] > nnz) return ORACLE_ERR_ARG;
+        for (int64_t t = indptr[r]; t < indptr[r + 1]; ++t)
+            if (indices[t] < 0 || indices[t] >= Nq) return ORACLE_ERR_ARG;
+        if (indptr[r + 1] - indptr[r] > maxlen) maxlen = indptr[r + 1] - indptr[r];
+    }
+    int failed = 0;
+#pragma omp parallel
+    {
+        int64_t *keys = (int64_t *)malloc((size_t)(maxlen * 64 + 1) * sizeof(int64_t));
+        int32_t *omitted = (int32_t *)malloc((size_t)Nq * sizeof(int32_t));
+        char *chosen = (char *)malloc((size_t)Nq);
+        double *x = (double *)malloc((size_t)(maxlen * 64 + Nq + 1) * sizeof(double));
+        if (!keys || !omitted || !chosen || !x) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t it = 0; it < n_items; ++it) {
+            if (!keys || !omitted || !chosen || !x) continue;
+            int b = items[3 * it], h = items[3 * it + 1], i = items[3 * it + 2];
+            int64_t r = ((int64_t)b * H + h) * Nq + i;
+            /* the listed cubes' tokens (multiplicity kept) and, with proxies, the cubes not listed */
+            int64_t nkeys = 0;
+            for (int c = 0; c < Nq; ++c) chosen[c] = 0;
+            for (int64_t t = indptr[r]; t < indptr[r + 1]; ++t) {
+                int j = indices[t];
+                chosen[j] = 1;
+                for (int u = 0; u < vbs[j]; ++u) keys[nkeys++] = 64LL * j + u;
+            }
+            int nom = 0;
+            if (kc != NULL)
+                for (int c = 0; c < Nq; ++c)
+                    if (!chosen[c] && vbs[c] > 0) omitted[nom++] = c;
+            for (int rr = 0; rr < 64; ++rr) {
+                int64_t s = 64LL * i + rr;
+                const uint16_t *qs = q + (((int64_t)b * S + s) * H + h) * D;
+                double *o = out + (it * 64 + rr) * D;
+                if (nkeys == 0 && nom == 0) {
+                    for (int d = 0; d < D; ++d) o[d] = 0.0;
+                    if (wabs != NULL)
+                        for (int d = 0; d < D; ++d) wabs[(it * 64 + rr) * D + d] = 0.0;
+                    lse[it * 64 + rr] = -INFINITY;
+                    continue;
+                }
+                double m = -INFINITY;
+                for (int64_t n = 0; n < nkeys; ++n) {
+                    const uint16_t *ku = k + (((int64_t)b * S + keys[n]) * H + h) * D;
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) dot += bf16_bits_to_f64(qs[d]) * bf16_bits_to_f64(ku[d]);
+                    x[n] = sigma * dot;
+                    if (x[n] > m) m = x[n];
+                }
+                for (int n = 0; n < nom; ++n) {
+                    const uint16_t *kj = kc + (((int64_t)b * H + h) * Nq + omitted[n]) * D;
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) dot += bf16_bits_to_f64(qs[d]) * bf16_bits_to_f64(kj[d]);
+                    x[nkeys + n] = sigma * dot;
+                    if (x[nkeys + n] > m) m = x[nkeys + n];
+                }
+                double l = 0.0;
+                for (int d = 0; d < D; ++d) o[d] = 0.0;
+                for (int64_t n = 0; n < nkeys; ++n) {
+                    double p = exp(x[n] - m);
+                    const uint16_t *vu = v + (((int64_t)b * S + keys[n]) * H + h) * D;
+                    l += p;
+                    for (int d = 0; d < D; ++d) o[d] += p * bf16_bits_to_f64(vu[d]);
+                }
+                for (int n = 0; n < nom; ++n) {
+                    double p = exp(x[nkeys + n] - m);
+                    const uint16_t *vj = vc + (((int64_t)b * H + h) * Nq + omitted[n]) * D;
+                    l += (double)vbs[omitted[n]] * p; /* the token mass the proxy stands for */
+                    for (int d = 0; d < D; ++d) o[d] += p * bf16_bits_to_f64(vj[d]);
+                }
+                for (int d = 0; d < D; ++d) o[d] /= l;
+                lse[it * 64 + rr] = m + log(l);
+                if (wabs != NULL) {
+                    double *a = wabs + (it * 64 + rr) * D;
+                    for (int d = 0; d < D; ++d) a[d] = 0.0;
+                    for (int64_t n = 0; n < nkeys; ++n) {
+                        double w = exp(x[n] - m) / l;
+                        const uint16_t *vu = v + (((int64_t)b * S + keys[n]) * H + h) * D;
+                        for (int d = 0; d < D; ++d) a[d] += w * fabs(bf16_bits_to_f64(vu[d]));
+                    }
+                }
+            }
+        }
+        free(keys);
+        free(omitted);
+        free(chosen);
+        free(x);
+    }
+    return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}
+
 int oracle_fwd_items(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                      const int32_t *topk_idx, const int32_t *vbs,
                      int B, int S, int H, int D, int Nq, int topk, double sigma,

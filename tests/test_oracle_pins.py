@@ -642,3 +642,100 @@ def test_proxy_uniform_logits_closed_form(oracle_lib):
         cnt = sum(int(vbs[j]) for j in sel) + sum(int(vbs[j]) for j in om)
         assert np.allclose(out[n], np.broadcast_to(num / cnt, (64, 128)), rtol=0, atol=1e-13)
         assert np.allclose(lse[n], math.log(cnt), rtol=0, atol=1e-13)
+
+
+# ------------------------------------------------------------------ route formats
+# TensorRT-LLM PR #7 (the embedded FlashInfer PR, "Bitmask format"): canonical BSR rows and
+# packed UInt32 exact-block bitmaps per (batch, head, query block); padding bits in the last
+# word are ignored.
+
+def _bsr_case(seed, nq=7, H=2, max_len=5, dup=True):
+    g = np.random.default_rng(seed)
+    x = [synth.f32_to_bf16_bits((g.standard_normal((1, 64 * nq, H, 128)) * 1.5).astype(np.float32))
+         for _ in range(3)]
+    vbs = g.integers(0, 65, size=nq).astype(np.int32)
+    vbs[0] = 64
+    indptr, indices = [0], []
+    for r in range(H * nq):
+        n = int(g.integers(0, max_len + 1)) if r % 5 else 0  # some rows empty
+        row = g.choice(nq, size=n, replace=dup).tolist()
+        indices.extend(row)
+        indptr.append(len(indices))
+    return x[0], x[1], x[2], vbs, np.asarray(indptr, np.int32), np.asarray(indices, np.int32)
+
+
+def test_bsr_rows_equal_softmax_over_listed_tokens(oracle_lib):
+    """Variable-length rows, repeats and empty rows: the softmax over exactly the listed
+    tokens (a cube named twice counts twice), written out with torch in float64."""
+    q, k, v, vbs, indptr, indices = _bsr_case(21)
+    nq, H = len(vbs), q.shape[2]
+    items = oracle_lib.all_items(1, H, nq)
+    out, lse, wabs = oracle_lib.fwd_bsr_items(q, k, v, indptr, indices, vbs, 0.125, items, want_wabs=True)
+    sigma = float(np.float32(0.125))
+    f = lambda a: torch.from_numpy(oracle_lib.bf16_to_f64(a))
+    Q, K, V = f(q)[0], f(k)[0], f(v)[0]
+    for n, (b, h, i) in enumerate(items):
+        r = h * nq + i
+        toks = [64 * j + u for j in indices[indptr[r]:indptr[r + 1]].tolist() for u in range(vbs[j])]
+        if not toks:
+            assert np.all(out[n] == 0.0) and np.all(np.isneginf(lse[n])) and np.all(wabs[n] == 0.0)
+            continue
+        logits = sigma * Q[64 * i: 64 * i + 64, h] @ K[toks, h].T
+        w = torch.softmax(logits, dim=1)
+        assert np.allclose(out[n], (w @ V[toks, h]).numpy(), rtol=0, atol=1e-12)
+        assert np.allclose(lse[n], torch.logsumexp(logits, dim=1).numpy(), rtol=0, atol=1e-12)
+        assert np.allclose(wabs[n], (w @ V[toks, h].abs()).numpy(), rtol=0, atol=1e-12)
+
+
+def test_bsr_rows_with_proxies_equal_softmax_with_proxy_keys(oracle_lib):
+    """Proxies over the cubes a row does not list: the softmax over the listed tokens and
+    one key per other cube with valid tokens (mean key, log-weight log vbs[j], value
+    vc_j / vbs[j])."""
+    q, k, v, vbs, indptr, indices = _bsr_case(22, dup=False)
+    nq, H = len(vbs), q.shape[2]
+    kc, vc = oracle_lib.cube_means(k, vbs), oracle_lib.cube_sums(v, vbs)
+    items = oracle_lib.all_items(1, H, nq)
+    out, lse = oracle_lib.fwd_bsr_items(q, k, v, indptr, indices, vbs, 0.25, items, kc=kc, vc=vc)
+    sigma = 0.25
+    f = lambda a: torch.from_numpy(oracle_lib.bf16_to_f64(a))
+    Q, K, V, KC, VC = f(q)[0], f(k)[0], f(v)[0], f(kc)[0], f(vc)[0]
+    for n, (b, h, i) in enumerate(items):
+        r = h * nq + i
+        sel = indices[indptr[r]:indptr[r + 1]].tolist()
+        toks = [64 * j + u for j in sel for u in range(vbs[j])]
+        om = [j for j in range(nq) if j not in sel and vbs[j] > 0]
+        qs = Q[64 * i: 64 * i + 64, h]
+        logits = torch.cat([sigma * qs @ K[toks, h].T,
+                            sigma * qs @ KC[h, om].T + torch.log(torch.tensor(vbs[om], dtype=torch.float64))], dim=1)
+        vals = torch.cat([V[toks, h], VC[h, om] / torch.tensor(vbs[om], dtype=torch.float64)[:, None]], dim=0)
+        assert np.allclose(out[n], (torch.softmax(logits, dim=1) @ vals).numpy(), rtol=0, atol=1e-12)
+        assert np.allclose(lse[n], torch.logsumexp(logits, dim=1).numpy(), rtol=0, atol=1e-12)
+
+
+def test_bitmask_bit_order_and_padding(oracle_lib):
+    """A hand-worked 37-cube row: bit c % 32 of word c / 32 selects cube c, and the
+    27 bits past cube 36 in the last word are ignored."""
+    nq = 37
+    mask = np.zeros((1, 1, nq, 2), np.uint32)
+    mask[0, 0, 3] = [(1 << 0) | (1 << 5) | (1 << 31), (1 << 0) | (1 << 4) | np.uint32(0xFFFFFFE0)]
+    indptr, indices = oracle_lib.bitmask_to_bsr(mask, nq)
+    assert indptr[3] == 0 and indptr[4] == 5 and indptr[-1] == 5
+    assert indices.tolist() == [0, 5, 31, 32, 36]
+    back = oracle_lib.bsr_to_bitmask(indptr, indices, 1, 1, nq)
+    assert back[0, 0, 3].tolist() == [(1 << 0) | (1 << 5) | (1 << 31), (1 << 0) | (1 << 4)]
+    assert int(back.sum()) == int(back[0, 0, 3].sum())
+
+
+def test_route_formats_describe_the_same_selection(oracle_lib):
+    """Distinct lists in ascending order, their BSR rows and their bitmaps give the same
+    forward; the BSR rows of fixed lists are the lists in order."""
+    q, k, v, vbs, _ = _proxy_case(23, nq=6, topk=3)
+    idx = np.sort(synth.random_topk(23, 1, 2, 6, 3), axis=-1).astype(np.int32)
+    indptr, indices = oracle_lib.lists_to_bsr(idx)
+    assert indptr.tolist() == list(range(0, 3 * 12 + 1, 3)) and indices.tolist() == idx.reshape(-1).tolist()
+    ip2, ix2 = oracle_lib.bitmask_to_bsr(oracle_lib.bsr_to_bitmask(indptr, indices, 1, 2, 6), 6)
+    assert ip2.tolist() == indptr.tolist() and ix2.tolist() == indices.tolist()
+    items = oracle_lib.all_items(1, 2, 6)
+    o1, l1 = oracle_lib.fwd_items(q, k, v, idx, vbs, 0.1, items)
+    o2, l2 = oracle_lib.fwd_bsr_items(q, k, v, indptr, indices, vbs, 0.1, items)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
