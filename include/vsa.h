@@ -184,6 +184,45 @@ VSA_API int vsa_fwd_proxy(const vsa_bf16 *q, const vsa_bf16 *k, const vsa_bf16 *
                           int flags, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * vsa_fwd_bsr / vsa_fwd_bitmask -- the fine forward with the selections in the
+ * route formats of TensorRT-LLM PR #7 (the embedded FlashInfer PR "support
+ * proxy-compensated block-sparse attention", "Bitmask format"): canonical BSR
+ * rows, or packed UInt32 exact-block bitmaps per (batch, head, query cube),
+ * either one with or without proxy compensation.  Both formats become the same
+ * per-tile step list as topk_idx rows, so a BSR row, a bitmap row and a
+ * topk_idx row that name the same cubes in ascending order give bit-identical
+ * results.
+ *
+ * vsa_fwd_bsr: row r = (b*H + h)*Nq + i (query cube i of batch b, head h)
+ * selects the cubes block_indices[block_indptr[r] .. block_indptr[r+1]), in
+ * that order, any number from 0 to 1024 (a cube named twice counts twice).
+ *   block_indptr   [B*H*Nq + 1] int32 in
+ *   block_indices  [nnz] int32 in (may be NULL when nnz == 0)
+ * A row outside [0, nnz] or with end < start is taken as empty and latches
+ * device error 5; a row of more than 1024 entries keeps its first 1024 and
+ * latches 5; an index outside [0, Nq) is dropped and latches 1.
+ *
+ * vsa_fwd_bitmask: bit c % 32 of word c / 32 of row (b, h, i) selects cube c.
+ *   mask  [B, H, Nq, ceil(Nq / 32)] uint32 in
+ * Bits at c >= Nq in a row's last word are ignored.  A row of more than 1024
+ * cubes keeps its lowest 1024 and latches device error 5.
+ *
+ * Both: kc and vc both NULL (plain forward) or both set (proxy compensation as
+ * in vsa_fwd_proxy, over the cubes a row does not select); plan as in
+ * vsa_fwd_planned (NULL: consecutive pairs).  Other arguments, numerics and
+ * errors as vsa_fwd_ex; VSA_ERR_NULL also for exactly one of kc, vc, and
+ * VSA_ERR_ARG for nnz < 0.  Every pointer is a device pointer, 16-byte aligned.
+ * ---------------------------------------------------------------------- */
+VSA_API int vsa_fwd_bsr(const vsa_bf16 *q, const vsa_bf16 *k, const vsa_bf16 *v, const int32_t *block_indptr,
+                        const int32_t *block_indices, int nnz, const int32_t *vbs, const vsa_bf16 *kc,
+                        const vsa_bf16 *vc, const int32_t *plan, vsa_bf16 *out, float *lse, int B, int S, int H,
+                        int D, int Nq, float sm_scale, int flags, cudaStream_t stream);
+VSA_API int vsa_fwd_bitmask(const vsa_bf16 *q, const vsa_bf16 *k, const vsa_bf16 *v, const uint32_t *mask,
+                            const int32_t *vbs, const vsa_bf16 *kc, const vsa_bf16 *vc, const int32_t *plan,
+                            vsa_bf16 *out, float *lse, int B, int S, int H, int D, int Nq, float sm_scale, int flags,
+                            cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * vsa_route -- cube-mean q.k routing that builds topk_idx.
  *
  * "align VisualGen VSA with block-sparse FMHA" (TensorRT-LLM PR #7), review
@@ -360,7 +399,9 @@ VSA_API int vsa_stall_check(int *result, cudaStream_t stream);
  * VSA_ERR_DEVICE (and clears the word), or VSA_ERR_LAUNCH if the stream
  * reports a CUDA error.  `detail` (may be NULL) receives the latched code:
  * 1 = topk_idx value out of range, 2 = vbs value out of range,
- * 3 = a bounded pipeline wait ran out, 4 = a tile plan entry out of range.
+ * 3 = a bounded pipeline wait ran out, 4 = a tile plan entry out of range,
+ * 5 = a BSR row outside the index array or longer than 1024 entries, or a
+ * bitmap row of more than 1024 cubes.
  * ---------------------------------------------------------------------- */
 VSA_API int vsa_device_status(cudaStream_t stream, int *detail);
 

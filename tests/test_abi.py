@@ -150,6 +150,27 @@ def test_fwd_proxy_rejects_bad_arguments_without_a_device(vsa):
     assert lib.vsa_fwd_proxy(p, p, p, p, p, p, p, None, p, None, 1, 512, 2, 128, 8, 2, 0.1, 2, None) == -1  # flag
 
 
+def test_fwd_bsr_and_bitmask_reject_bad_arguments_without_a_device(vsa):
+    p = _fake(1 << 20)
+    lib = vsa.get_lib()
+    tail = (1, 512, 2, 128, 8, 0.1, 0, None)  # B, S, H, D, Nq, scale, flags, stream
+    # vsa_fwd_bsr(q, k, v, indptr, indices, nnz, vbs, kc, vc, plan, out, lse, ...)
+    assert lib.vsa_fwd_bsr(p, p, p, p, p, -1, p, None, None, None, p, None, *tail) == -1  # nnz < 0
+    assert lib.vsa_fwd_bsr(p, p, p, p, p, 4, p, None, None, None, p, None, 1, 512, 2, 64, 8, 0.1, 0, None) == -1
+    assert lib.vsa_fwd_bsr(p, p, p, p, p, 4, p, None, None, None, p, None, 1, 512, 2, 128, 8, 0.1, 4, None) == -1
+    assert lib.vsa_fwd_bsr(p, p, p, None, p, 4, p, None, None, None, p, None, *tail) == -2  # indptr
+    assert lib.vsa_fwd_bsr(p, p, p, p, None, 4, p, None, None, None, p, None, *tail) == -2  # indices, nnz > 0
+    assert lib.vsa_fwd_bsr(p, p, p, p, p, 4, p, p, None, None, p, None, *tail) == -2  # kc without vc
+    assert lib.vsa_fwd_bsr(p, p, p, _fake((1 << 20) + 4), p, 4, p, None, None, None, p, None, *tail) == -3
+    assert lib.vsa_fwd_bsr(p, p, p, p, _fake((1 << 20) + 4), 4, p, None, None, None, p, None, *tail) == -3
+    # vsa_fwd_bitmask(q, k, v, mask, vbs, kc, vc, plan, out, lse, ...)
+    assert lib.vsa_fwd_bitmask(p, p, p, p, p, None, None, None, p, None, 1, 512, 2, 64, 8, 0.1, 0, None) == -1
+    assert lib.vsa_fwd_bitmask(p, p, p, p, p, None, None, None, p, None, 1, 512, 2, 128, 9000, 0.1, 0, None) == -1
+    assert lib.vsa_fwd_bitmask(p, p, p, None, p, None, None, None, p, None, *tail) == -2  # mask
+    assert lib.vsa_fwd_bitmask(p, p, p, p, p, None, p, None, p, None, *tail) == -2  # vc without kc
+    assert lib.vsa_fwd_bitmask(p, p, p, _fake((1 << 20) + 8), p, None, None, None, p, None, *tail) == -3
+
+
 def test_route_noalloc_checks_arguments_before_its_array_limit(vsa):
     """Bad arguments are reported as by vsa_route, even for a problem larger than
     the fixed array, and before any device is touched."""

@@ -563,3 +563,206 @@ def test_fwd_proxy_with_every_cube_selected_is_the_plain_forward(vsa):
     torch.cuda.synchronize()
     _no_device_error(vsa)
     assert torch.equal(a.float(), b.float()) and torch.equal(la, lb)
+
+
+# ------------------------------------------------------------------ route formats (BSR, bitmaps)
+
+def _i32(a) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
+
+
+def _mask_dev(mask: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(mask).view(np.int32)).cuda()
+
+
+def _check_bsr(p: common.Prepared, indptr, indices, out, lse, items, tag, flags=0, kc=None, vc=None, rule=True):
+    """A forward over BSR rows (or bitmaps written out as BSR rows) against the oracle's,
+    every listed row: the card's rule (rule=True), else for the plain forward the
+    default mode's bound (with proxies the cosine and lse checks alone, as for
+    vsa_fwd_proxy)."""
+    bound_mode = not rule and kc is None
+    got = oracle.fwd_bsr_items(p.qt, p.kt, p.vt, indptr, indices, p.vbs, p.cfg.sm_scale, items, kc=kc, vc=vc,
+                               want_wabs=bound_mode)
+    o64, l64, wabs = got if bound_mode else (*got, None)
+    rows = common.gather_items(out, items)
+    res = common.compare(rows, o64, items[:, 1] + 1000 * items[:, 0])
+    print(f"\n[{tag}] gate {res['gate']}\n[{tag}] vs fp64 {res['fp64']}")
+    if rule:
+        assert res["gate"]["ok"], res
+    elif bound_mode:
+        bnd = common.within_default_bound(rows, o64, wabs)
+        print(f"[{tag}] default-mode bound {bnd}")
+        assert bnd["ok"], bnd
+    assert res["fp64"]["finite"] and res["fp64"]["min_head_cos"] >= 0.9999, res["fp64"]
+    got_lse = common.gather_lse(lse, items)
+    fin = np.isfinite(l64)
+    assert np.array_equal(fin, np.isfinite(got_lse))
+    assert np.all(rows[~fin] == 0.0)
+    bound = common.lse_bound(p.qt, p.kt, items, p.cfg.sm_scale, default_mode=flags == 0)
+    assert np.all(np.abs(got_lse[fin] - l64[fin]) <= bound[fin]), float(np.max(np.abs(got_lse[fin] - l64[fin])))
+
+
+@pytest.mark.parametrize("proxy", [False, True])
+@pytest.mark.parametrize("plan", [False, True])
+def test_fwd_route_formats_are_bit_identical(vsa, proxy, plan):
+    """Distinct lists in ascending order as topk_idx rows, as BSR rows and as bitmaps:
+    the same step lists, so bit-identical out and lse; every row against the oracle."""
+    p = common.prepare("wan480", H=3, grid=(9, 10, 11), topk=7, B=2)
+    p.idx = np.sort(p.idx, axis=-1).astype(np.int32)
+    B, H, nq = p.cfg.B, p.cfg.H, p.nq
+    indptr, indices = oracle.lists_to_bsr(p.idx)
+    mask = oracle.bsr_to_bitmask(indptr, indices, B, H, nq)
+    q, k, v = common.dev(p.qt), common.dev(p.kt), common.dev(p.vt)
+    idx, vbs = _i32(p.idx), _i32(p.vbs)
+    kc, vc = _proxy_inputs(p) if proxy else (None, None)
+    kcd, vcd = (common.dev(kc), common.dev(vc)) if proxy else (None, None)
+    pl = vsa.plan(idx) if plan else None
+    if proxy:
+        a, la = vsa.fwd_proxy(q, k, v, idx, vbs, kcd, vcd, p.cfg.sm_scale, want_lse=True, plan=pl)
+    else:
+        a, la = vsa.fwd(q, k, v, idx, vbs, p.cfg.sm_scale, want_lse=True, plan=pl)
+    b, lb = vsa.fwd_bsr(q, k, v, _i32(indptr), _i32(indices), vbs, p.cfg.sm_scale, kc=kcd, vc=vcd, want_lse=True,
+                        plan=pl)
+    c, lc = vsa.fwd_bitmask(q, k, v, _mask_dev(mask), vbs, p.cfg.sm_scale, kc=kcd, vc=vcd, want_lse=True, plan=pl)
+    torch.cuda.synchronize()
+    _no_device_error(vsa)
+    for x, lx in ((b, lb), (c, lc)):
+        assert torch.equal(a.view(torch.int16), x.view(torch.int16))
+        assert torch.equal(la.view(torch.int32), lx.view(torch.int32))
+    _check_bsr(p, indptr, indices, c, lc, oracle.all_items(B, H, nq), f"formats/{int(proxy)}/{int(plan)}", 0,
+               kc=kc, vc=vc)
+
+
+@pytest.mark.parametrize("flags", [0, 1])
+@pytest.mark.parametrize("proxy", [False, True])
+def test_fwd_bsr_variable_rows(vsa, flags, proxy):
+    """BSR rows of 0 to 12 cubes in any order, repeats included, empty cubes: every row."""
+    p = _small(40, nq=14, H=3, topk=1, vbs=[64, 0, 17, 33, 1, 64, 0, 48, 5, 64, 64, 9, 64, 22])
+    g = np.random.default_rng(41)
+    B, H, nq = 1, 3, 14
+    indptr, indices = [0], []
+    for r in range(B * H * nq):
+        n = int(g.integers(0, 13)) if r % 7 else 0
+        indices.extend(g.choice(nq, size=n, replace=bool(r % 3 == 0)).tolist())
+        indptr.append(len(indices))
+    indptr, indices = np.asarray(indptr, np.int32), np.asarray(indices, np.int32)
+    q, k, v = common.dev(p.qt), common.dev(p.kt), common.dev(p.vt)
+    kc, vc = _proxy_inputs(p) if proxy else (None, None)
+    out, lse = vsa.fwd_bsr(q, k, v, _i32(indptr), _i32(indices), _i32(p.vbs), p.cfg.sm_scale,
+                           kc=common.dev(kc) if proxy else None, vc=common.dev(vc) if proxy else None,
+                           want_lse=True, flags=flags)
+    torch.cuda.synchronize()
+    _no_device_error(vsa)
+    _check_bsr(p, indptr, indices, out, lse, oracle.all_items(B, H, nq), f"bsr-var/{flags}/{int(proxy)}", flags,
+               kc=kc, vc=vc, rule=flags == 1)
+
+
+def test_fwd_bitmask_padding_bits_are_ignored(vsa):
+    """Random bitmaps of a 37-cube grid: setting the 27 padding bits of every row's last
+    word changes nothing (bit for bit, no error); every row against the oracle."""
+    p = _small(42, nq=37, H=2, topk=1)
+    g = np.random.default_rng(43)
+    B, H, nq = 1, 2, 37
+    mask = (g.random((B, H, nq, 2, 32)) < 0.2)
+    mask[..., 1, 5:] = False
+    words = (mask.astype(np.uint64) << np.arange(32, dtype=np.uint64)).sum(axis=-1).astype(np.uint32)
+    dirty = words.copy()
+    dirty[..., 1] |= np.uint32(0xFFFFFFE0)
+    q, k, v = common.dev(p.qt), common.dev(p.kt), common.dev(p.vt)
+    vbs = _i32(p.vbs)
+    a, la = vsa.fwd_bitmask(q, k, v, _mask_dev(words), vbs, p.cfg.sm_scale, want_lse=True)
+    b, lb = vsa.fwd_bitmask(q, k, v, _mask_dev(dirty), vbs, p.cfg.sm_scale, want_lse=True)
+    torch.cuda.synchronize()
+    _no_device_error(vsa)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16)) and torch.equal(la.view(torch.int32),
+                                                                                  lb.view(torch.int32))
+    indptr, indices = oracle.bitmask_to_bsr(dirty, nq)
+    _check_bsr(p, indptr, indices, b, lb, oracle.all_items(B, H, nq), "bitmask-pad", 0, rule=False)
+
+
+def test_fwd_bsr_bad_rows_latch_error_and_are_empty(vsa):
+    """A row reaching past nnz and a row with end < start latch error 5 and are taken as
+    empty (out 0, lse -inf); an index out of range latches 1 and is dropped; the other
+    rows are unaffected."""
+    p = _small(44, nq=5, H=1, topk=1, vbs=[64, 64, 30, 64, 64])
+    indptr = np.array([0, 2, 4, 3, 5, 9], np.int32)  # row 2: end < start; row 4: past nnz = 8
+    indices = np.array([0, 1, 2, 3, 4, 0, 1, 2], np.int32)
+    q, k, v = common.dev(p.qt), common.dev(p.kt), common.dev(p.vt)
+    out, lse = vsa.fwd_bsr(q, k, v, _i32(indptr), _i32(indices), _i32(p.vbs), p.cfg.sm_scale, want_lse=True)
+    rc, detail = vsa.device_status()
+    assert rc == -7 and detail == 5
+    clean_ptr = np.array([0, 2, 4, 4, 6, 6], np.int32)  # the same rows, the bad ones empty
+    clean_idx = np.array([0, 1, 2, 3, 3, 4], np.int32)
+    _check_bsr(p, clean_ptr, clean_idx, out, lse, oracle.all_items(1, 1, 5), "bsr-bad", 0, rule=False)
+    bad = clean_idx.copy()
+    bad[1] = 9
+    out2 = vsa.fwd_bsr(q, k, v, _i32(clean_ptr), _i32(bad), _i32(p.vbs), p.cfg.sm_scale)
+    rc, detail = vsa.device_status()
+    assert rc == -7 and detail == 1
+    assert torch.isfinite(out2.float()).all()
+
+
+def test_fwd_bitmask_row_over_1024_cubes_keeps_its_first_1024(vsa):
+    """1100 cubes, one row selecting all of them: error 5, and the row attends to its
+    lowest 1024 cubes (the oracle over those); the other rows are unaffected."""
+    nq = 1100
+    p = _small(45, nq=nq, H=1, topk=1, vbs=np.full(nq, 64, np.int32))
+    g = np.random.default_rng(46)
+    W = (nq + 31) // 32
+    words = np.zeros((1, 1, nq, W), np.uint32)
+    sel = [g.choice(nq, size=5, replace=False) for _ in range(nq)]
+    for i in range(nq):
+        for c in sel[i]:
+            words[0, 0, i, c // 32] |= np.uint32(1 << (c % 32))
+    words[0, 0, 7] = np.uint32(0xFFFFFFFF)
+    q, k, v = common.dev(p.qt), common.dev(p.kt), common.dev(p.vt)
+    out, lse = vsa.fwd_bitmask(q, k, v, _mask_dev(words), _i32(p.vbs), p.cfg.sm_scale, want_lse=True)
+    rc, detail = vsa.device_status()
+    assert rc == -7 and detail == 5
+    kept = words.copy()
+    kept[0, 0, 7] = 0
+    kept[0, 0, 7, :32] = np.uint32(0xFFFFFFFF)  # cubes 0..1023
+    indptr, indices = oracle.bitmask_to_bsr(kept, nq)
+    items = np.array([[0, 0, 7], [0, 0, 0], [0, 0, nq - 1]], np.int32)
+    _check_bsr(p, indptr, indices, out, lse, items, "bitmask-1024", 0, rule=False)
+
+
+def test_fwd_routes_live_under_cuda_graph_replay(vsa):
+    """A captured forward reads its routes from the same buffers at every replay: new
+    bitmaps (and new topk lists) written in place between replays give the results an
+    eager call gives for them."""
+    p = common.prepare("wan480", H=2, grid=(9, 10, 11), topk=6, B=1)
+    B, H, nq = 1, 2, p.nq
+    q, k, v = common.dev(p.qt), common.dev(p.kt), common.dev(p.vt)
+    vbs = _i32(p.vbs)
+    g = np.random.default_rng(47)
+    lists = [np.sort(synth.random_topk(int(s), B, H, nq, 6), axis=-1).astype(np.int32) for s in g.integers(0, 1000, 3)]
+    masks = [oracle.bsr_to_bitmask(*oracle.lists_to_bsr(x), B, H, nq) for x in lists]
+    mask_buf, idx_buf = _mask_dev(masks[0]), _i32(lists[0])
+    out_m, out_l = torch.empty_like(q), torch.empty_like(q)
+    lse_m = torch.empty(B, H, q.shape[1], dtype=torch.float32, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):  # warm-up outside capture
+        vsa.fwd_bitmask(q, k, v, mask_buf, vbs, p.cfg.sm_scale, out=out_m, lse=lse_m)
+        vsa.fwd(q, k, v, idx_buf, vbs, p.cfg.sm_scale, out=out_l)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        vsa.fwd_bitmask(q, k, v, mask_buf, vbs, p.cfg.sm_scale, out=out_m, lse=lse_m)
+        vsa.fwd(q, k, v, idx_buf, vbs, p.cfg.sm_scale, out=out_l)
+    for x, m in zip(lists[1:], masks[1:]):
+        mask_buf.copy_(_mask_dev(m))
+        idx_buf.copy_(_i32(x))
+        graph.replay()
+        torch.cuda.synchronize()
+        want_m, want_lse = vsa.fwd_bitmask(q, k, v, _mask_dev(m), vbs, p.cfg.sm_scale, want_lse=True)
+        want_l = vsa.fwd(q, k, v, _i32(x), vbs, p.cfg.sm_scale)
+        torch.cuda.synchronize()
+        _no_device_error(vsa)
+        assert torch.equal(out_m.view(torch.int16), want_m.view(torch.int16))
+        assert torch.equal(lse_m.view(torch.int32), want_lse.view(torch.int32))
+        assert torch.equal(out_l.view(torch.int16), want_l.view(torch.int16))
+        assert torch.equal(out_m.view(torch.int16), out_l.view(torch.int16))
+    del graph

@@ -31,6 +31,7 @@ _STATUS = {0: "VSA_OK", -1: "VSA_ERR_ARG", -2: "VSA_ERR_NULL", -3: "VSA_ERR_ALIG
 
 # every symbol include/vsa.h declares
 EXPORTS = ("vsa_status_string", "vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_fwd_planned", "vsa_fwd_proxy",
+           "vsa_fwd_bsr", "vsa_fwd_bitmask",
            "vsa_plan_workspace_size", "vsa_plan", "vsa_route_workspace_size", "vsa_route", "vsa_route_means",
            "vsa_route_noalloc", "vsa_cube_counts", "vsa_tile", "vsa_tile_qkv", "vsa_untile", "vsa_stall_check",
            "vsa_device_status")
@@ -65,10 +66,13 @@ def _load():
     lib.vsa_untile.argtypes = [P, P, I, I, I, I, I, I, P]
     lib.vsa_tile_qkv.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, P]
     lib.vsa_fwd_proxy.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
+    lib.vsa_fwd_bsr.argtypes = [P, P, P, P, P, I, P, P, P, P, P, P, I, I, I, I, I, F, I, P]
+    lib.vsa_fwd_bitmask.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, I, P]
     lib.vsa_route_means.argtypes = [P, P, P, I, I, I, I, I, P]
     lib.vsa_device_status.argtypes = [P, P]
     lib.vsa_stall_check.argtypes = [P, P]
-    for name in ("vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_fwd_planned", "vsa_fwd_proxy", "vsa_plan", "vsa_route",
+    for name in ("vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_fwd_planned", "vsa_fwd_proxy", "vsa_fwd_bsr",
+                 "vsa_fwd_bitmask", "vsa_plan", "vsa_route",
                  "vsa_route_means", "vsa_route_noalloc", "vsa_cube_counts", "vsa_tile", "vsa_tile_qkv", "vsa_untile",
                  "vsa_device_status", "vsa_stall_check"):
         getattr(lib, name).restype = I
@@ -317,6 +321,66 @@ def fwd_proxy(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, topk_idx: torch
     _check(get_lib().vsa_fwd_proxy(_ptr(q), _ptr(k), _ptr(v), _ptr(topk_idx), _ptr(vbs), _ptr(kc), _ptr(vc),
                                    _ptr(plan), _ptr(out), _ptr(lse), B, S, H, D, nq, topk, float(sm_scale),
                                    int(flags), _stream(stream)), "vsa_fwd_proxy")
+    return (out, lse) if (want_lse or lse is not None) else out
+
+
+def _fwd_common(q, k, v, vbs, kc, vc, plan, sm_scale, out, lse, want_lse):
+    B, S, H, D = q.shape
+    nq = S // 64
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _bf16(t, n)
+    if (kc is None) != (vc is None):
+        raise ValueError("kc and vc go together")
+    if kc is not None:
+        for t, n in ((kc, "kc"), (vc, "vc")):
+            _bf16(t, n)
+        if kc.shape != (B, H, nq, D) or vc.shape != kc.shape:
+            raise ValueError("kc and vc must be [B, H, Nq, D]")
+    if vbs.dtype != torch.int32:
+        raise ValueError("vbs must be int32")
+    if plan is not None and (plan.dtype != torch.int32 or plan.numel() != B * H * ((nq + 1) // 2) * 2):
+        raise ValueError("plan must be int32 [B*H, ceil(Nq/2), 2]")
+    if sm_scale is None:
+        sm_scale = D ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, H, S, dtype=torch.float32, device=q.device)
+    return B, S, H, D, nq, float(sm_scale), out, lse
+
+
+def fwd_bsr(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_indptr: torch.Tensor,
+            block_indices: torch.Tensor, vbs: torch.Tensor, sm_scale: float | None = None, kc=None, vc=None,
+            out: torch.Tensor | None = None, lse: torch.Tensor | None = None, want_lse: bool = False,
+            flags: int = FWD_DEFAULT, plan: torch.Tensor | None = None, stream=None):
+    """vsa_fwd_bsr: the fine forward with the selections as BSR rows (block_indptr
+    [B*H*Nq + 1], block_indices [nnz], int32); kc, vc: optional proxies. Returns out
+    (and lse)."""
+    B, S, H, D, nq, sc, out, lse = _fwd_common(q, k, v, vbs, kc, vc, plan, sm_scale, out, lse, want_lse)
+    if block_indptr.dtype != torch.int32 or block_indices.dtype != torch.int32:
+        raise ValueError("block_indptr and block_indices must be int32")
+    if block_indptr.numel() != B * H * nq + 1:
+        raise ValueError("block_indptr must hold B*H*Nq + 1 entries")
+    nnz = block_indices.numel()
+    _check(get_lib().vsa_fwd_bsr(_ptr(q), _ptr(k), _ptr(v), _ptr(block_indptr), _ptr(block_indices) if nnz else None,
+                                 nnz, _ptr(vbs), _ptr(kc), _ptr(vc), _ptr(plan), _ptr(out), _ptr(lse), B, S, H, D,
+                                 nq, sc, int(flags), _stream(stream)), "vsa_fwd_bsr")
+    return (out, lse) if (want_lse or lse is not None) else out
+
+
+def fwd_bitmask(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask: torch.Tensor, vbs: torch.Tensor,
+                sm_scale: float | None = None, kc=None, vc=None, out: torch.Tensor | None = None,
+                lse: torch.Tensor | None = None, want_lse: bool = False, flags: int = FWD_DEFAULT,
+                plan: torch.Tensor | None = None, stream=None):
+    """vsa_fwd_bitmask: the fine forward with the selections as packed bitmaps
+    (mask [B, H, Nq, ceil(Nq/32)], 32-bit words, bit c % 32 of word c / 32 selects
+    cube c; int32 or uint32 storage); kc, vc: optional proxies. Returns out (and lse)."""
+    B, S, H, D, nq, sc, out, lse = _fwd_common(q, k, v, vbs, kc, vc, plan, sm_scale, out, lse, want_lse)
+    if mask.dtype not in (torch.int32, torch.uint32) or tuple(mask.shape) != (B, H, nq, (nq + 31) // 32):
+        raise ValueError("mask must be 32-bit [B, H, Nq, ceil(Nq/32)]")
+    _check(get_lib().vsa_fwd_bitmask(_ptr(q), _ptr(k), _ptr(v), _ptr(mask), _ptr(vbs), _ptr(kc), _ptr(vc),
+                                     _ptr(plan), _ptr(out), _ptr(lse), B, S, H, D, nq, sc, int(flags),
+                                     _stream(stream)), "vsa_fwd_bitmask")
     return (out, lse) if (want_lse or lse is not None) else out
 
 

@@ -78,10 +78,9 @@ int check_bshd(int B, int S, int H, int D, int Nq)
     return VSA_OK;
 }
 
-int fwd_dispatch(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const int32_t* topk_idx,
+int fwd_dispatch(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const vsa::Routes& rt,
                  const int32_t* vbs, const int32_t* plan, const vsa_bf16* kc, const vsa_bf16* vc, vsa_bf16* out,
-                 float* lse, int B, int S, int H, int D, int Nq, int topk, float sm_scale, int flags,
-                 cudaStream_t stream);
+                 float* lse, int B, int S, int H, int D, int Nq, float sm_scale, int flags, cudaStream_t stream);
 
 }  // namespace
 
@@ -108,28 +107,50 @@ int vsa_can_implement(int D, int sm_version) { return (D == 128 && sm_version ==
 
 namespace {
 
-// Shared by vsa_fwd_ex, vsa_fwd_planned and vsa_fwd_proxy: checks, then the kernel.
-int fwd_dispatch(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const int32_t* topk_idx,
+// Shared by every forward entry point: checks (sizes, then NULL pointers, then
+// alignment, then the device), then the kernel.  rt: the selections in one of
+// the three formats; kc and vc both NULL (plain) or both set (proxies).
+int fwd_dispatch(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const vsa::Routes& rt,
                  const int32_t* vbs, const int32_t* plan, const vsa_bf16* kc, const vsa_bf16* vc, vsa_bf16* out,
-                 float* lse, int B, int S, int H, int D, int Nq, int topk, float sm_scale, int flags,
-                 cudaStream_t stream)
+                 float* lse, int B, int S, int H, int D, int Nq, float sm_scale, int flags, cudaStream_t stream)
 {
     int rc = check_bshd(B, S, H, D, Nq);
     if (rc != VSA_OK) return rc;
-    if (topk < 1 || (flags & ~VSA_FWD_PRECISE_P) != 0) return VSA_ERR_ARG;
-    if (!vsa::fwd_pair_supported(Nq, topk)) return VSA_ERR_ARG;
-    if ((int64_t)B * H * Nq * topk > INT32_MAX) return VSA_ERR_ARG;
-    if (!q || !k || !v || !topk_idx || !vbs || !out) return VSA_ERR_NULL;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(topk_idx) ||
-        !aligned16(vbs) || (lse && !aligned16(lse)) || (plan && !aligned16(plan)) || (kc && !aligned16(kc)) ||
-        (vc && !aligned16(vc)))
+    const int64_t rows = (int64_t)B * H * Nq;
+    if (rt.kind == vsa::kRouteLists) {
+        if (rt.topk < 1 || (flags & ~VSA_FWD_PRECISE_P) != 0) return VSA_ERR_ARG;
+        if (!vsa::fwd_pair_supported(Nq, rt.topk)) return VSA_ERR_ARG;
+        if (rows * rt.topk > INT32_MAX) return VSA_ERR_ARG;
+    } else {
+        if ((flags & ~VSA_FWD_PRECISE_P) != 0 || !vsa::fwd_pair_supported(Nq, 1)) return VSA_ERR_ARG;
+        if (rt.kind == vsa::kRouteBsr && (rt.nnz < 0 || rows + 1 > INT32_MAX)) return VSA_ERR_ARG;
+        if (rt.kind == vsa::kRouteMask && rows * rt.words > INT32_MAX) return VSA_ERR_ARG;
+    }
+    const void* route_ptr = rt.kind == vsa::kRouteLists ? (const void*)rt.idx
+                            : rt.kind == vsa::kRouteBsr ? (const void*)rt.indptr
+                                                        : (const void*)rt.mask;
+    if (!q || !k || !v || !route_ptr || !vbs || !out) return VSA_ERR_NULL;
+    if (rt.kind == vsa::kRouteBsr && rt.nnz > 0 && !rt.idx) return VSA_ERR_NULL;
+    if ((kc == nullptr) != (vc == nullptr)) return VSA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(route_ptr) ||
+        (rt.kind == vsa::kRouteBsr && rt.idx && !aligned16(rt.idx)) || !aligned16(vbs) || (lse && !aligned16(lse)) ||
+        (plan && !aligned16(plan)) || (kc && !aligned16(kc)) || (vc && !aligned16(vc)))
         return VSA_ERR_ALIGN;
     if ((rc = check_arch()) != VSA_OK) return rc;
     int* err;
     if ((rc = device_error_word(&err)) != VSA_OK) return rc;
     const bool precise = (flags & VSA_FWD_PRECISE_P) != 0;
-    return launch_status(vsa::launch_fwd_pair(q, k, v, topk_idx, vbs, plan, kc, vc, out, lse, B, S, H, Nq, topk, sm_scale,
-                                              precise, err, stream));
+    return launch_status(
+        vsa::launch_fwd_pair(q, k, v, rt, vbs, plan, kc, vc, out, lse, B, S, H, Nq, sm_scale, precise, err, stream));
+}
+
+vsa::Routes route_lists(const int32_t* topk_idx, int topk)
+{
+    vsa::Routes rt{};
+    rt.idx = topk_idx;
+    rt.kind = vsa::kRouteLists;
+    rt.topk = topk;
+    return rt;
 }
 
 }  // namespace
@@ -156,8 +177,8 @@ int vsa_fwd_ex(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const in
                vsa_bf16* out, float* lse, int B, int S, int H, int D, int Nq, int topk, float sm_scale, int flags,
                cudaStream_t stream)
 {
-    return fwd_dispatch(q, k, v, topk_idx, vbs, nullptr, nullptr, nullptr, out, lse, B, S, H, D, Nq, topk, sm_scale,
-                        flags, stream);
+    return fwd_dispatch(q, k, v, route_lists(topk_idx, topk), vbs, nullptr, nullptr, nullptr, out, lse, B, S, H, D, Nq,
+                        sm_scale, flags, stream);
 }
 
 int vsa_fwd_planned(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const int32_t* topk_idx,
@@ -165,8 +186,8 @@ int vsa_fwd_planned(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, con
                     int Nq, int topk, float sm_scale, int flags, cudaStream_t stream)
 {
     if (!plan) return VSA_ERR_NULL;
-    return fwd_dispatch(q, k, v, topk_idx, vbs, plan, nullptr, nullptr, out, lse, B, S, H, D, Nq, topk, sm_scale,
-                        flags, stream);
+    return fwd_dispatch(q, k, v, route_lists(topk_idx, topk), vbs, plan, nullptr, nullptr, out, lse, B, S, H, D, Nq,
+                        sm_scale, flags, stream);
 }
 
 int vsa_fwd_proxy(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const int32_t* topk_idx,
@@ -175,8 +196,32 @@ int vsa_fwd_proxy(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const
                   cudaStream_t stream)
 {
     if (!kc || !vc) return VSA_ERR_NULL;
-    return fwd_dispatch(q, k, v, topk_idx, vbs, plan, kc, vc, out, lse, B, S, H, D, Nq, topk, sm_scale, flags,
-                        stream);
+    return fwd_dispatch(q, k, v, route_lists(topk_idx, topk), vbs, plan, kc, vc, out, lse, B, S, H, D, Nq, sm_scale,
+                        flags, stream);
+}
+
+int vsa_fwd_bsr(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const int32_t* block_indptr,
+                const int32_t* block_indices, int nnz, const int32_t* vbs, const vsa_bf16* kc, const vsa_bf16* vc,
+                const int32_t* plan, vsa_bf16* out, float* lse, int B, int S, int H, int D, int Nq, float sm_scale,
+                int flags, cudaStream_t stream)
+{
+    vsa::Routes rt{};
+    rt.idx = block_indices;
+    rt.indptr = block_indptr;
+    rt.kind = vsa::kRouteBsr;
+    rt.nnz = nnz;
+    return fwd_dispatch(q, k, v, rt, vbs, plan, kc, vc, out, lse, B, S, H, D, Nq, sm_scale, flags, stream);
+}
+
+int vsa_fwd_bitmask(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const uint32_t* mask,
+                    const int32_t* vbs, const vsa_bf16* kc, const vsa_bf16* vc, const int32_t* plan, vsa_bf16* out,
+                    float* lse, int B, int S, int H, int D, int Nq, float sm_scale, int flags, cudaStream_t stream)
+{
+    vsa::Routes rt{};
+    rt.mask = mask;
+    rt.kind = vsa::kRouteMask;
+    rt.words = Nq > 0 ? (Nq + 31) / 32 : 0;
+    return fwd_dispatch(q, k, v, rt, vbs, plan, kc, vc, out, lse, B, S, H, D, Nq, sm_scale, flags, stream);
 }
 
 int vsa_fwd(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const int32_t* topk_idx, const int32_t* vbs,

@@ -165,9 +165,9 @@ template <bool NEG, bool PRECISE, bool PROXY>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmkc,
-                    const __grid_constant__ CUtensorMap tmvc, const int32_t* __restrict__ topk_idx,
+                    const __grid_constant__ CUtensorMap tmvc, const Routes rt,
                     const int32_t* __restrict__ vbs, const int32_t* __restrict__ plan, uint16_t* __restrict__ out,
-                    float* __restrict__ lse, int S, int H, int nq, int topk, int tiles_per_bh, int n_tiles,
+                    float* __restrict__ lse, int S, int H, int nq, int tiles_per_bh, int n_tiles,
                     float scale_log2, int* err)
 {
     using L = Layout;
@@ -257,13 +257,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         TileRef t_next;
         if (my_tiles > 0) {
             t_next = checked_tile(blockIdx.x, H, nq, tiles_per_bh, plan, lane == 0 ? err : nullptr);
-            lists_fetch(t_next, topk_idx, H, nq, topk, m.list1[0], m.list2[0], lane);
+            lists_fetch(t_next, rt, H, nq, m.list1[0], m.list2[0], err, lane);
         }
         for (int n = 0; n < my_tiles && !aborted; ++n) {
             const TileRef t = t_next;
             int32_t* l1 = m.list1[n & 1];
             int32_t* l2 = m.list2[n & 1];
-            const int n_ent = steps_build(t, nq, topk, l1, l2, m.bits1, m.bits2, err, lane);
+            const int n_ent = rt.kind == kRouteMask ? steps_build_mask(t, nq, l1, l2, m.bits1, m.bits2, err, lane)
+                                                    : steps_build(t, nq, l1, l2, m.bits1, m.bits2, err, lane);
             const uint16_t* ent = reinterpret_cast<const uint16_t*>(l1);  // written over list 1
             const int tok0 = t.b * S;
             // proxy mode: after the selected cubes, ceil(nq / 128) steps over the proxy keys
@@ -326,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // into the other list buffer and its Q cubes prefetched into L2
                     t_next = checked_tile(blockIdx.x + (n + 1) * gridDim.x, H, nq, tiles_per_bh, plan,
                                           lane == 0 ? err : nullptr);
-                    lists_fetch(t_next, topk_idx, H, nq, topk, m.list1[(n + 1) & 1], m.list2[(n + 1) & 1], lane);
+                    lists_fetch(t_next, rt, H, nq, m.list1[(n + 1) & 1], m.list2[(n + 1) & 1], err, lane);
                     if (lane == 0) {
                         for (int q2 = 0; q2 < 2; ++q2) {
                             const int i = q2 == 0 ? t_next.i1 : t_next.i2;
@@ -870,8 +871,8 @@ struct FwdMaps {
 };
 
 template <bool NEG, bool PRECISE, bool PROXY>
-cudaError_t launch(const FwdMaps& mp, const int32_t* topk_idx, const int32_t* vbs, const int32_t* plan, uint16_t* out,
-                   float* lse, int B, int S, int H, int nq, int topk, float scale_log2, int* err, cudaStream_t s)
+cudaError_t launch(const FwdMaps& mp, const Routes& rt, const int32_t* vbs, const int32_t* plan, uint16_t* out,
+                   float* lse, int B, int S, int H, int nq, float scale_log2, int* err, cudaStream_t s)
 {
     auto kern = fwd_pair_kernel<NEG, PRECISE, PROXY>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Layout::SMEM_BYTES);
@@ -882,8 +883,8 @@ cudaError_t launch(const FwdMaps& mp, const int32_t* topk_idx, const int32_t* vb
     const int tiles_per_bh = (nq + 1) / 2;
     const int n_tiles = B * H * tiles_per_bh;
     const int grid = n_tiles < sms ? n_tiles : sms;
-    kern<<<grid, kThreads, Layout::SMEM_BYTES, s>>>(mp.q, mp.k, mp.v, mp.kc, mp.vc, topk_idx, vbs, plan, out,
-                                                    lse, S, H, nq, topk, tiles_per_bh, n_tiles, scale_log2, err);
+    kern<<<grid, kThreads, Layout::SMEM_BYTES, s>>>(mp.q, mp.k, mp.v, mp.kc, mp.vc, rt, vbs, plan, out, lse,
+                                                    S, H, nq, tiles_per_bh, n_tiles, scale_log2, err);
     return cudaGetLastError();
 }
 
@@ -891,10 +892,10 @@ cudaError_t launch(const FwdMaps& mp, const int32_t* topk_idx, const int32_t* vb
 
 bool fwd_pair_supported(int nq, int topk) { return nq <= kMaxNq && topk <= kMaxTopk; }
 
-cudaError_t launch_fwd_pair(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* topk_idx,
+cudaError_t launch_fwd_pair(const uint16_t* q, const uint16_t* k, const uint16_t* v, const Routes& rt,
                             const int32_t* vbs, const int32_t* plan, const uint16_t* kc, const uint16_t* vc,
-                            uint16_t* out, float* lse, int B, int S, int H, int nq, int topk, float sm_scale,
-                            bool precise_p, int* err, cudaStream_t s)
+                            uint16_t* out, float* lse, int B, int S, int H, int nq, float sm_scale, bool precise_p,
+                            int* err, cudaStream_t s)
 {
     FwdMaps mp;
     const int64_t tokens = (int64_t)B * S;
@@ -910,13 +911,13 @@ cudaError_t launch_fwd_pair(const uint16_t* q, const uint16_t* k, const uint16_t
     }
     const float scale_log2 = sm_scale * 1.4426950408889634f;
     // one kernel per (sign of the scale, weight precision, proxy steps)
-    using Launch = cudaError_t (*)(const FwdMaps&, const int32_t*, const int32_t*, const int32_t*, uint16_t*, float*,
-                                   int, int, int, int, int, float, int*, cudaStream_t);
+    using Launch = cudaError_t (*)(const FwdMaps&, const Routes&, const int32_t*, const int32_t*, uint16_t*, float*, int,
+                                   int, int, int, float, int*, cudaStream_t);
     static constexpr Launch table[8] = {
         launch<false, false, false>, launch<true, false, false>, launch<false, true, false>, launch<true, true, false>,
         launch<false, false, true>,  launch<true, false, true>,  launch<false, true, true>,  launch<true, true, true>};
     const int which = (scale_log2 < 0.f ? 1 : 0) | (precise_p ? 2 : 0) | (proxy ? 4 : 0);
-    return table[which](mp, topk_idx, vbs, plan, out, lse, B, S, H, nq, topk, scale_log2, err, s);
+    return table[which](mp, rt, vbs, plan, out, lse, B, S, H, nq, scale_log2, err, s);
 }
 
 }  // namespace vsa

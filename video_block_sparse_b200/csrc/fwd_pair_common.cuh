@@ -318,11 +318,13 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, ui
 // The CTA's tiles are t = blockIdx.x + n * gridDim.x; tile n goes to slot n & 1.
 struct TileRef {
     int b, h, i1, i2;  // i2 = -1: a single query cube (rows 64-127 unused)
+    int len1, len2;    // the rows' lengths as copied in (entries, or words of a bitmap row)
 };
 
 __device__ __forceinline__ TileRef tile_ref(int t, int H, int nq, int tiles_per_bh, const int32_t* plan)
 {
     TileRef r;
+    r.len1 = r.len2 = 0;
     const int bh = t / tiles_per_bh, p = t - bh * tiles_per_bh;
     r.b = bh / H;
     r.h = bh - r.b * H;
@@ -360,18 +362,41 @@ __device__ __forceinline__ void vbs_stage(const int32_t* __restrict__ vbs, int n
     }
 }
 
-// Copy a tile's two selection lists into shared memory asynchronously
-// (cp.async, one entry per lane and pass); steps_build waits for them.  Run one
-// tile ahead, so that the copies overlap the previous tile's steps.
-__device__ __forceinline__ void lists_fetch(const TileRef& t, const int32_t* __restrict__ topk_idx, int H, int nq,
-                                            int topk, int32_t* l1, int32_t* l2, uint32_t lane)
+// Copy a tile's two rows of the selection into shared memory asynchronously
+// (cp.async, one 4-byte word per lane and pass) and set their lengths in t
+// (entries, or words of a bitmap row); the build waits for them.  Run one tile
+// ahead, so that the copies overlap the previous tile's steps.  A BSR row that
+// does not lie within the index array latches an error and is taken as empty;
+// one longer than kMaxTopk latches an error and is cut to its first kMaxTopk.
+__device__ __forceinline__ void lists_fetch(TileRef& t, const Routes& rt, int H, int nq, int32_t* l1, int32_t* l2,
+                                            int* err, uint32_t lane)
 {
     for (int s = 0; s < 2; ++s) {
         const int i = s == 0 ? t.i1 : t.i2;
-        if (i < 0) continue;
-        const int32_t* src = topk_idx + (((int64_t)t.b * H + t.h) * nq + i) * topk;
-        int32_t* dst = s == 0 ? l1 : l2;
-        for (int e = lane; e < topk; e += 32) cp_async4(dst + e, src + e);
+        int len = 0;
+        if (i >= 0) {
+            const int64_t r = ((int64_t)t.b * H + t.h) * nq + i;
+            const int32_t* src;
+            if (rt.kind == kRouteBsr) {
+                const int a = __ldg(rt.indptr + r), e = __ldg(rt.indptr + r + 1);
+                const bool inside = a >= 0 && e >= a && e <= rt.nnz;
+                len = inside ? min(e - a, kMaxTopk) : 0;
+                if ((!inside || e - a > kMaxTopk) && lane == 0) atomicCAS(err, 0, (int)kErrRoute);
+                src = rt.idx + (inside ? a : 0);
+            } else if (rt.kind == kRouteMask) {
+                len = rt.words;
+                src = reinterpret_cast<const int32_t*>(rt.mask + r * rt.words);
+            } else {
+                len = rt.topk;
+                src = rt.idx + r * rt.topk;
+            }
+            int32_t* dst = s == 0 ? l1 : l2;
+            for (int e = lane; e < len; e += 32) cp_async4(dst + e, src + e);
+        }
+        if (s == 0)
+            t.len1 = len;
+        else
+            t.len2 = len;
     }
     cp_async_commit();
 }
@@ -387,7 +412,7 @@ __device__ __forceinline__ void lists_fetch(const TileRef& t, const int32_t* __r
 // are dropped.  Returns the number of entries (warp-uniform).
 constexpr int kBuildBatch = 4;
 
-__device__ int steps_build(const TileRef& t, int nq, int topk, int32_t* l1, int32_t* l2, uint32_t* b1, uint32_t* b2,
+__device__ int steps_build(const TileRef& t, int nq, int32_t* l1, int32_t* l2, uint32_t* b1, uint32_t* b2,
                            int* err, uint32_t lane)
 {
     const int words = (nq + 31) >> 5;
@@ -395,15 +420,14 @@ __device__ int steps_build(const TileRef& t, int nq, int topk, int32_t* l1, int3
         b1[w] = 0u;
         b2[w] = 0u;
     }
-    const int len1 = t.i1 >= 0 ? topk : 0;
-    const int len2 = t.i2 >= 0 ? topk : 0;
+    const int len1 = t.len1, len2 = t.len2;
     cp_async_wait_all();
     __syncwarp();
     // bitmaps by shared-memory ORs; a list names a cube twice iff one of its ORs
     // finds the bit already set
     bool dup = false;
     int j0[2][kBuildBatch];  // the first batch (-1: none or invalid)
-    for (int base = 0; base < topk; base += 32 * kBuildBatch) {
+    for (int base = 0; base < max(len1, len2); base += 32 * kBuildBatch) {
         int j[2][kBuildBatch];
 #pragma unroll
         for (int s = 0; s < 2; ++s)
@@ -467,6 +491,84 @@ __device__ int steps_build(const TileRef& t, int nq, int topk, int32_t* l1, int3
                 if (q[u]) ent[count + __popc(mask & lt)] = (uint16_t)code[u];
                 count += __popc(mask);
             }
+        }
+    }
+    __syncwarp();
+    return count;
+}
+
+// Inclusive prefix sum of x over the warp's lanes.
+__device__ __forceinline__ int warp_incl_sum(int x, uint32_t lane)
+{
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if ((int)lane >= o) x += y;
+    }
+    return x;
+}
+
+// The same for bitmap rows (copied in by lists_fetch): the rows become the
+// membership bitmaps (bits at cubes >= nq cleared; a row of more than
+// kMaxTopk cubes latches an error and keeps its first kMaxTopk), then the
+// entries are written over list 1 in the order of steps_build with each
+// list in ascending cube order: row 1's cubes (membership 3 where row 2 has
+// the cube too), then row 2's others.
+__device__ int steps_build_mask(const TileRef& t, int nq, int32_t* l1, int32_t* l2, uint32_t* b1, uint32_t* b2,
+                                int* err, uint32_t lane)
+{
+    const int words = (nq + 31) >> 5;
+    const uint32_t last = (nq & 31) ? (1u << (nq & 31)) - 1u : 0xffffffffu;
+    cp_async_wait_all();
+    __syncwarp();
+    for (int s = 0; s < 2; ++s) {
+        const int len = s == 0 ? t.len1 : t.len2;
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(s == 0 ? l1 : l2);
+        uint32_t* dst = s == 0 ? b1 : b2;
+        int seen = 0;  // cubes in the words before this pass's
+        for (int base = 0; base < words; base += 32) {
+            const int w = base + (int)lane;
+            uint32_t m = w < len ? src[w] : 0u;
+            if (w == words - 1) m &= last;
+            const int c = __popc(m);
+            const int incl = warp_incl_sum(c, lane);
+            const int before = seen + incl - c;
+            if (before + c > kMaxTopk) {
+                atomicCAS(err, 0, (int)kErrRoute);
+                uint32_t keep = 0u;  // the lowest kMaxTopk - before of its cubes
+                for (int n = max(0, kMaxTopk - before); n > 0 && m != 0u; --n) {
+                    const uint32_t lo = m & (0u - m);
+                    keep |= lo;
+                    m ^= lo;
+                }
+                m = keep;
+            }
+            seen += __shfl_sync(0xffffffffu, incl, 31);
+            if (w < words) dst[w] = m;
+        }
+    }
+    __syncwarp();
+    uint16_t* ent = reinterpret_cast<uint16_t*>(l1);  // the row of list 1 is in b1 now
+    int count = 0;
+    for (int s = 0; s < 2; ++s) {
+        for (int base = 0; base < words; base += 32) {
+            const int w = base + (int)lane;
+            uint32_t m = 0u, both = 0u;
+            if (w < words) {
+                const uint32_t x1 = b1[w], x2 = b2[w];
+                m = s == 0 ? x1 : (x2 & ~x1);
+                both = s == 0 ? (x1 & x2) : 0u;
+            }
+            const int c = __popc(m);
+            const int incl = warp_incl_sum(c, lane);
+            int pos = count + incl - c;
+            while (m != 0u) {
+                const int bit = __ffs((int)m) - 1;
+                const uint32_t mem = s == 1 ? 2u : (((both >> bit) & 1u) ? 3u : 1u);
+                ent[pos++] = (uint16_t)((uint32_t)(32 * w + bit) | (mem << 14));
+                m &= m - 1u;
+            }
+            count += __shfl_sync(0xffffffffu, incl, 31);
         }
     }
     __syncwarp();

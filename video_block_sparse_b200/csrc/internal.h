@@ -16,6 +16,7 @@ enum DeviceError : int {
     kErrVbs = 2,
     kErrWaitTimeout = 3,
     kErrPlan = 4,
+    kErrRoute = 5,  // a BSR row outside the index array or longer than 1024, or a bitmap row of more than 1024 cubes
 };
 
 struct CubeGeom {
@@ -53,11 +54,27 @@ cudaError_t launch_score_topk(const uint16_t* qc, const uint16_t* kc, int32_t* t
 
 // ---- fwd_pair.cu (tcgen05 kernel, two query cubes per 128-row tile)
 bool fwd_pair_supported(int nq, int topk);
+
+// The forward's selections, row r = (b*H + h)*Nq + i for query cube i: fixed-length
+// lists (topk_idx [B, H, Nq, topk]), BSR rows (indices[indptr[r] .. indptr[r+1]), nnz
+// entries in all), or packed UInt32 bitmaps ([B, H, Nq, words], bit c % 32 of word c / 32
+// selects cube c).
+enum RouteKind : int { kRouteLists = 0, kRouteBsr = 1, kRouteMask = 2 };
+struct Routes {
+    const int32_t* idx;     // lists: topk_idx; BSR: indices
+    const int32_t* indptr;  // BSR: [B*H*Nq + 1]
+    const uint32_t* mask;   // bitmaps
+    int kind;
+    int topk;   // lists: row length
+    int nnz;    // BSR: entries of indices
+    int words;  // bitmaps: words per row, ceil(Nq / 32)
+};
+
 // kc, vc: the proxies' mean keys and summed values [B, H, Nq, 128] (both NULL: no proxies)
-cudaError_t launch_fwd_pair(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* topk_idx,
+cudaError_t launch_fwd_pair(const uint16_t* q, const uint16_t* k, const uint16_t* v, const Routes& rt,
                             const int32_t* vbs, const int32_t* plan, const uint16_t* kc, const uint16_t* vc,
-                            uint16_t* out, float* lse, int B, int S, int H, int nq, int topk, float sm_scale,
-                            bool precise_p, int* err, cudaStream_t s);
+                            uint16_t* out, float* lse, int B, int S, int H, int nq, float sm_scale, bool precise_p,
+                            int* err, cudaStream_t s);
 
 // ---- plan.cu (pairing of query cubes by selection overlap)
 size_t plan_workspace_bytes(int B, int H, int nq);
