@@ -377,7 +377,28 @@ def run_extras(vsa, dev, cfg, qt, kt, vt, qc, kc, idx, vbs, peak):
                         fn=vsa.fwd_proxy)
     res["proxy"] = {"fwd_ms": ms_plain, "fwd_proxy_ms": ms_proxy, "overhead": ms_proxy / ms_plain - 1.0,
                     "proxy_steps_per_tile": (len(vbs_h) + 127) // 128}
-    del vc
+
+    # route formats: the routed lists in ascending order as topk rows, BSR rows and
+    # packed bitmaps (the same step lists), and the bitmaps with proxies
+    ix_sorted = torch.sort(idx, dim=-1).values.contiguous()
+    B, H, nq, topk = ix_sorted.shape
+    indptr = (torch.arange(B * H * nq + 1, device=dev, dtype=torch.int32) * topk).contiguous()
+    indices = ix_sorted.reshape(-1).contiguous()
+    W = (nq + 31) // 32
+    bits = torch.zeros(B, H, nq, W, dtype=torch.int64, device=dev)
+    bits.scatter_add_(3, (ix_sorted // 32).long(), torch.ones_like(ix_sorted, dtype=torch.int64) << (ix_sorted % 32).long())
+    mask = torch.where(bits >= 2 ** 31, bits - 2 ** 32, bits).to(torch.int32).contiguous()
+    pl_s = vsa.plan(ix_sorted)
+    fmt = {"fwd_lists_ms": fwd_case(qt, kt, vt, ix_sorted, vbs, cfg, pl_s)}
+    fmt["fwd_bsr_ms"] = time_fwd(vsa, ((qt, kt, vt, indptr, indices, vbs, cfg.sm_scale), {"out": out, "plan": pl_s}),
+                                 fn=vsa.fwd_bsr)
+    fmt["fwd_bitmask_ms"] = time_fwd(vsa, ((qt, kt, vt, mask, vbs, cfg.sm_scale), {"out": out, "plan": pl_s}),
+                                     fn=vsa.fwd_bitmask)
+    fmt["fwd_bitmask_proxy_ms"] = time_fwd(
+        vsa, ((qt, kt, vt, mask, vbs, cfg.sm_scale), {"out": out, "plan": pl_s, "kc": kc, "vc": vc}),
+        fn=vsa.fwd_bitmask)
+    res["route_formats"] = fmt
+    del vc, mask, bits, indices
 
     # other configurations: forward alone (inputs tiled and routed by the library first)
     cfgs = {}
