@@ -600,6 +600,63 @@ int oracle_fwd_bsr_items(const uint16_t *q, const uint16_t *k, const uint16_t *v
     return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
 }
 
+/* ------------------------------------------------------------------ short-KV cross-attention
+ *
+ * maxdiffusion PR #509 (a fused short-KV cross-attention kernel for Wan's 512-token
+ * text KV): every query row attends to every key of a separate, short key/value
+ * sequence with one exact softmax (no mask).  q: [B, S, H, D], k and v: [B, S_kv,
+ * H, D]; items (b, h, i) are query blocks of 64 rows (S = 64 * number of blocks):
+ *   out[b, s, h] = sum_u e^{x_u} v_u / sum_u e^{x_u},  x_u = sigma q_s . k_u
+ *   lse          = log sum_u e^{x_u}  (u over all S_kv keys). */
+int oracle_cross_items(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B, int S, int S_kv, int H,
+                       int D, double sigma, const int32_t *items, int64_t n_items, double *out, double *lse)
+{
+    if (B <= 0 || H <= 0 || D <= 0 || S <= 0 || S % 64 != 0 || S_kv <= 0) return ORACLE_ERR_ARG;
+    for (int64_t it = 0; it < n_items; ++it) {
+        int b = items[3 * it], h = items[3 * it + 1], i = items[3 * it + 2];
+        if (b < 0 || b >= B || h < 0 || h >= H || i < 0 || i >= S / 64) return ORACLE_ERR_ARG;
+    }
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *x = (double *)malloc((size_t)S_kv * sizeof(double));
+        if (!x) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t it = 0; it < n_items; ++it) {
+            if (!x) continue;
+            int b = items[3 * it], h = items[3 * it + 1], i = items[3 * it + 2];
+            for (int r = 0; r < 64; ++r) {
+                int64_t s = 64LL * i + r;
+                const uint16_t *qs = q + (((int64_t)b * S + s) * H + h) * D;
+                double *o = out + (it * 64 + r) * D;
+                double m = -INFINITY;
+                for (int u = 0; u < S_kv; ++u) {
+                    const uint16_t *ku = k + (((int64_t)b * S_kv + u) * H + h) * D;
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) dot += bf16_bits_to_f64(qs[d]) * bf16_bits_to_f64(ku[d]);
+                    x[u] = sigma * dot;
+                    if (x[u] > m) m = x[u];
+                }
+                double l = 0.0;
+                for (int d = 0; d < D; ++d) o[d] = 0.0;
+                for (int u = 0; u < S_kv; ++u) {
+                    double p = exp(x[u] - m);
+                    const uint16_t *vu = v + (((int64_t)b * S_kv + u) * H + h) * D;
+                    l += p;
+                    for (int d = 0; d < D; ++d) o[d] += p * bf16_bits_to_f64(vu[d]);
+                }
+                for (int d = 0; d < D; ++d) o[d] /= l;
+                lse[it * 64 + r] = m + log(l);
+            }
+        }
+        free(x);
+    }
+    return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}
+
 int oracle_fwd_items(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                      const int32_t *topk_idx, const int32_t *vbs,
                      int B, int S, int H, int D, int Nq, int topk, double sigma,

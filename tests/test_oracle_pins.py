@@ -739,3 +739,52 @@ def test_route_formats_describe_the_same_selection(oracle_lib):
     o1, l1 = oracle_lib.fwd_items(q, k, v, idx, vbs, 0.1, items)
     o2, l2 = oracle_lib.fwd_bsr_items(q, k, v, indptr, indices, vbs, 0.1, items)
     assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+# ------------------------------------------------------------------ short-KV cross-attention
+# maxdiffusion PR #509: every query row over every key of a short text key/value sequence,
+# one exact softmax, no mask.
+
+def _cross_case(seed, nblk=3, S_kv=77, H=2, scale=1.5):
+    g = np.random.default_rng(seed)
+    q = synth.f32_to_bf16_bits((g.standard_normal((1, 64 * nblk, H, 128)) * scale).astype(np.float32))
+    k = synth.f32_to_bf16_bits((g.standard_normal((1, S_kv, H, 128)) * scale).astype(np.float32))
+    v = synth.f32_to_bf16_bits(g.standard_normal((1, S_kv, H, 128)).astype(np.float32))
+    return q, k, v
+
+
+def test_cross_over_its_own_sequence_is_the_dense_fine_forward(oracle_lib):
+    """K/V the query sequence itself (S_kv = S) and every cube listed with 64 valid
+    tokens: the fine-stage forward, already pinned to dense attention."""
+    q, k, v = _cross_case(50, nblk=4, S_kv=256)
+    items = oracle_lib.all_items(1, 2, 4)
+    o1, l1 = oracle_lib.cross_items(q, k, v, 0.125, items)
+    dense = np.broadcast_to(np.arange(4, dtype=np.int32), (1, 2, 4, 4)).copy()
+    o2, l2 = oracle_lib.fwd_items(q, k, v, dense, np.full(4, 64, np.int32), 0.125, items)
+    assert np.allclose(o1, o2, rtol=0, atol=1e-13) and np.allclose(l1, l2, rtol=0, atol=1e-13)
+
+
+def test_cross_closed_forms(oracle_lib):
+    """q = 0: the mean of v and lse = log S_kv; one key: its value and its logit."""
+    q, k, v = _cross_case(51, S_kv=77)
+    items = oracle_lib.all_items(1, 2, 3)
+    out, lse = oracle_lib.cross_items(np.zeros_like(q), k, v, 0.3, items)
+    V = oracle_lib.bf16_to_f64(v)[0]
+    for n, (b, h, i) in enumerate(items):
+        assert np.allclose(out[n], np.broadcast_to(V[:, h].mean(axis=0), (64, 128)), rtol=0, atol=1e-13)
+        assert np.allclose(lse[n], math.log(77), rtol=0, atol=1e-13)
+    q, k, v = _cross_case(52, S_kv=1)
+    out, lse = oracle_lib.cross_items(q, k, v, 0.25, items)
+    Q, K, V = (oracle_lib.bf16_to_f64(a)[0] for a in (q, k, v))
+    for n, (b, h, i) in enumerate(items):
+        assert np.array_equal(out[n], np.broadcast_to(V[0, h], (64, 128)))
+        assert np.allclose(lse[n], 0.25 * (Q[64 * i: 64 * i + 64, h] @ K[0, h]), rtol=0, atol=1e-12)
+
+
+def test_cross_ignores_the_order_of_keys(oracle_lib):
+    q, k, v = _cross_case(53, S_kv=130)
+    perm = np.random.default_rng(54).permutation(130)
+    items = oracle_lib.all_items(1, 2, 3)
+    o1, l1 = oracle_lib.cross_items(q, k, v, 0.2, items)
+    o2, l2 = oracle_lib.cross_items(q, k[:, perm], v[:, perm], 0.2, items)
+    assert np.allclose(o1, o2, rtol=0, atol=1e-13) and np.allclose(l1, l2, rtol=0, atol=1e-13)
