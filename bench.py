@@ -400,6 +400,18 @@ def run_extras(vsa, dev, cfg, qt, kt, vt, qc, kc, idx, vbs, peak):
     res["route_formats"] = fmt
     del vc, mask, bits, indices
 
+    # short-KV cross-attention: the step's queries over a 512-token text key/value
+    # sequence (seeded draws), every key attended
+    S_kv = 512
+    g = torch.Generator(device="cpu").manual_seed(512)
+    kt_txt = torch.randn(cfg.B, S_kv, cfg.H, 128, generator=g).to(torch.bfloat16).to(dev)
+    vt_txt = torch.randn(cfg.B, S_kv, cfg.H, 128, generator=g).to(torch.bfloat16).to(dev)
+    ms_x = time_fwd(vsa, ((qt, kt_txt, vt_txt, cfg.sm_scale), {"out": out}), fn=vsa.cross_attn)
+    fl_x = 4.0 * cfg.B * qt.shape[1] * S_kv * 128 * cfg.H
+    res["cross_attn"] = {"S_q": qt.shape[1], "S_kv": S_kv, "tflop_per_call": fl_x / 1e12, "ms": ms_x,
+                         "tflops": fl_x / (ms_x * 1e-3) / 1e12, "frac": fl_x / (ms_x * 1e-3) / 1e12 / peak}
+    del kt_txt, vt_txt
+
     # other configurations: forward alone (inputs tiled and routed by the library first)
     cfgs = {}
     for name in ("sweep32", "sweep156", "sweep312", "dense624", "wan720"):

@@ -217,6 +217,24 @@ VSA_API int vsa_fwd_bsr(const vsa_bf16 *q, const vsa_bf16 *k, const vsa_bf16 *v,
                         const int32_t *block_indices, int nnz, const int32_t *vbs, const vsa_bf16 *kc,
                         const vsa_bf16 *vc, const int32_t *plan, vsa_bf16 *out, float *lse, int B, int S, int H,
                         int D, int Nq, float sm_scale, int flags, cudaStream_t stream);
+/* ------------------------------------------------------------------------
+ * vsa_cross_attn -- short-KV cross-attention (maxdiffusion PR #509: Wan's
+ * cross-attention over the 512-token text KV, one exact softmax per query row
+ * over every key, no mask):
+ *   out[b, s, h, :] = softmax_u(sm_scale q[b, s, h, :] . k[b, u, h, :]) v[b, u, h, :]
+ * over all u < S_kv.  The same tcgen05 kernel as the fine stage: query rows in
+ * blocks of 64, two blocks to a 128-row tile, the keys in 64-key cubes (the
+ * last holding the S_kv % 64 left, if any); the softmax is online over the
+ * ceil(S_kv / 64) cubes, which is the exact softmax up to rounding.
+ *   q, out  [B, S, H, D] bf16 (any row order, S a multiple of 64, S <= 64 * 8192)
+ *   k, v    [B, S_kv, H, D] bf16, 1 <= S_kv <= 65536
+ *   lse     [B, H, S] fp32 natural log-sum-exp, or NULL
+ * flags: VSA_FWD_PRECISE_P as for vsa_fwd_ex.  Errors: VSA_ERR_ARG for sizes
+ * out of range or D != 128, VSA_ERR_NULL, VSA_ERR_ALIGN (16 bytes),
+ * VSA_ERR_ARCH, VSA_ERR_LAUNCH.
+ * ---------------------------------------------------------------------- */
+VSA_API int vsa_cross_attn(const vsa_bf16 *q, const vsa_bf16 *k, const vsa_bf16 *v, vsa_bf16 *out, float *lse,
+                           int B, int S, int S_kv, int H, int D, float sm_scale, int flags, cudaStream_t stream);
 VSA_API int vsa_fwd_bitmask(const vsa_bf16 *q, const vsa_bf16 *k, const vsa_bf16 *v, const uint32_t *mask,
                             const int32_t *vbs, const vsa_bf16 *kc, const vsa_bf16 *vc, const int32_t *plan,
                             vsa_bf16 *out, float *lse, int B, int S, int H, int D, int Nq, float sm_scale, int flags,

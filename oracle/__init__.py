@@ -62,7 +62,7 @@ def _load():
         lib.oracle_fwd_proxy_items.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, ctypes.c_double, P, I64, P, P]
         lib.oracle_fwd_bsr_items.argtypes = [P, P, P, P, P, P, P, I64, P, I, I, I, I, I, ctypes.c_double, P, I64, P, P,
                                              P]
-        lib.oracle_cross_items.argtypes = [P, P, P, I, I, I, I, I, ctypes.c_double, P, I64, P, P]
+        lib.oracle_cross_items.argtypes = [P, P, P, I, I, I, I, I, ctypes.c_double, P, I64, P, P, P]
         for name in ("oracle_f64_to_bf16", "oracle_bf16_to_f64", "oracle_cube_counts", "oracle_tile",
                      "oracle_untile", "oracle_cube_means", "oracle_route", "oracle_fwd_items", "oracle_fwd_items_ex",
                      "oracle_num_threads", "oracle_plan", "oracle_cube_sums", "oracle_fwd_proxy_items",
@@ -255,11 +255,11 @@ def fwd_bsr_items(q, k, v, indptr, indices, vbs, sm_scale: float, items: np.ndar
     return (out, lse, wabs) if want_wabs else (out, lse)
 
 
-def cross_items(q, k, v, sm_scale: float, items: np.ndarray):
+def cross_items(q, k, v, sm_scale: float, items: np.ndarray, want_wabs: bool = False):
     """Short-KV cross-attention (every query row over every key of k, v [B, S_kv, H, D],
     one exact softmax) for the listed (b, h, query block of 64 rows) items of q [B, S, H, D].
-    Returns out [n, 64, D] and lse [n, 64], float64; sm_scale is used as the binary32 value
-    a GPU kernel receives."""
+    Returns out [n, 64, D] and lse [n, 64] (and the weighted mean of |v| [n, 64, D]),
+    float64; sm_scale is used as the binary32 value a GPU kernel receives."""
     B, S, H, D = q.shape
     S_kv = k.shape[1]
     assert k.shape == (B, S_kv, H, D) and v.shape == k.shape and S % 64 == 0
@@ -268,9 +268,11 @@ def cross_items(q, k, v, sm_scale: float, items: np.ndarray):
     n = items.shape[0]
     out = np.empty((n, 64, D), dtype=np.float64)
     lse = np.empty((n, 64), dtype=np.float64)
+    wabs = np.empty((n, 64, D), dtype=np.float64) if want_wabs else None
     _check(_load().oracle_cross_items(*(_ptr(a) for a in arrs), B, S, S_kv, H, D, float(np.float32(sm_scale)),
-                                      _ptr(items), n, _ptr(out), _ptr(lse)), "cross_items")
-    return out, lse
+                                      _ptr(items), n, _ptr(out), _ptr(lse), None if wabs is None else _ptr(wabs)),
+           "cross_items")
+    return (out, lse, wabs) if want_wabs else (out, lse)
 
 
 def fwd_items(q, k, v, topk_idx, vbs, sm_scale: float, items: np.ndarray, want_wabs: bool = False):

@@ -607,9 +607,11 @@ int oracle_fwd_bsr_items(const uint16_t *q, const uint16_t *k, const uint16_t *v
  * sequence with one exact softmax (no mask).  q: [B, S, H, D], k and v: [B, S_kv,
  * H, D]; items (b, h, i) are query blocks of 64 rows (S = 64 * number of blocks):
  *   out[b, s, h] = sum_u e^{x_u} v_u / sum_u e^{x_u},  x_u = sigma q_s . k_u
- *   lse          = log sum_u e^{x_u}  (u over all S_kv keys). */
+ *   lse          = log sum_u e^{x_u}  (u over all S_kv keys).
+ * wabs (may be NULL): the softmax-weighted mean of |v|. */
 int oracle_cross_items(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B, int S, int S_kv, int H,
-                       int D, double sigma, const int32_t *items, int64_t n_items, double *out, double *lse)
+                       int D, double sigma, const int32_t *items, int64_t n_items, double *out, double *lse,
+                       double *wabs)
 {
     if (B <= 0 || H <= 0 || D <= 0 || S <= 0 || S % 64 != 0 || S_kv <= 0) return ORACLE_ERR_ARG;
     for (int64_t it = 0; it < n_items; ++it) {
@@ -650,6 +652,15 @@ int oracle_cross_items(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
                 }
                 for (int d = 0; d < D; ++d) o[d] /= l;
                 lse[it * 64 + r] = m + log(l);
+                if (wabs != NULL) {
+                    double *a = wabs + (it * 64 + r) * D;
+                    for (int d = 0; d < D; ++d) a[d] = 0.0;
+                    for (int u = 0; u < S_kv; ++u) {
+                        double w = exp(x[u] - m) / l;
+                        const uint16_t *vu = v + (((int64_t)b * S_kv + u) * H + h) * D;
+                        for (int d = 0; d < D; ++d) a[d] += w * fabs(bf16_bits_to_f64(vu[d]));
+                    }
+                }
             }
         }
         free(x);

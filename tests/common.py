@@ -157,13 +157,21 @@ def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
     return 2.0 ** (np.floor(np.log2(a)) - 8)
 
 
-def within_default_bound(gpu_rows: np.ndarray, o64: np.ndarray, wabs: np.ndarray) -> dict:
+# The precise mode's weights are hi + lo, within u = 2^-17 of P: by the same argument
+# as above, 2 u / (1 - u) < 2^-15.
+PRECISE_WEIGHT_BOUND = 2.0 ** -15
+
+
+def within_default_bound(gpu_rows: np.ndarray, o64: np.ndarray, wabs: np.ndarray, coeff: float | None = None
+                         ) -> dict:
     """The default mode's stated per-element error bound (not the card's rule):
     |gpu - exact| <= half a bf16 ulp + 2^-7 * sum_u w_u |v_u| (+ 2^-20 |exact|
-    for the fp32 accumulation)."""
+    for the fp32 accumulation).  coeff replaces the 2^-7 (another mode's weight
+    bound, plus any accumulation term a caller states in units of sum w |v|)."""
+    coeff = DEFAULT_WEIGHT_BOUND if coeff is None else coeff
     g = gpu_rows.astype(np.float64)
     err = np.abs(g - o64)
-    lim = bf16_half_ulp(np.maximum(np.abs(g), np.abs(o64))) + DEFAULT_WEIGHT_BOUND * wabs + 2.0 ** -20 * np.abs(o64)
+    lim = bf16_half_ulp(np.maximum(np.abs(g), np.abs(o64))) + coeff * wabs + 2.0 ** -20 * np.abs(o64)
     worst = float(np.max(err - lim))
     return {"ok": bool(np.isfinite(g).all() and worst <= 0), "worst_excess": worst,
             "max_err": float(err.max())}

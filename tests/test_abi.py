@@ -171,6 +171,19 @@ def test_fwd_bsr_and_bitmask_reject_bad_arguments_without_a_device(vsa):
     assert lib.vsa_fwd_bitmask(p, p, p, _fake((1 << 20) + 8), p, None, None, None, p, None, *tail) == -3
 
 
+def test_cross_attn_rejects_bad_arguments_without_a_device(vsa):
+    p = _fake(1 << 20)
+    lib = vsa.get_lib()
+    # vsa_cross_attn(q, k, v, out, lse, B, S, S_kv, H, D, scale, flags, stream)
+    assert lib.vsa_cross_attn(p, p, p, p, None, 1, 500, 512, 2, 128, 0.1, 0, None) == -1  # S % 64
+    assert lib.vsa_cross_attn(p, p, p, p, None, 1, 512, 0, 2, 128, 0.1, 0, None) == -1  # S_kv
+    assert lib.vsa_cross_attn(p, p, p, p, None, 1, 512, 70000, 2, 128, 0.1, 0, None) == -1
+    assert lib.vsa_cross_attn(p, p, p, p, None, 1, 512, 512, 2, 64, 0.1, 0, None) == -1  # D
+    assert lib.vsa_cross_attn(p, p, p, p, None, 1, 512, 512, 2, 128, 0.1, 4, None) == -1  # flag
+    assert lib.vsa_cross_attn(p, None, p, p, None, 1, 512, 512, 2, 128, 0.1, 0, None) == -2
+    assert lib.vsa_cross_attn(p, p, p, _fake((1 << 20) + 4), None, 1, 512, 512, 2, 128, 0.1, 0, None) == -3
+
+
 def test_route_noalloc_checks_arguments_before_its_array_limit(vsa):
     """Bad arguments are reported as by vsa_route, even for a problem larger than
     the fixed array, and before any device is touched."""

@@ -766,3 +766,93 @@ def test_fwd_routes_live_under_cuda_graph_replay(vsa):
         assert torch.equal(out_l.view(torch.int16), want_l.view(torch.int16))
         assert torch.equal(out_m.view(torch.int16), out_l.view(torch.int16))
     del graph
+
+
+# ------------------------------------------------------------------ short-KV cross-attention
+
+def _cross_inputs(seed, B, nblk, S_kv, H, scale=1.0):
+    g = np.random.default_rng(seed)
+    q = synth.f32_to_bf16_bits((g.standard_normal((B, 64 * nblk, H, 128)) * scale).astype(np.float32))
+    k = synth.f32_to_bf16_bits((g.standard_normal((B, S_kv, H, 128)) * scale).astype(np.float32))
+    v = synth.f32_to_bf16_bits(g.standard_normal((B, S_kv, H, 128)).astype(np.float32))
+    return q, k, v
+
+
+def _check_cross(q, k, v, out, lse, items, sm_scale, tag, precise):
+    """Each mode against its stated bound: the weights' rounding (2^-7 default, 2^-15
+    precise, times sum w |v|) plus the fp32 accumulation of S_kv products (S_kv 2^-24
+    sum w |v|), half an ulp for the output's rounding.  Rows over hundreds of random keys
+    are means of many terms of both signs: the accumulation error, relative to the small
+    result, moves more outputs across a bf16 midpoint than in the fine stage.  And the
+    card's cosine against FP64."""
+    o64, l64, wabs = oracle.cross_items(q, k, v, sm_scale, items, want_wabs=True)
+    rows = common.gather_items(out, items)
+    res = common.compare(rows, o64, items[:, 1] + 1000 * items[:, 0])
+    print(f"\n[{tag}] gate {res['gate']}\n[{tag}] vs fp64 {res['fp64']}")
+    weights = common.PRECISE_WEIGHT_BOUND if precise else common.DEFAULT_WEIGHT_BOUND
+    bnd = common.within_default_bound(rows, o64, wabs, coeff=weights + k.shape[1] * 2.0 ** -24)
+    print(f"[{tag}] bound {bnd}")
+    assert bnd["ok"], bnd
+    assert res["fp64"]["finite"] and res["fp64"]["min_head_cos"] >= 0.9999, res["fp64"]
+    got_lse = common.gather_lse(lse, items)
+    bound = common.lse_bound(q, k, items, sm_scale, default_mode=not precise)
+    assert np.all(np.abs(got_lse - l64) <= bound), float(np.max(np.abs(got_lse - l64)))
+
+
+@pytest.mark.parametrize("flags", [0, 1])
+@pytest.mark.parametrize("S_kv", [512, 77, 1, 1000])
+def test_cross_attn_every_row(vsa, S_kv, flags):
+    """Every query row over every key of a short sequence: Wan's 512 text tokens, a
+    ragged length (last cube partial), a single key, and 16 cubes (8 steps a tile)."""
+    B, nblk, H = 2, 9, 3
+    q, k, v = _cross_inputs(60 + S_kv, B, nblk, S_kv, H)
+    sm = 128 ** -0.5
+    out, lse = vsa.cross_attn(common.dev(q), common.dev(k), common.dev(v), sm, want_lse=True, flags=flags)
+    torch.cuda.synchronize()
+    _no_device_error(vsa)
+    _check_cross(q, k, v, out, lse, oracle.all_items(B, H, nblk), sm, f"cross/{S_kv}/{flags}", flags == 1)
+
+
+def test_cross_attn_over_its_own_sequence_is_the_dense_forward(vsa):
+    """K/V = the query sequence and every cube listed in order: the fine-stage forward's
+    step lists exactly, so bit-identical results."""
+    p = _small(61, nq=6, H=2, topk=6, vbs=[64] * 6)
+    p.idx = np.broadcast_to(np.arange(6, dtype=np.int32), p.idx.shape).copy()
+    q, k, v = common.dev(p.qt), common.dev(p.kt), common.dev(p.vt)
+    a, la = vsa.cross_attn(q, k, v, p.cfg.sm_scale, want_lse=True)
+    b, lb = vsa.fwd(q, k, v, torch.from_numpy(p.idx).cuda(), torch.from_numpy(p.vbs).cuda(), p.cfg.sm_scale,
+                    want_lse=True)
+    torch.cuda.synchronize()
+    _no_device_error(vsa)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16)) and torch.equal(la.view(torch.int32),
+                                                                                  lb.view(torch.int32))
+
+
+def test_cross_attn_wan_shape_sampled(vsa):
+    """Wan 832x480 queries (39936 tokens, 40 heads) over a 512-token text KV: sampled
+    query blocks of every head against the oracle."""
+    B, nblk, H, S_kv = 1, 624, 40, 512
+    q, k, v = _cross_inputs(62, B, nblk, S_kv, H)
+    sm = 128 ** -0.5
+    out, lse = vsa.cross_attn(common.dev(q), common.dev(k), common.dev(v), sm, want_lse=True)
+    torch.cuda.synchronize()
+    _no_device_error(vsa)
+    items = common.sample_items(B, H, nblk, 120, seed=63)
+    _check_cross(q, k, v, out, lse, items, sm, "cross/wan", False)
+
+
+@pytest.mark.parametrize("nq,topk", [(8, 8), (6, 5)])
+def test_fwd_four_step_tiles_many_per_cta(vsa, nq, topk):
+    """Tiles of exactly four steps (one more than the S buffers) and more tiles than SMs:
+    the epilogue hands the next tile's first step to its product only after taking that
+    step's offsets, so the softmax cannot lap the correction warps on the three-buffer
+    ring (which stalled this case until a bounded wait gave up).  Every row."""
+    p = _small(64, nq=nq, H=40, topk=topk, vbs=[64] * nq)
+    p.idx = np.sort(np.stack([np.stack([np.random.default_rng(65 + h).permutation(nq)[:topk] for _ in range(nq)])
+                              for h in range(40)])[None], axis=-1).astype(np.int32)
+    q, k, v = common.dev(p.qt), common.dev(p.kt), common.dev(p.vt)
+    out, lse = vsa.fwd(q, k, v, torch.from_numpy(p.idx).cuda(), torch.from_numpy(p.vbs).cuda(), p.cfg.sm_scale,
+                       want_lse=True)
+    torch.cuda.synchronize()
+    _no_device_error(vsa)
+    _check_items(p, out, lse, oracle.all_items(1, 40, nq), f"four-step/{nq}", rule=False)

@@ -768,11 +768,12 @@ def test_cross_closed_forms(oracle_lib):
     """q = 0: the mean of v and lse = log S_kv; one key: its value and its logit."""
     q, k, v = _cross_case(51, S_kv=77)
     items = oracle_lib.all_items(1, 2, 3)
-    out, lse = oracle_lib.cross_items(np.zeros_like(q), k, v, 0.3, items)
+    out, lse, wabs = oracle_lib.cross_items(np.zeros_like(q), k, v, 0.3, items, want_wabs=True)
     V = oracle_lib.bf16_to_f64(v)[0]
     for n, (b, h, i) in enumerate(items):
         assert np.allclose(out[n], np.broadcast_to(V[:, h].mean(axis=0), (64, 128)), rtol=0, atol=1e-13)
         assert np.allclose(lse[n], math.log(77), rtol=0, atol=1e-13)
+        assert np.allclose(wabs[n], np.broadcast_to(np.abs(V[:, h]).mean(axis=0), (64, 128)), rtol=0, atol=1e-13)
     q, k, v = _cross_case(52, S_kv=1)
     out, lse = oracle_lib.cross_items(q, k, v, 0.25, items)
     Q, K, V = (oracle_lib.bf16_to_f64(a)[0] for a in (q, k, v))

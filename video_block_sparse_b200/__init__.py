@@ -31,7 +31,7 @@ _STATUS = {0: "VSA_OK", -1: "VSA_ERR_ARG", -2: "VSA_ERR_NULL", -3: "VSA_ERR_ALIG
 
 # every symbol include/vsa.h declares
 EXPORTS = ("vsa_status_string", "vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_fwd_planned", "vsa_fwd_proxy",
-           "vsa_fwd_bsr", "vsa_fwd_bitmask",
+           "vsa_fwd_bsr", "vsa_fwd_bitmask", "vsa_cross_attn",
            "vsa_plan_workspace_size", "vsa_plan", "vsa_route_workspace_size", "vsa_route", "vsa_route_means",
            "vsa_route_noalloc", "vsa_cube_counts", "vsa_tile", "vsa_tile_qkv", "vsa_untile", "vsa_stall_check",
            "vsa_device_status")
@@ -68,11 +68,12 @@ def _load():
     lib.vsa_fwd_proxy.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.vsa_fwd_bsr.argtypes = [P, P, P, P, P, I, P, P, P, P, P, P, I, I, I, I, I, F, I, P]
     lib.vsa_fwd_bitmask.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, I, P]
+    lib.vsa_cross_attn.argtypes = [P, P, P, P, P, I, I, I, I, I, F, I, P]
     lib.vsa_route_means.argtypes = [P, P, P, I, I, I, I, I, P]
     lib.vsa_device_status.argtypes = [P, P]
     lib.vsa_stall_check.argtypes = [P, P]
     for name in ("vsa_can_implement", "vsa_fwd", "vsa_fwd_ex", "vsa_fwd_planned", "vsa_fwd_proxy", "vsa_fwd_bsr",
-                 "vsa_fwd_bitmask", "vsa_plan", "vsa_route",
+                 "vsa_fwd_bitmask", "vsa_cross_attn", "vsa_plan", "vsa_route",
                  "vsa_route_means", "vsa_route_noalloc", "vsa_cube_counts", "vsa_tile", "vsa_tile_qkv", "vsa_untile",
                  "vsa_device_status", "vsa_stall_check"):
         getattr(lib, name).restype = I
@@ -381,6 +382,28 @@ def fwd_bitmask(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask: torch.T
     _check(get_lib().vsa_fwd_bitmask(_ptr(q), _ptr(k), _ptr(v), _ptr(mask), _ptr(vbs), _ptr(kc), _ptr(vc),
                                      _ptr(plan), _ptr(out), _ptr(lse), B, S, H, D, nq, sc, int(flags),
                                      _stream(stream)), "vsa_fwd_bitmask")
+    return (out, lse) if (want_lse or lse is not None) else out
+
+
+def cross_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, sm_scale: float | None = None,
+               out: torch.Tensor | None = None, lse: torch.Tensor | None = None, want_lse: bool = False,
+               flags: int = FWD_DEFAULT, stream=None):
+    """vsa_cross_attn: every query row of q [B, S, H, D] (S a multiple of 64) over every
+    key of the short k, v [B, S_kv, H, D]; returns out (and lse [B, H, S])."""
+    B, S, H, D = q.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _bf16(t, n)
+    S_kv = k.shape[1]
+    if k.shape != (B, S_kv, H, D) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, S_kv, H, D]")
+    if sm_scale is None:
+        sm_scale = D ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, H, S, dtype=torch.float32, device=q.device)
+    _check(get_lib().vsa_cross_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, S, S_kv, H, D,
+                                    float(sm_scale), int(flags), _stream(stream)), "vsa_cross_attn")
     return (out, lse) if (want_lse or lse is not None) else out
 
 

@@ -140,8 +140,8 @@ int fwd_dispatch(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const 
     int* err;
     if ((rc = device_error_word(&err)) != VSA_OK) return rc;
     const bool precise = (flags & VSA_FWD_PRECISE_P) != 0;
-    return launch_status(
-        vsa::launch_fwd_pair(q, k, v, rt, vbs, plan, kc, vc, out, lse, B, S, H, Nq, sm_scale, precise, err, stream));
+    return launch_status(vsa::launch_fwd_pair(q, k, v, rt, vbs, plan, kc, vc, out, lse, B, S, H, Nq, S, Nq, sm_scale,
+                                              precise, err, stream));
 }
 
 vsa::Routes route_lists(const int32_t* topk_idx, int topk)
@@ -211,6 +211,27 @@ int vsa_fwd_bsr(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const i
     rt.kind = vsa::kRouteBsr;
     rt.nnz = nnz;
     return fwd_dispatch(q, k, v, rt, vbs, plan, kc, vc, out, lse, B, S, H, D, Nq, sm_scale, flags, stream);
+}
+
+int vsa_cross_attn(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, vsa_bf16* out, float* lse, int B, int S,
+                   int S_kv, int H, int D, float sm_scale, int flags, cudaStream_t stream)
+{
+    if (S < 64 || S % 64 != 0) return VSA_ERR_ARG;
+    int rc = check_bshd(B, S, H, D, S / 64);
+    if (rc != VSA_OK) return rc;
+    if ((flags & ~VSA_FWD_PRECISE_P) != 0 || !vsa::fwd_pair_supported(S / 64, 1)) return VSA_ERR_ARG;
+    if (S_kv < 1 || S_kv > 64 * 1024 || (int64_t)B * S_kv * H * D > (int64_t)INT32_MAX * 8) return VSA_ERR_ARG;
+    if (!q || !k || !v || !out) return VSA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (lse && !aligned16(lse)))
+        return VSA_ERR_ALIGN;
+    if ((rc = check_arch()) != VSA_OK) return rc;
+    int* err;
+    if ((rc = device_error_word(&err)) != VSA_OK) return rc;
+    vsa::Routes rt{};
+    rt.kind = vsa::kRouteAll;
+    const int nkv = (S_kv + 63) / 64;
+    return launch_status(vsa::launch_fwd_pair(q, k, v, rt, nullptr, nullptr, nullptr, nullptr, out, lse, B, S, H, S / 64,
+                                              S_kv, nkv, sm_scale, (flags & VSA_FWD_PRECISE_P) != 0, err, stream));
 }
 
 int vsa_fwd_bitmask(const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v, const uint32_t* mask,

@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmkc,
                     const __grid_constant__ CUtensorMap tmvc, const Routes rt,
                     const int32_t* __restrict__ vbs, const int32_t* __restrict__ plan, uint16_t* __restrict__ out,
-                    float* __restrict__ lse, int S, int H, int nq, int tiles_per_bh, int n_tiles,
+                    float* __restrict__ lse, int S, int H, int nq, int S_kv, int nkv, int tiles_per_bh, int n_tiles,
                     float scale_log2, int* err)
 {
     using L = Layout;
@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         m.end_g = 0x7fffffff;
         fence_mbar_init();
     }
-    vbs_stage(vbs, nq, m.vbs8, err);
+    vbs_stage(vbs, nkv, S_kv, m.vbs8, err);
     if (warp == kWarpMma) {
         tmem_alloc(&m.tmem_base, 512);
         tmem_relinquish();
@@ -263,14 +263,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const TileRef t = t_next;
             int32_t* l1 = m.list1[n & 1];
             int32_t* l2 = m.list2[n & 1];
-            const int n_ent = rt.kind == kRouteMask ? steps_build_mask(t, nq, l1, l2, m.bits1, m.bits2, err, lane)
-                                                    : steps_build(t, nq, l1, l2, m.bits1, m.bits2, err, lane);
+            const int n_ent = rt.kind == kRouteMask  ? steps_build_mask(t, nkv, l1, l2, m.bits1, m.bits2, err, lane)
+                              : rt.kind == kRouteAll ? steps_build_all(t, nkv, l1, lane)
+                                                     : steps_build(t, nkv, l1, l2, m.bits1, m.bits2, err, lane);
             const uint16_t* ent = reinterpret_cast<const uint16_t*>(l1);  // written over list 1
-            const int tok0 = t.b * S;
+            const int tok0 = t.b * S;        // the tile's query tokens
+            const int tok0kv = t.b * S_kv;   // its key / value tokens
             // proxy mode: after the selected cubes, ceil(nq / 128) steps over the proxy keys
             // (cube j's mean key and summed value), 128 cubes per step; a tile without
             // entries then has no plain step (else it takes one empty step)
-            const int n_proxy = PROXY ? (nq + 127) / 128 : 0;
+            const int n_proxy = PROXY ? (nkv + 127) / 128 : 0;
             const int n_plain = PROXY ? (n_ent + 1) / 2 : max(1, (n_ent + 1) / 2);
             const int n_steps = n_plain + n_proxy;
             // Step s of the tile: its K pair (rows ka, kb of head kh of map kmap; -1: none),
@@ -355,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool last = s + 1 == n_steps;
                 meta.flags = (s == 0 ? 1 : 0) | (last ? 2 : 0);
                 const uint32_t word = step_word(meta) | (last && n == my_tiles - 1 ? kFinal : 0u);
-                issue(s, &tmk, t.h, meta.na > 0 ? tok0 + 64 * ja : -1, meta.nb > 0 ? tok0 + 64 * jb : -1, t.h, word,
+                issue(s, &tmk, t.h, meta.na > 0 ? tok0kv + 64 * ja : -1, meta.nb > 0 ? tok0kv + 64 * jb : -1, t.h, word,
                       nullptr, 0);
             }
             if constexpr (PROXY) {
@@ -366,18 +368,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int pc = 0; pc < n_proxy && !aborted; ++pc) {
                     const int s = n_plain + pc, pbase = 128 * pc;
                     StepMeta meta;
-                    meta.na = min(64, nq - pbase);
-                    meta.nb = min(64, max(0, nq - pbase - 64));
+                    meta.na = min(64, nkv - pbase);
+                    meta.nb = min(64, max(0, nkv - pbase - 64));
                     meta.ma = cubes_here;
                     meta.mb = meta.nb > 0 ? cubes_here : 0;
                     uint32_t pm = 0;  // lane w < 8: mask word w, [cube][key half][32-key word]
 #pragma unroll
                     for (int w = 0; w < 4; ++w) {
                         const int j = pbase + 32 * w + (int)lane;
-                        const int nj = j < nq ? (int)m.vbs8[j] : 0;
+                        const int nj = j < nkv ? (int)m.vbs8[j] : 0;
                         const uint32_t valid = __ballot_sync(0xffffffffu, nj >= 1 && nj <= 64);
                         const int word = (pbase >> 5) + w;
-                        const bool in_range = pbase + 32 * w < nq;
+                        const bool in_range = pbase + 32 * w < nkv;
                         const uint32_t m1 = t.i1 >= 0 && in_range ? valid & ~m.bits1[word] : 0u;
                         const uint32_t m2 = t.i2 >= 0 && in_range ? valid & ~m.bits2[word] : 0u;
                         if ((int)lane == w) pm = m1;
@@ -390,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     meta.flags = (s == 0 ? 1 : 0) | (last ? 2 : 0);
                     const uint32_t word =
                         step_word(meta) | (last && n == my_tiles - 1 ? kFinal : 0u) | kProxyStep;
-                    const int row = (t.b * H + t.h) * nq + pbase;
+                    const int row = (t.b * H + t.h) * nkv + pbase;
                     issue(s, &tmkc, 0, row, meta.nb > 0 ? row + 64 : -1, 0, word, pmw, pbase);
                 }
             }
@@ -555,10 +557,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int qbit = r >> 6;
         const uint32_t oa = tbase + ((uint32_t)(32 * wq) << 16) + kOCol;
         int g = 0;
-        bool released = false;  // this tile's first step was released by the previous tile's epilogue
+        bool released = false;    // this tile's first step was handled by the previous tile's epilogue
+        uint32_t released_meta = 0;  // and this was its step word
         for (int n = 0; n < my_tiles; ++n) {
             for (;;) {
                 const int b = g % kSBuf;
+                if (released) {  // a first step: no rescale, its arrival made already
+                    released = false;
+                    ++g;
+                    if (sw_flags(released_meta) & 2) break;
+                    continue;
+                }
                 if (!wait_warp(&bb.a_full[b], (g / kSBuf) & 1, &m.abort, err)) goto corr_exit;
                 const uint32_t meta = m.s_meta[b];
                 const int rescale = __shfl_sync(0xffffffffu, !(sw_flags(meta) & 1) && m.rflag[b][wq] != 0, 0);
@@ -580,11 +589,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tmem_st_wait();
                 }
-                if (!released) {
-                    tc_fence_before();
-                    mbar_arrive(&bb.p_full[b]);
-                }
-                released = false;
+                tc_fence_before();
+                mbar_arrive(&bb.p_full[b]);
                 ++g;
                 if (sw_flags(meta) & 2) break;
             }
@@ -603,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float inv = has ? __frcp_rn(l) : 0.f;
                 const int64_t token = (int64_t)t.b * S + 64LL * cube + (r & 63);
                 uint16_t* dst = out + (token * H + t.h) * kD;
-                // read and round the whole row first ...
+                // read and round the whole row
                 uint32_t pk[4][16];
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
@@ -614,14 +620,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int e = 0; e < 16; ++e)
                         pk[c4][e] = has ? pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv)
                                         : 0u;
-                }
-                // ... so that the next tile's first product, which overwrites O, need not
-                // wait for the stores.  Every product of this tile has completed (o_full),
-                // so this arrival can only count toward the next step's phase.
-                if (n + 1 < my_tiles) {
-                    tc_fence_before();
-                    mbar_arrive(&bb.p_full[g % kSBuf]);
-                    released = true;
                 }
                 if (cube >= 0) {
 #pragma unroll
@@ -634,6 +632,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lse != nullptr && cube >= 0)
                     lse[((int64_t)t.b * H + t.h) * S + 64LL * cube + (r & 63)] =
                         has ? (m_row + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+                // The next tile's first step (a first step, which never rescales) is handled
+                // here, so that its product, which overwrites O (read above), need not wait
+                // for this warp's next pass.  Every product of this tile has completed
+                // (o_full), so the arrival can only count toward that step's phase.  Its
+                // offsets are waited for first: until this arrival no product of that step
+                // can be issued, so no later step can complete a_full of its buffer again
+                // before this wait (a release ahead of the wait let the softmax lap this warp
+                // on that ring when tiles are four steps long).
+                if (n + 1 < my_tiles) {
+                    const int b1 = g % kSBuf;
+                    if (!wait_warp(&bb.a_full[b1], (g / kSBuf) & 1, &m.abort, err)) goto corr_exit;
+                    released_meta = __shfl_sync(0xffffffffu, m.s_meta[b1], 0);
+                    tc_fence_before();
+                    mbar_arrive(&bb.p_full[b1]);
+                    released = true;
+                }
             }
             tc_fence_before();
         }
@@ -872,7 +886,8 @@ struct FwdMaps {
 
 template <bool NEG, bool PRECISE, bool PROXY>
 cudaError_t launch(const FwdMaps& mp, const Routes& rt, const int32_t* vbs, const int32_t* plan, uint16_t* out,
-                   float* lse, int B, int S, int H, int nq, float scale_log2, int* err, cudaStream_t s)
+                   float* lse, int B, int S, int H, int nq, int S_kv, int nkv, float scale_log2, int* err,
+                   cudaStream_t s)
 {
     auto kern = fwd_pair_kernel<NEG, PRECISE, PROXY>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Layout::SMEM_BYTES);
@@ -884,7 +899,7 @@ cudaError_t launch(const FwdMaps& mp, const Routes& rt, const int32_t* vbs, cons
     const int n_tiles = B * H * tiles_per_bh;
     const int grid = n_tiles < sms ? n_tiles : sms;
     kern<<<grid, kThreads, Layout::SMEM_BYTES, s>>>(mp.q, mp.k, mp.v, mp.kc, mp.vc, rt, vbs, plan, out, lse,
-                                                    S, H, nq, tiles_per_bh, n_tiles, scale_log2, err);
+                                                    S, H, nq, S_kv, nkv, tiles_per_bh, n_tiles, scale_log2, err);
     return cudaGetLastError();
 }
 
@@ -894,16 +909,16 @@ bool fwd_pair_supported(int nq, int topk) { return nq <= kMaxNq && topk <= kMaxT
 
 cudaError_t launch_fwd_pair(const uint16_t* q, const uint16_t* k, const uint16_t* v, const Routes& rt,
                             const int32_t* vbs, const int32_t* plan, const uint16_t* kc, const uint16_t* vc,
-                            uint16_t* out, float* lse, int B, int S, int H, int nq, float sm_scale, bool precise_p,
-                            int* err, cudaStream_t s)
+                            uint16_t* out, float* lse, int B, int S, int H, int nq, int S_kv, int nkv, float sm_scale,
+                            bool precise_p, int* err, cudaStream_t s)
 {
     FwdMaps mp;
-    const int64_t tokens = (int64_t)B * S;
-    if (!make_map(&mp.q, q, tokens, H) || !make_map(&mp.k, k, tokens, H) || !make_map(&mp.v, v, tokens, H))
+    const int64_t tokens = (int64_t)B * S, kv_tokens = (int64_t)B * S_kv;
+    if (!make_map(&mp.q, q, tokens, H) || !make_map(&mp.k, k, kv_tokens, H) || !make_map(&mp.v, v, kv_tokens, H))
         return cudaErrorInvalidValue;
     const bool proxy = kc != nullptr && vc != nullptr;
     if (proxy) {
-        const int64_t rows = (int64_t)B * H * nq;
+        const int64_t rows = (int64_t)B * H * nkv;
         if (!make_map(&mp.kc, kc, rows, 1) || !make_map(&mp.vc, vc, rows, 1)) return cudaErrorInvalidValue;
     } else {
         mp.kc = mp.k;  // not read
@@ -912,12 +927,12 @@ cudaError_t launch_fwd_pair(const uint16_t* q, const uint16_t* k, const uint16_t
     const float scale_log2 = sm_scale * 1.4426950408889634f;
     // one kernel per (sign of the scale, weight precision, proxy steps)
     using Launch = cudaError_t (*)(const FwdMaps&, const Routes&, const int32_t*, const int32_t*, uint16_t*, float*, int,
-                                   int, int, int, float, int*, cudaStream_t);
+                                   int, int, int, int, int, float, int*, cudaStream_t);
     static constexpr Launch table[8] = {
         launch<false, false, false>, launch<true, false, false>, launch<false, true, false>, launch<true, true, false>,
         launch<false, false, true>,  launch<true, false, true>,  launch<false, true, true>,  launch<true, true, true>};
     const int which = (scale_log2 < 0.f ? 1 : 0) | (precise_p ? 2 : 0) | (proxy ? 4 : 0);
-    return table[which](mp, rt, vbs, plan, out, lse, B, S, H, nq, scale_log2, err, s);
+    return table[which](mp, rt, vbs, plan, out, lse, B, S, H, nq, S_kv, nkv, scale_log2, err, s);
 }
 
 }  // namespace vsa

@@ -350,12 +350,14 @@ __device__ __forceinline__ TileRef tile_ref(int t, int H, int nq, int tiles_per_
 // a step is empty.
 __device__ __forceinline__ bool test_bit(const uint32_t* bits, int j) { return (bits[j >> 5] >> (j & 31)) & 1u; }
 
-// The valid counts as bytes in shared memory; a count outside [0, 64] latches
-// an error and is kept as 255, which the kernel treats as an empty cube.
-__device__ __forceinline__ void vbs_stage(const int32_t* __restrict__ vbs, int nq, uint8_t* vbs8, int* err)
+// The valid counts of the nkv KV cubes as bytes in shared memory; a count
+// outside [0, 64] latches an error and is kept as 255, which the kernel treats
+// as an empty cube.  vbs NULL: every cube full but the last, which holds the
+// S_kv - 64 (nkv - 1) tokens left.
+__device__ __forceinline__ void vbs_stage(const int32_t* __restrict__ vbs, int nkv, int S_kv, uint8_t* vbs8, int* err)
 {
-    for (int c = threadIdx.x; c < nq; c += blockDim.x) {
-        const int n = __ldg(vbs + c);
+    for (int c = threadIdx.x; c < nkv; c += blockDim.x) {
+        const int n = vbs != nullptr ? __ldg(vbs + c) : min(64, S_kv - 64 * c);
         const bool bad = n < 0 || n > 64;
         if (bad) atomicCAS(err, 0, (int)kErrVbs);
         vbs8[c] = (uint8_t)(bad ? 255 : n);
@@ -386,6 +388,9 @@ __device__ __forceinline__ void lists_fetch(TileRef& t, const Routes& rt, int H,
             } else if (rt.kind == kRouteMask) {
                 len = rt.words;
                 src = reinterpret_cast<const int32_t*>(rt.mask + r * rt.words);
+            } else if (rt.kind == kRouteAll) {
+                len = 0;  // nothing to copy: every KV cube
+                src = nullptr;
             } else {
                 len = rt.topk;
                 src = rt.idx + r * rt.topk;
@@ -573,6 +578,19 @@ __device__ int steps_build_mask(const TileRef& t, int nq, int32_t* l1, int32_t* 
     }
     __syncwarp();
     return count;
+}
+
+// The step list of a tile that attends to every one of the nkv KV cubes (both
+// query cubes, cube order).
+__device__ int steps_build_all(const TileRef& t, int nkv, int32_t* l1, uint32_t lane)
+{
+    cp_async_wait_all();
+    __syncwarp();
+    const uint32_t mem = (t.i1 >= 0 ? 1u : 0u) | (t.i2 >= 0 ? 2u : 0u);
+    uint16_t* ent = reinterpret_cast<uint16_t*>(l1);
+    for (int j = (int)lane; j < nkv; j += 32) ent[j] = (uint16_t)((uint32_t)j | (mem << 14));
+    __syncwarp();
+    return nkv;
 }
 
 // A tile with an out-of-range plan entry latches an error; the bad cube is dropped.

@@ -59,7 +59,7 @@ bool fwd_pair_supported(int nq, int topk);
 // lists (topk_idx [B, H, Nq, topk]), BSR rows (indices[indptr[r] .. indptr[r+1]), nnz
 // entries in all), or packed UInt32 bitmaps ([B, H, Nq, words], bit c % 32 of word c / 32
 // selects cube c).
-enum RouteKind : int { kRouteLists = 0, kRouteBsr = 1, kRouteMask = 2 };
+enum RouteKind : int { kRouteLists = 0, kRouteBsr = 1, kRouteMask = 2, kRouteAll = 3 };  // all: every KV cube
 struct Routes {
     const int32_t* idx;     // lists: topk_idx; BSR: indices
     const int32_t* indptr;  // BSR: [B*H*Nq + 1]
@@ -71,10 +71,12 @@ struct Routes {
 };
 
 // kc, vc: the proxies' mean keys and summed values [B, H, Nq, 128] (both NULL: no proxies)
+// S_kv, nkv: the key/value sequence's tokens and cubes (the query sequence's for the fine
+// stage); vbs NULL: every KV cube full but the last, which holds S_kv - 64 (nkv - 1) tokens
 cudaError_t launch_fwd_pair(const uint16_t* q, const uint16_t* k, const uint16_t* v, const Routes& rt,
                             const int32_t* vbs, const int32_t* plan, const uint16_t* kc, const uint16_t* vc,
-                            uint16_t* out, float* lse, int B, int S, int H, int nq, float sm_scale, bool precise_p,
-                            int* err, cudaStream_t s);
+                            uint16_t* out, float* lse, int B, int S, int H, int nq, int S_kv, int nkv, float sm_scale,
+                            bool precise_p, int* err, cudaStream_t s);
 
 // ---- plan.cu (pairing of query cubes by selection overlap)
 size_t plan_workspace_bytes(int B, int H, int nq);
