@@ -294,6 +294,15 @@ def run_gpu(args, rank, world, local_rank):
 
 # --------------------------------------------------------------------------- extras
 
+def lists_to_bitmask(idx: torch.Tensor) -> torch.Tensor:
+    """[B, H, Nq, topk] lists of distinct cubes -> [B, H, Nq, ceil(Nq/32)] packed bitmaps
+    (bit c % 32 of word c / 32 selects cube c), as int32 words."""
+    B, H, nq, _ = idx.shape
+    bits = torch.zeros(B, H, nq, (nq + 31) // 32, dtype=torch.int64, device=idx.device)
+    bits.scatter_add_(3, (idx // 32).long(), torch.ones_like(idx, dtype=torch.int64) << (idx % 32).long())
+    return torch.where(bits >= 2 ** 31, bits - 2 ** 32, bits).to(torch.int32).contiguous()
+
+
 def steps_per_tile(idx: np.ndarray, plan: np.ndarray | None, vbs: np.ndarray) -> np.ndarray:
     """Steps each tile of the paired forward walks: the distinct cubes with a valid
     token that either list names (every entry when a list repeats a cube), two per step.
@@ -384,10 +393,7 @@ def run_extras(vsa, dev, cfg, qt, kt, vt, qc, kc, idx, vbs, peak):
     B, H, nq, topk = ix_sorted.shape
     indptr = (torch.arange(B * H * nq + 1, device=dev, dtype=torch.int32) * topk).contiguous()
     indices = ix_sorted.reshape(-1).contiguous()
-    W = (nq + 31) // 32
-    bits = torch.zeros(B, H, nq, W, dtype=torch.int64, device=dev)
-    bits.scatter_add_(3, (ix_sorted // 32).long(), torch.ones_like(ix_sorted, dtype=torch.int64) << (ix_sorted % 32).long())
-    mask = torch.where(bits >= 2 ** 31, bits - 2 ** 32, bits).to(torch.int32).contiguous()
+    mask = lists_to_bitmask(ix_sorted)
     pl_s = vsa.plan(ix_sorted)
     fmt = {"fwd_lists_ms": fwd_case(qt, kt, vt, ix_sorted, vbs, cfg, pl_s)}
     fmt["fwd_bsr_ms"] = time_fwd(vsa, ((qt, kt, vt, indptr, indices, vbs, cfg.sm_scale), {"out": out, "plan": pl_s}),
@@ -398,7 +404,7 @@ def run_extras(vsa, dev, cfg, qt, kt, vt, qc, kc, idx, vbs, peak):
         vsa, ((qt, kt, vt, mask, vbs, cfg.sm_scale), {"out": out, "plan": pl_s, "kc": kc, "vc": vc}),
         fn=vsa.fwd_bitmask)
     res["route_formats"] = fmt
-    del vc, mask, bits, indices
+    del vc, mask, indices
 
     # short-KV cross-attention: the step's queries over a 512-token text key/value
     # sequence (seeded draws), every key attended

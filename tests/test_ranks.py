@@ -70,3 +70,19 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--gpus", "2", "--steps", "1"])
     bench.main()
     assert capsys.readouterr().out == ""
+
+
+def test_bench_bitmaps_are_the_oracle_format():
+    """The bench's bitmap input (the routed lists as packed words) is the format the
+    oracle defines: the same words as the lists' BSR rows written out as bitmaps."""
+    import numpy as np
+
+    import bench
+    import oracle
+    import synth
+
+    for nq in (37, 64, 624):
+        idx = np.sort(synth.random_topk(nq, 1, 2, nq, 9), axis=-1).astype(np.int32)
+        got = bench.lists_to_bitmask(torch.from_numpy(idx)).numpy().view(np.uint32)
+        want = oracle.bsr_to_bitmask(*oracle.lists_to_bsr(idx), 1, 2, nq)
+        assert np.array_equal(got, want)
