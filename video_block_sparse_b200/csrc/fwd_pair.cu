@@ -159,8 +159,9 @@ struct Flag {
 };
 
 // PROXY: the kernel runs the proxy steps after each tile's selected cubes.  It is a
-// template parameter so that the plain kernels hold none of that code: the extra
-// instructions cost the plain forward ~25% through instruction fetches alone.
+// template parameter so that the plain kernels hold none of that code: as a run-time
+// flag it cost the plain forward 25-40 % (its branches and instructions sat in the
+// producer's and the softmax's per-step paths, whose issue slots the softmax needs).
 template <bool NEG, bool PRECISE, bool PROXY>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
