@@ -204,3 +204,23 @@ def test_product_package_does_not_reach_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "liboracle" not in text and "from oracle" not in text, f
+
+
+def test_binding_checks_route_format_and_cross_arguments_on_the_host(vsa):
+    """The Python wrappers of the route-format and cross-attention entry points reject
+    mismatched tensors before any device call."""
+    import torch
+
+    bf = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)  # noqa: E731
+    q = bf(1, 128, 2, 128)
+    vbs = torch.zeros(2, dtype=torch.int32)
+    with pytest.raises(ValueError):  # indptr must hold B*H*Nq + 1 entries
+        vsa.fwd_bsr(q, q, q, torch.zeros(4, dtype=torch.int32), torch.zeros(0, dtype=torch.int32), vbs)
+    with pytest.raises(ValueError):  # int32 only
+        vsa.fwd_bsr(q, q, q, torch.zeros(5, dtype=torch.int64), torch.zeros(0, dtype=torch.int32), vbs)
+    with pytest.raises(ValueError):  # kc without vc
+        vsa.fwd_bitmask(q, q, q, torch.zeros(1, 2, 2, 1, dtype=torch.int32), vbs, kc=bf(1, 2, 2, 128))
+    with pytest.raises(ValueError):  # bitmap shape
+        vsa.fwd_bitmask(q, q, q, torch.zeros(1, 2, 2, 2, dtype=torch.int32), vbs)
+    with pytest.raises(ValueError):  # k and v of different lengths
+        vsa.cross_attn(q, bf(1, 64, 2, 128), bf(1, 32, 2, 128))
